@@ -1,0 +1,183 @@
+/*
+ * moe.h — C ABI of the routed, weight-quantized Mixture-of-Experts layer for NVIDIA B200
+ * (sm_100a): softmax top-k router, token-to-expert alignment, W4A16 and block-FP8 grouped
+ * expert GEMMs with a fused SiLU*up epilogue, and a deterministic weighted combine.
+ *
+ * Where the operations are defined (titles of the pages that describe the method):
+ *  - "AWS Details H200 Kernel Optimizations for MoE Inference", section "Three bottlenecks
+ *    require different fixes": a fused MoE operator combines token routing, data movement
+ *    and expert calculations (moe_route, moe_align, moe_w4a16_forward).
+ *  - "Chord Rewrites the INT4 MoE Kernel for Kimi K2.x ...", second paragraph: W4A16 =
+ *    BF16 inputs, INT4 weights dequantized with one BF16 scale per group of 32 weights, gate /
+ *    up / down projections, scheduling from each expert's actual token count
+ *    (moe_w4a16_forward, moe_w4a16_gemm).
+ *  - "Helion Brings Autotuned GEMM Kernels to vLLM ...", section "Scope: Hopper and
+ *    quantized formats": Block_FP8 = FP8 with 1x128 activation scaling and 128x128 weight
+ *    scaling (moe_blockfp8_forward).
+ *  The router (softmax, top-k, renormalised weights), SiLU*up activation and top-k-weighted
+ *  combine are not written out on those pages; this library takes the textbook readings
+ *  stated with each call below.
+ *
+ * Conventions for every call:
+ *  - All tensor pointers are DEVICE pointers owned by the caller, row-major, 16-byte aligned.
+ *    The library never allocates, frees or synchronises inside these calls; all scratch
+ *    memory is the caller's workspace (size from the matching *_workspace_size call).
+ *  - Work is enqueued on `stream` and returns immediately; no host reads of device data, so
+ *    the calls may be captured in a CUDA graph.
+ *  - Argument, shape and alignment errors return an error code synchronously with nothing
+ *    enqueued.  A failed kernel launch returns MOE_ERR_CUDA.
+ *  - Faults the GPU detects (an expert id outside [0,E), a wait that timed out) are recorded
+ *    in a per-device status word that moe_get_device_status() reads.
+ *  - There is no CPU fallback: without a usable sm_100 GPU the calls return MOE_ERR_CUDA or
+ *    MOE_ERR_UNSUPPORTED.
+ *  - Shape limits: 1 <= k <= E <= 1024, T >= 1, H and I multiples of 128, T*k < 2^31.
+ */
+#ifndef MOE_H_
+#define MOE_H_
+
+#include <stddef.h>
+#include <stdint.h>
+#include <cuda_runtime_api.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  MOE_OK = 0,
+  MOE_ERR_INVALID_ARG = 1,  /* null / misaligned pointer, bad size */
+  MOE_ERR_UNSUPPORTED = 2,  /* shape outside the limits above, or no sm_100 device */
+  MOE_ERR_WORKSPACE = 3,    /* workspace smaller than the *_workspace_size value */
+  MOE_ERR_CUDA = 4,         /* a CUDA runtime / driver call failed */
+  MOE_ERR_TIMEOUT = 5,      /* (device status) a bounded in-kernel wait gave up */
+  MOE_ERR_DEVICE_CHECK = 6  /* (device status) an input failed a device-side check */
+} moe_status_t;
+
+/* Human-readable name of a status code (static string). */
+const char* moe_status_string(moe_status_t s);
+
+/* ------------------------------------------------------------------ a1: router
+ * Per token t: the k experts with the largest logits, ordered by (logit descending, expert
+ * index ascending); slot s holds the s-th.  Weights are the softmax of the logits over all
+ * E experts restricted to the winners, renormalised to sum to 1 when `renormalize` != 0 (then
+ * w_s = exp(l_s - l_max) / sum_{s'} exp(l_s' - l_max)), otherwise the plain softmax
+ * probabilities.  Logits must be finite.
+ *   logits   fp32  [T, E]   (in)
+ *   topk_ids int32 [T, k]   (out)
+ *   topk_w   fp32  [T, k]   (out)
+ * One warp per token; no workspace. */
+moe_status_t moe_route(const float* logits, int T, int E, int k, int renormalize, int32_t* topk_ids,
+                       float* topk_w, cudaStream_t stream);
+
+/* ------------------------------------------------------------------ a2: alignment
+ * Stable counting sort of the T*k (token, slot) pairs by expert.  Pair p = t*k + s.
+ *   expert_counts  int32 [E]     pairs routed to each expert
+ *   expert_offsets int32 [E+1]   offsets[0] = 0, offsets[e+1] = offsets[e] +
+ *                                ceil(counts[e]/align)*align
+ *   sorted_ids     int32 [moe_align_capacity()]  sorted_ids[offsets[e] + r] = r-th pair of
+ *                  expert e in ascending p; the padding of each expert's run holds the
+ *                  sentinel T*k; entries at and beyond offsets[E] are left untouched
+ *   inv_pos        int32 [T*k]   row of pair p in sorted_ids (-1 for a pair whose id is out of
+ *                  range; such pairs are skipped and MOE_ERR_DEVICE_CHECK is recorded)
+ * align >= 1.  ws: moe_align_workspace_size(T, k, E) bytes. */
+size_t moe_align_capacity(int T, int k, int E, int align); /* T*k + E*(align-1) entries */
+size_t moe_align_workspace_size(int T, int k, int E);
+moe_status_t moe_align(const int32_t* topk_ids, int T, int k, int E, int align, int32_t* expert_counts,
+                       int32_t* expert_offsets, int32_t* sorted_ids, int32_t* inv_pos, void* ws, size_t ws_bytes,
+                       cudaStream_t stream);
+
+/* ------------------------------------------------------------------ a2..a8: W4A16 layer
+ * out[t] = sum_{s<k} topk_w[t,s] * y_{t,s},   y = h . W2[e]^T,   h_j = SiLU(g_j) * g_{I+j},
+ * g = x[t] . W13[e]^T,   e = topk_ids[t,s],   SiLU(v) = v / (1 + e^-v),
+ * with dequantized weights W[n][c] = int4(q) * bf16(scale of (n, c/32)).
+ *   x      bf16  [T, H]
+ *   w13_q  int32 [E, 2I, H/8]  rows 0..I-1 = gate, I..2I-1 = up; word c/8 of row n holds K
+ *                              indices 8*(c/8)..+7, nibble j (bits 4j..4j+3) = index 8w+j,
+ *                              two's complement in [-8, 7]
+ *   w13_s  bf16  [E, 2I, H/32] one scale per 32 K elements per output row
+ *   w2_q   int32 [E, H, I/8],  w2_s bf16 [E, H, I/32]   (down projection, same packing)
+ *   out    bf16  [T, H] (RNE of the fp32 result), or fp32 [T, H] when out_fp32 != 0
+ * Numerics: activations and dequantized weights are fed to the tensor cores in fp16, which
+ * is exact for bf16 x inside the fp16 normal range and for |q*s| inside it (scales in
+ * [2^-14/8... , 65504/8]); accumulation is fp32; h is rounded to fp16; the combine sums the
+ * k slots in fp32 in slot order, so the result is deterministic run to run.
+ * ws: moe_w4a16_workspace_size(T, H, I, E, k) bytes. */
+typedef struct {
+  const void* x;
+  const int32_t* topk_ids;
+  const float* topk_w;
+  const int32_t* w13_q;
+  const void* w13_s;
+  const int32_t* w2_q;
+  const void* w2_s;
+  int T, H, I, E, k;
+  void* out;
+  int out_fp32;
+} moe_w4a16_args;
+
+size_t moe_w4a16_workspace_size(int T, int H, int I, int E, int k);
+moe_status_t moe_w4a16_forward(const moe_w4a16_args* args, void* ws, size_t ws_bytes, cudaStream_t stream);
+
+/* ------------------------------------------------------------------ a9: block-FP8 layer
+ * Same layer with e4m3 (OCP E4M3FN) operands:
+ *   x      e4m3 [T, H] with fp32 scales xs [T, H/128]        (x = q * xs[t][c/128])
+ *   w13    e4m3 [E, 2I, H] with fp32 scales [E, 2I/128, H/128] (W = q * s[n/128][c/128])
+ *   w2     e4m3 [E, H, I]  with fp32 scales [E, H/128, I/128]
+ * The intermediate h = SiLU(gate) * up (fp32) is requantized per (pair, 128-column group):
+ * s = max(amax, 1e-10) / 448, q = e4m3_rne_satfinite(h / s), before the down projection.
+ * out bf16 [T, H] or fp32 when out_fp32 != 0.
+ * ws: moe_blockfp8_workspace_size(T, H, I, E, k) bytes. */
+typedef struct {
+  const uint8_t* x;
+  const float* xs;
+  const int32_t* topk_ids;
+  const float* topk_w;
+  const uint8_t* w13;
+  const float* w13_s;
+  const uint8_t* w2;
+  const float* w2_s;
+  int T, H, I, E, k;
+  void* out;
+  int out_fp32;
+} moe_blockfp8_args;
+
+size_t moe_blockfp8_workspace_size(int T, int H, int I, int E, int k);
+moe_status_t moe_blockfp8_forward(const moe_blockfp8_args* args, void* ws, size_t ws_bytes, cudaStream_t stream);
+
+/* ------------------------------------------------------------------ grouped W4A16 GEMM
+ * No activation: rows [expert_offsets[e], expert_offsets[e+1]) of a are multiplied by
+ * expert e's dequantized weights:  out[m][n] = sum_c a[m][c] * W[e][n][c].
+ *   a              bf16 (a_is_bf16 != 0) or fp16 [M, K]
+ *   w_q            int32 [E, N, K/8], w_s bf16 [E, N, K/32] (packing as in moe_w4a16_forward)
+ *   expert_offsets int32 [E+1] (device), non-decreasing, offsets[0] >= 0, offsets[E] <= M;
+ *                  rows outside every range are not written
+ *   out            bf16 or fp32 (out_fp32 != 0) [M, N]
+ * K and N multiples of 128.  ws: moe_w4a16_gemm_workspace_size(M, K, N, E) bytes. */
+size_t moe_w4a16_gemm_workspace_size(int M, int K, int N, int E);
+moe_status_t moe_w4a16_gemm(const void* a, int a_is_bf16, const int32_t* w_q, const void* w_s,
+                            const int32_t* expert_offsets, int M, int K, int N, int E, void* out, int out_fp32,
+                            void* ws, size_t ws_bytes, cudaStream_t stream);
+
+/* ------------------------------------------------------------------ status, diagnostics
+ * moe_get_device_status: synchronises `stream`, returns the device status word of the
+ * current device (MOE_OK if no kernel recorded a fault) and clears it. */
+moe_status_t moe_get_device_status(cudaStream_t stream);
+
+/* Test hook: launches one CTA that waits on an mbarrier nothing will ever arrive on, with a
+ * bound of `limit_ns` nanoseconds (1 <= limit_ns <= 10^9).  The wait gives up, the kernel
+ * records MOE_ERR_TIMEOUT in the status word and returns normally. */
+moe_status_t moe_debug_wait_timeout(int64_t limit_ns, cudaStream_t stream);
+
+/* Per-kernel timing for benchmarks: while enabled, every kernel launch of this library is
+ * bracketed by a pair of CUDA events on its stream.  moe_timing_read synchronises the
+ * device, writes for up to `max` kernel names the summed milliseconds and launch counts
+ * since the last read (names are static strings), returns how many kernel names there are,
+ * and resets the sums.  Not thread-safe; keep disabled outside benchmarks. */
+moe_status_t moe_timing_enable(int enable);
+int moe_timing_read(const char** names, double* ms, int* launches, int max);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* MOE_H_ */

@@ -1,0 +1,375 @@
+// The C ABI (include/moe.h): argument checks, workspace carving, tensor-map encoding,
+// launch sequencing, the device status word and the benchmark timing hooks.
+#include <cuda.h>
+#include <cudaTypedefs.h>
+
+#include <algorithm>
+#include <cstring>
+#include <mutex>
+#include <vector>
+
+#include "common.cuh"
+#include "internal.h"
+
+namespace moe {
+
+
+// ------------------------------------------------------------------ device facts
+namespace {
+constexpr int kMaxDevices = 64;
+int g_sm_count[kMaxDevices];
+int g_cc_major[kMaxDevices];
+std::mutex g_mu;
+
+int current_device() {
+  int d = 0;
+  if (cudaGetDevice(&d) != cudaSuccess) return -1;
+  return d;
+}
+bool device_facts(int d) {
+  if (d < 0 || d >= kMaxDevices) return false;
+  std::lock_guard<std::mutex> lk(g_mu);
+  if (g_sm_count[d] > 0) return true;
+  int sms = 0, major = 0;
+  if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, d) != cudaSuccess) return false;
+  if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, d) != cudaSuccess) return false;
+  g_cc_major[d] = major;
+  g_sm_count[d] = sms;
+  return true;
+}
+
+// sm_100 family only: the kernels are built for sm_100a
+moe_status_t check_device() {
+  const int d = current_device();
+  if (!device_facts(d)) return MOE_ERR_CUDA;
+  return g_cc_major[d] == 10 ? MOE_OK : MOE_ERR_UNSUPPORTED;
+}
+
+bool aligned(const void* p, size_t a) { return p != nullptr && (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+// Sub-allocates a caller workspace; with a null base it only measures.
+struct Carver {
+  uint8_t* base;
+  size_t off = 0;
+  explicit Carver(void* b) : base(static_cast<uint8_t*>(b)) {}
+  template <class T>
+  T* take(size_t n) {
+    off = (off + 255) & ~size_t(255);
+    T* p = base ? reinterpret_cast<T*>(base + off) : nullptr;
+    off += n * sizeof(T);
+    return p;
+  }
+};
+}  // namespace
+
+int sm_count() {
+  const int d = current_device();
+  return device_facts(d) ? g_sm_count[d] : 148;
+}
+
+uint64_t wait_limit_ns() { return 1000000000ull; }  // 1 s per barrier wait
+
+// ------------------------------------------------------------------ tensor maps
+CUresult encode_tmap_2d(CUtensorMap* map, const void* base, CUtensorMapDataType dt, uint64_t cols, uint64_t rows,
+                        uint64_t row_bytes, uint32_t box_cols, uint32_t box_rows, CUtensorMapSwizzle swz) {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  if (!fn) {
+    std::lock_guard<std::mutex> lk(g_mu);
+    if (!fn) {
+      void* ptr = nullptr;
+      cudaDriverEntryPointQueryResult q;
+      if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) != cudaSuccess ||
+          q != cudaDriverEntryPointSuccess || !ptr)
+        return CUDA_ERROR_NOT_FOUND;
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(ptr);
+    }
+  }
+  const cuuint64_t gdim[2] = {cols, rows};
+  const cuuint64_t gstride[1] = {row_bytes};
+  const cuuint32_t box[2] = {box_cols, box_rows};
+  const cuuint32_t estride[2] = {1, 1};
+  return fn(map, dt, 2, const_cast<void*>(base), gdim, gstride, box, estride, CU_TENSOR_MAP_INTERLEAVE_NONE, swz,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+}
+
+// ------------------------------------------------------------------ timing hooks
+namespace {
+bool g_timing_on = false;
+struct Rec {
+  const char* name;
+  cudaEvent_t a, b;
+};
+struct Agg {
+  const char* name;
+  double ms;
+  int n;
+};
+std::vector<Rec> g_recs;
+std::vector<cudaEvent_t> g_free_ev;
+std::vector<Agg> g_agg;
+cudaEvent_t get_event() {
+  if (!g_free_ev.empty()) {
+    cudaEvent_t e = g_free_ev.back();
+    g_free_ev.pop_back();
+    return e;
+  }
+  cudaEvent_t e = nullptr;
+  cudaEventCreate(&e);
+  return e;
+}
+}  // namespace
+
+void timing_before(const char* name, cudaStream_t s) {
+  if (!g_timing_on) return;
+  Rec r{name, get_event(), get_event()};
+  cudaEventRecord(r.a, s);
+  g_recs.push_back(r);
+}
+void timing_after(const char*, cudaStream_t s) {
+  if (!g_timing_on || g_recs.empty()) return;
+  cudaEventRecord(g_recs.back().b, s);
+}
+
+// ------------------------------------------------------------------ workspace layouts
+namespace {
+struct FwdWs {
+  int32_t *counts, *offsets, *sorted, *inv, *blockcnt, *tile_prefix, *chunk;
+  __half *x_perm, *h;
+  float* y;
+  size_t bytes;
+};
+FwdWs carve_w4_forward(void* ws, int T, int H, int I, int E, int k) {
+  Carver c(ws);
+  FwdWs w;
+  const size_t P = (size_t)T * k;
+  w.counts = c.take<int32_t>(E);
+  w.offsets = c.take<int32_t>(E + 1);
+  w.sorted = c.take<int32_t>(P);
+  w.inv = c.take<int32_t>(P);
+  w.blockcnt = c.take<int32_t>((size_t)align_blocks(T, k) * E);
+  w.tile_prefix = c.take<int32_t>(E + 1);
+  w.chunk = c.take<int32_t>(E);
+  w.x_perm = c.take<__half>(P * H);
+  w.h = c.take<__half>(P * I);
+  w.y = c.take<float>(P * H);
+  w.bytes = c.off + 256;
+  return w;
+}
+struct GemmWs {
+  int32_t *row_count, *tile_prefix, *chunk;
+  __half* a;
+  size_t bytes;
+};
+GemmWs carve_gemm(void* ws, int M, int K, int E) {
+  Carver c(ws);
+  GemmWs w;
+  w.row_count = c.take<int32_t>(E);
+  w.tile_prefix = c.take<int32_t>(E + 1);
+  w.chunk = c.take<int32_t>(E);
+  w.a = c.take<__half>((size_t)M * K);
+  w.bytes = c.off + 256;
+  return w;
+}
+int pick_nmax(int max_rows_per_expert) { return max_rows_per_expert <= 64 ? 64 : 256; }
+
+bool shape_ok(int T, int H, int I, int E, int k) {
+  if (T < 1 || k < 1 || E < k || E > 1024) return false;
+  if (H < 128 || I < 128 || H % 128 || I % 128) return false;
+  if ((int64_t)T * k >= (1ll << 31) || (int64_t)E * 2 * I >= (1ll << 31) || (int64_t)E * H >= (1ll << 31)) return false;
+  return true;
+}
+}  // namespace
+
+}  // namespace moe
+
+using namespace moe;
+
+// ================================================================== C ABI
+extern "C" {
+
+const char* moe_status_string(moe_status_t s) {
+  switch (s) {
+    case MOE_OK: return "MOE_OK";
+    case MOE_ERR_INVALID_ARG: return "MOE_ERR_INVALID_ARG";
+    case MOE_ERR_UNSUPPORTED: return "MOE_ERR_UNSUPPORTED";
+    case MOE_ERR_WORKSPACE: return "MOE_ERR_WORKSPACE";
+    case MOE_ERR_CUDA: return "MOE_ERR_CUDA";
+    case MOE_ERR_TIMEOUT: return "MOE_ERR_TIMEOUT";
+    case MOE_ERR_DEVICE_CHECK: return "MOE_ERR_DEVICE_CHECK";
+  }
+  return "MOE_ERR_UNKNOWN";
+}
+
+moe_status_t moe_route(const float* logits, int T, int E, int k, int renormalize, int32_t* topk_ids, float* topk_w,
+                       cudaStream_t stream) {
+  if (T < 1 || k < 1 || E < k || E > 1024) return MOE_ERR_UNSUPPORTED;
+  if (!aligned(logits, 4) || !aligned(topk_ids, 4) || !aligned(topk_w, 4)) return MOE_ERR_INVALID_ARG;
+  if (moe_status_t st = check_device()) return st;
+  return launch_route(logits, T, E, k, renormalize, topk_ids, topk_w, stream) == cudaSuccess ? MOE_OK
+                                                                                               : MOE_ERR_CUDA;
+}
+
+size_t moe_align_capacity(int T, int k, int E, int align) {
+  if (T < 1 || k < 1 || E < 1 || align < 1) return 0;
+  return (size_t)T * k + (size_t)E * (align - 1);
+}
+
+size_t moe_align_workspace_size(int T, int k, int E) {
+  if (T < 1 || k < 1 || E < 1) return 0;
+  return (size_t)align_blocks(T, k) * E * sizeof(int32_t) + 256;
+}
+
+moe_status_t moe_align(const int32_t* topk_ids, int T, int k, int E, int align, int32_t* expert_counts,
+                       int32_t* expert_offsets, int32_t* sorted_ids, int32_t* inv_pos, void* ws, size_t ws_bytes,
+                       cudaStream_t stream) {
+  if (T < 1 || k < 1 || E < 1 || E > 1024 || align < 1 || (int64_t)T * k >= (1ll << 31)) return MOE_ERR_UNSUPPORTED;
+  if ((int64_t)moe_align_capacity(T, k, E, align) >= (1ll << 31)) return MOE_ERR_UNSUPPORTED;
+  if (!aligned(topk_ids, 4) || !aligned(expert_counts, 4) || !aligned(expert_offsets, 4) || !aligned(sorted_ids, 4) ||
+      !aligned(inv_pos, 4) || !aligned(ws, 16))
+    return MOE_ERR_INVALID_ARG;
+  if (ws_bytes < moe_align_workspace_size(T, k, E)) return MOE_ERR_WORKSPACE;
+  if (moe_status_t st = check_device()) return st;
+  const cudaError_t e = launch_align(topk_ids, T, k, E, align, expert_counts, expert_offsets, sorted_ids, inv_pos,
+                                     static_cast<int32_t*>(ws), 256, nullptr, nullptr, stream);
+  return e == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
+}
+
+size_t moe_w4a16_workspace_size(int T, int H, int I, int E, int k) {
+  if (!shape_ok(T, H, I, E, k)) return 0;
+  return carve_w4_forward(nullptr, T, H, I, E, k).bytes;
+}
+
+moe_status_t moe_w4a16_forward(const moe_w4a16_args* a, void* ws, size_t ws_bytes, cudaStream_t stream) {
+  if (!a) return MOE_ERR_INVALID_ARG;
+  if (!shape_ok(a->T, a->H, a->I, a->E, a->k)) return MOE_ERR_UNSUPPORTED;
+  if (!aligned(a->x, 16) || !aligned(a->topk_ids, 4) || !aligned(a->topk_w, 4) || !aligned(a->w13_q, 16) ||
+      !aligned(a->w13_s, 16) || !aligned(a->w2_q, 16) || !aligned(a->w2_s, 16) || !aligned(a->out, 16) ||
+      !aligned(ws, 256))
+    return MOE_ERR_INVALID_ARG;
+  const int T = a->T, H = a->H, I = a->I, E = a->E, k = a->k;
+  if (ws_bytes < moe_w4a16_workspace_size(T, H, I, E, k)) return MOE_ERR_WORKSPACE;
+  if (moe_status_t st = check_device()) return st;
+  const FwdWs w = carve_w4_forward(ws, T, H, I, E, k);
+  const int nmax = pick_nmax(T);
+  const int P = T * k;
+  cudaError_t e = launch_align(a->topk_ids, T, k, E, 1, w.counts, w.offsets, w.sorted, w.inv, w.blockcnt, nmax,
+                               w.tile_prefix, w.chunk, stream);
+  if (e == cudaSuccess) e = launch_permute_w4(static_cast<const uint16_t*>(a->x), w.inv, T, k, H, w.x_perm, stream);
+  const TileSched sched{w.offsets, w.counts, w.tile_prefix, w.chunk};
+  if (e == cudaSuccess) {
+    W4GemmProblem g{a->w13_q, static_cast<const uint16_t*>(a->w13_s), w.x_perm, P, H, E, 2 * I, true, I, sched, nmax,
+                    w.h, I, OUT_H_F16_INTERLEAVED};
+    e = launch_w4a16_gemm(g, stream);
+  }
+  if (e == cudaSuccess) {
+    W4GemmProblem g{a->w2_q, static_cast<const uint16_t*>(a->w2_s), w.h, P, I, E, H, false, 0, sched, nmax, w.y, H,
+                    OUT_F32};
+    e = launch_w4a16_gemm(g, stream);
+  }
+  if (e == cudaSuccess) e = launch_combine(w.y, w.inv, a->topk_w, T, k, H, a->out, a->out_fp32, stream);
+  return e == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
+}
+
+size_t moe_blockfp8_workspace_size(int T, int H, int I, int E, int k) {
+  (void)T, (void)H, (void)I, (void)E, (void)k;
+  return 0;
+}
+
+moe_status_t moe_blockfp8_forward(const moe_blockfp8_args* a, void* ws, size_t ws_bytes, cudaStream_t stream) {
+  (void)a, (void)ws, (void)ws_bytes, (void)stream;
+  return MOE_ERR_UNSUPPORTED;
+}
+
+size_t moe_w4a16_gemm_workspace_size(int M, int K, int N, int E) {
+  if (M < 1 || K < 128 || N < 128 || K % 128 || N % 128 || E < 1 || E > 1024) return 0;
+  return carve_gemm(nullptr, M, K, E).bytes;
+}
+
+moe_status_t moe_w4a16_gemm(const void* a, int a_is_bf16, const int32_t* w_q, const void* w_s,
+                            const int32_t* expert_offsets, int M, int K, int N, int E, void* out, int out_fp32,
+                            void* ws, size_t ws_bytes, cudaStream_t stream) {
+  if (M < 1 || K < 128 || N < 128 || K % 128 || N % 128 || E < 1 || E > 1024) return MOE_ERR_UNSUPPORTED;
+  if ((int64_t)E * N >= (1ll << 31) || (int64_t)M * K >= (1ll << 40)) return MOE_ERR_UNSUPPORTED;
+  if (!aligned(a, 16) || !aligned(w_q, 16) || !aligned(w_s, 16) || !aligned(expert_offsets, 4) || !aligned(out, 16) ||
+      !aligned(ws, 256))
+    return MOE_ERR_INVALID_ARG;
+  if (ws_bytes < moe_w4a16_gemm_workspace_size(M, K, N, E)) return MOE_ERR_WORKSPACE;
+  if (moe_status_t st = check_device()) return st;
+  const GemmWs w = carve_gemm(ws, M, K, E);
+  const int nmax = pick_nmax(M);
+  cudaError_t e = launch_sched_from_offsets(expert_offsets, E, M, nmax, w.row_count, w.tile_prefix, w.chunk, stream);
+  if (e == cudaSuccess) e = launch_convert_rows(static_cast<const uint16_t*>(a), a_is_bf16, M, K, w.a, stream);
+  if (e == cudaSuccess) {
+    const TileSched sched{expert_offsets, w.row_count, w.tile_prefix, w.chunk};
+    W4GemmProblem g{w_q, static_cast<const uint16_t*>(w_s), w.a, M, K, E, N, false, 0, sched, nmax, out, N,
+                    out_fp32 ? OUT_F32 : OUT_BF16};
+    e = launch_w4a16_gemm(g, stream);
+  }
+  return e == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
+}
+
+moe_status_t moe_get_device_status(cudaStream_t stream) {
+  if (cudaStreamSynchronize(stream) != cudaSuccess) return MOE_ERR_CUDA;
+  int v = 0;
+  if (cudaMemcpyFromSymbol(&v, g_device_status, sizeof(int)) != cudaSuccess) return MOE_ERR_CUDA;
+  if (v != 0) {
+    const int zero = 0;
+    if (cudaMemcpyToSymbol(g_device_status, &zero, sizeof(int)) != cudaSuccess) return MOE_ERR_CUDA;
+  }
+  return static_cast<moe_status_t>(v);
+}
+
+moe_status_t moe_timing_enable(int enable) {
+  g_timing_on = enable != 0;
+  return MOE_OK;
+}
+
+int moe_timing_read(const char** names, double* ms, int* launches, int max) {
+  cudaDeviceSynchronize();
+  for (const Rec& r : g_recs) {
+    float t = 0.f;
+    cudaEventElapsedTime(&t, r.a, r.b);
+    auto it = std::find_if(g_agg.begin(), g_agg.end(), [&](const Agg& a) { return std::strcmp(a.name, r.name) == 0; });
+    if (it == g_agg.end()) {
+      g_agg.push_back(Agg{r.name, 0.0, 0});
+      it = g_agg.end() - 1;
+    }
+    it->ms += t;
+    it->n += 1;
+    g_free_ev.push_back(r.a);
+    g_free_ev.push_back(r.b);
+  }
+  g_recs.clear();
+  const int n = (int)g_agg.size();
+  for (int i = 0; i < n && i < max; ++i) {
+    if (names) names[i] = g_agg[i].name;
+    if (ms) ms[i] = g_agg[i].ms;
+    if (launches) launches[i] = g_agg[i].n;
+  }
+  g_agg.clear();
+  return n;
+}
+
+}  // extern "C"
+
+// ------------------------------------------------------------------ debug: a wait that must time out
+namespace moe {
+__global__ void debug_wait_kernel(uint64_t limit_ns) {
+  __shared__ __align__(8) uint64_t bar;
+  __shared__ int abort_flag;
+  if (threadIdx.x == 0) {
+    mbar_init(&bar, 1);
+    abort_flag = 0;
+    fence_mbar_init();
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) mbar_wait(&bar, 0, &abort_flag, limit_ns);  // nothing ever arrives
+}
+}  // namespace moe
+
+extern "C" moe_status_t moe_debug_wait_timeout(int64_t limit_ns, cudaStream_t stream) {
+  if (limit_ns < 1 || limit_ns > 1000000000ll) return MOE_ERR_INVALID_ARG;
+  if (moe_status_t st = check_device()) return st;
+  moe::debug_wait_kernel<<<1, 32, 0, stream>>>((uint64_t)limit_ns);
+  return cudaGetLastError() == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
+}

@@ -1,0 +1,70 @@
+// Host-side declarations shared by the library's translation units (not part of the ABI).
+#pragma once
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "moe.h"
+
+namespace moe {
+
+// Kernel launch bookkeeping (per-kernel event timing for benchmarks).
+void timing_before(const char* name, cudaStream_t s);
+void timing_after(const char* name, cudaStream_t s);
+
+// Scheduler outputs for the grouped GEMMs.  Expert e owns activation / output rows
+// [row_start[e], row_start[e] + row_count[e]); those rows are cut into tile_prefix[e+1] -
+// tile_prefix[e] token tiles of `chunk[e]` rows (the last may be shorter); a GEMM over
+// m_tiles weight tiles per expert then has m_tiles * tile_prefix[E] work items.
+struct TileSched {
+  const int32_t* row_start;
+  const int32_t* row_count;
+  const int32_t* tile_prefix;  // [E+1]
+  const int32_t* chunk;        // [E]
+};
+
+// route / align / scheduler (route_align.cu)
+cudaError_t launch_route(const float* logits, int T, int E, int k, int renormalize, int32_t* ids, float* w,
+                         cudaStream_t s);
+int align_blocks(int T, int k);
+// blockcnt: [align_blocks * E] int32 scratch.  tile_prefix/chunk may be null (no scheduler).
+cudaError_t launch_align(const int32_t* ids, int T, int k, int E, int align, int32_t* counts, int32_t* offsets,
+                         int32_t* sorted_ids, int32_t* inv_pos, int32_t* blockcnt, int nmax, int32_t* tile_prefix,
+                         int32_t* chunk, cudaStream_t s);
+// Scheduler for the public grouped GEMM: from expert_offsets [E+1] (arbitrary row counts).
+cudaError_t launch_sched_from_offsets(const int32_t* offsets, int E, int M, int nmax, int32_t* row_count,
+                                      int32_t* tile_prefix, int32_t* chunk, cudaStream_t s);
+
+// permute / combine (permute_combine.cu)
+cudaError_t launch_permute_w4(const uint16_t* x_bf16, const int32_t* inv_pos, int T, int k, int H, __half* x_perm,
+                              cudaStream_t s);
+cudaError_t launch_convert_rows(const uint16_t* a, int a_is_bf16, int M, int K, __half* out, cudaStream_t s);
+cudaError_t launch_combine(const float* y_perm, const int32_t* inv_pos, const float* topk_w, int T, int k, int H,
+                           void* out, int out_fp32, cudaStream_t s);
+
+// W4A16 grouped GEMM (gemm_w4a16.cu)
+enum OutKind { OUT_H_F16_INTERLEAVED = 0, OUT_F32 = 1, OUT_BF16 = 2 };
+struct W4GemmProblem {
+  const int32_t* w_q;  // [E, rows_per_expert, K/8]
+  const uint16_t* w_s; // [E, rows_per_expert, K/32]
+  const __half* act;   // [act_rows, K] fp16, K interleaved in groups of 8
+  int act_rows;
+  int K, E, rows_per_expert;
+  bool gated;          // gate rows [0, I), up rows [I, 2I); output h [*, I]
+  int I;               // gated only
+  TileSched sched;
+  int nmax;
+  void* out;
+  int out_ld;          // elements per output row
+  OutKind out_kind;
+};
+cudaError_t launch_w4a16_gemm(const W4GemmProblem& p, cudaStream_t s);
+
+// driver entry point for tensor maps (api.cu)
+// 2-D tiled tensor map over a row-major [rows, cols] tensor at `base` (zero fill out of bounds).
+CUresult encode_tmap_2d(CUtensorMap* map, const void* base, CUtensorMapDataType dt, uint64_t cols, uint64_t rows,
+                        uint64_t row_bytes, uint32_t box_cols, uint32_t box_rows, CUtensorMapSwizzle swz);
+int sm_count();
+uint64_t wait_limit_ns();
+
+}  // namespace moe

@@ -1,0 +1,116 @@
+// a4 permute (x rows -> expert-sorted fp16 rows) and a8 combine (weighted sum of each token's
+// k expert outputs, in slot order, fp32).
+//
+// Activation rows that feed the W4A16 tensor-core GEMMs are stored in fp16 with the K index
+// interleaved inside every group of 8: position (0..7) holds K offset (0,4,1,5,2,6,3,7).
+// That is the order in which one packed INT4 word dequantizes with two-nibbles-per-lane
+// bit tricks, so the GEMM never has to shuffle weights; applying the same permutation to
+// both operands of a dot product leaves it unchanged.
+#include "common.cuh"
+#include "internal.h"
+
+namespace moe {
+
+__device__ __forceinline__ uint32_t pack_h2(float lo, float hi) {
+  const __half2 h = __floats2half2_rn(lo, hi);
+  return *reinterpret_cast<const uint32_t*>(&h);
+}
+__device__ __forceinline__ float bf16lo(uint32_t u) { return __uint_as_float(u << 16); }
+__device__ __forceinline__ float bf16hi(uint32_t u) { return __uint_as_float(u & 0xFFFF0000u); }
+
+// 8 bf16 (k0..k7 in order) -> 8 fp16 in the interleaved order (k0,k4,k1,k5,k2,k6,k3,k7)
+__device__ __forceinline__ uint4 bf16x8_to_f16x8_interleaved(uint4 v) {
+  const float f0 = bf16lo(v.x), f1 = bf16hi(v.x), f2 = bf16lo(v.y), f3 = bf16hi(v.y);
+  const float f4 = bf16lo(v.z), f5 = bf16hi(v.z), f6 = bf16lo(v.w), f7 = bf16hi(v.w);
+  return make_uint4(pack_h2(f0, f4), pack_h2(f1, f5), pack_h2(f2, f6), pack_h2(f3, f7));
+}
+__device__ __forceinline__ uint4 f16x8_interleave(uint4 v) {
+  // halves: v.x=(k0,k1) v.y=(k2,k3) v.z=(k4,k5) v.w=(k6,k7)
+  const uint32_t a = __byte_perm(v.x, v.z, 0x5410);  // (k0,k4)
+  const uint32_t b = __byte_perm(v.x, v.z, 0x7632);  // (k1,k5)
+  const uint32_t c = __byte_perm(v.y, v.w, 0x5410);  // (k2,k6)
+  const uint32_t d = __byte_perm(v.y, v.w, 0x7632);  // (k3,k7)
+  return make_uint4(a, b, c, d);
+}
+
+// one warp per (token, slot) pair: x_perm[inv_pos[p]] = interleave(fp16(x[p / k]))
+__global__ void __launch_bounds__(256) permute_w4_kernel(const uint4* __restrict__ x, const int32_t* __restrict__ inv_pos,
+                                                         int P, int k, int H8, uint4* __restrict__ x_perm) {
+  const int p = (int)((blockIdx.x * blockDim.x + threadIdx.x) >> 5);
+  const int lane = threadIdx.x & 31;
+  if (p >= P) return;
+  const int r = inv_pos[p];
+  if (r < 0) return;
+  const uint4* src = x + (size_t)(p / k) * H8;
+  uint4* dst = x_perm + (size_t)r * H8;
+  for (int c = lane; c < H8; c += 32) dst[c] = bf16x8_to_f16x8_interleaved(__ldg(src + c));
+}
+
+cudaError_t launch_permute_w4(const uint16_t* x_bf16, const int32_t* inv_pos, int T, int k, int H, __half* x_perm,
+                              cudaStream_t s) {
+  const int P = T * k;
+  timing_before("permute", s);
+  permute_w4_kernel<<<ceil_div(P, 8), 256, 0, s>>>(reinterpret_cast<const uint4*>(x_bf16), inv_pos, P, k, H / 8,
+                                                  reinterpret_cast<uint4*>(x_perm));
+  timing_after("permute", s);
+  return cudaGetLastError();
+}
+
+__global__ void __launch_bounds__(256) convert_rows_kernel(const uint4* __restrict__ a, int a_is_bf16, size_t n8,
+                                                           uint4* __restrict__ out) {
+  for (size_t i = blockIdx.x * (size_t)blockDim.x + threadIdx.x; i < n8; i += (size_t)gridDim.x * blockDim.x) {
+    const uint4 v = __ldg(a + i);
+    out[i] = a_is_bf16 ? bf16x8_to_f16x8_interleaved(v) : f16x8_interleave(v);
+  }
+}
+
+cudaError_t launch_convert_rows(const uint16_t* a, int a_is_bf16, int M, int K, __half* out, cudaStream_t s) {
+  const size_t n8 = (size_t)M * K / 8;
+  const int blocks = (int)std::min<size_t>((n8 + 255) / 256, (size_t)sm_count() * 8);
+  timing_before("convert", s);
+  convert_rows_kernel<<<blocks, 256, 0, s>>>(reinterpret_cast<const uint4*>(a), a_is_bf16, n8,
+                                             reinterpret_cast<uint4*>(out));
+  timing_after("convert", s);
+  return cudaGetLastError();
+}
+
+// out[t][c..c+3] = sum_s w[t][s] * y_perm[inv_pos[t*k+s]][c..c+3], fp32, slot order
+__global__ void __launch_bounds__(256) combine_kernel(const float4* __restrict__ y, const int32_t* __restrict__ inv_pos,
+                                                      const float* __restrict__ w, int T, int k, int H4,
+                                                      void* __restrict__ out, int out_fp32) {
+  const size_t i = blockIdx.x * (size_t)blockDim.x + threadIdx.x;
+  if (i >= (size_t)T * H4) return;
+  const int t = (int)(i / H4), c = (int)(i % H4);
+  float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+  for (int s = 0; s < k; ++s) {
+    const int r = __ldg(inv_pos + (size_t)t * k + s);
+    if (r < 0) continue;
+    const float ws = __ldg(w + (size_t)t * k + s);
+    const float4 v = __ldg(y + (size_t)r * H4 + c);
+    acc.x = fmaf(ws, v.x, acc.x);
+    acc.y = fmaf(ws, v.y, acc.y);
+    acc.z = fmaf(ws, v.z, acc.z);
+    acc.w = fmaf(ws, v.w, acc.w);
+  }
+  if (out_fp32) {
+    reinterpret_cast<float4*>(out)[i] = acc;
+  } else {
+    const __nv_bfloat162 lo = __floats2bfloat162_rn(acc.x, acc.y), hi = __floats2bfloat162_rn(acc.z, acc.w);
+    uint2 u;
+    u.x = *reinterpret_cast<const uint32_t*>(&lo);
+    u.y = *reinterpret_cast<const uint32_t*>(&hi);
+    reinterpret_cast<uint2*>(out)[i] = u;
+  }
+}
+
+cudaError_t launch_combine(const float* y_perm, const int32_t* inv_pos, const float* topk_w, int T, int k, int H,
+                           void* out, int out_fp32, cudaStream_t s) {
+  const size_t n = (size_t)T * (H / 4);
+  timing_before("combine", s);
+  combine_kernel<<<(unsigned)((n + 255) / 256), 256, 0, s>>>(reinterpret_cast<const float4*>(y_perm), inv_pos, topk_w,
+                                                              T, k, H / 4, out, out_fp32);
+  timing_after("combine", s);
+  return cudaGetLastError();
+}
+
+}  // namespace moe

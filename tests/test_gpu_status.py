@@ -1,0 +1,33 @@
+"""Failure detection on the GPU without a fault: bounded waits and device-side input checks
+report through the device status word; the context stays usable afterwards."""
+import numpy as np
+import pytest
+import torch
+
+from helpers import dev
+
+pytestmark = pytest.mark.gpu
+moe = pytest.importorskip("quantized_mixture_experts_softmax_b200")
+
+
+def test_bounded_wait_times_out_and_reports():
+    moe.moe_get_device_status()
+    moe.moe_debug_wait_timeout(2_000_000)  # 2 ms on a barrier nothing arrives on
+    assert moe.moe_get_device_status() == moe.MOE_ERR_TIMEOUT
+    assert moe.moe_get_device_status() == 0
+    # the context is still healthy: a normal call works and reports nothing
+    lg = np.random.default_rng(0).normal(size=(4, 16)).astype(np.float32)
+    ids, _ = moe.moe_route(dev(lg), 2)
+    torch.cuda.synchronize()
+    assert moe.moe_get_device_status() == 0
+    assert ids.shape == (4, 2)
+
+
+def test_bad_offsets_in_grouped_gemm_are_flagged_not_used():
+    a = torch.zeros(16, 128, dtype=torch.bfloat16, device="cuda")
+    w_q = torch.zeros(2, 128, 16, dtype=torch.int32, device="cuda")
+    w_s = torch.zeros(2, 128, 4, dtype=torch.bfloat16, device="cuda")
+    off = dev(np.array([0, 20, 16], np.int32))  # expert 0 reaches past M: flagged and skipped
+    moe.moe_get_device_status()
+    moe.moe_w4a16_gemm(a, w_q, w_s, off, out_fp32=True)
+    assert moe.moe_get_device_status() == moe.MOE_ERR_DEVICE_CHECK
