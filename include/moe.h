@@ -21,9 +21,10 @@
  * Conventions for every call:
  *  - All tensor pointers are DEVICE pointers owned by the caller, row-major, 16-byte aligned.
  *    The library never allocates, frees or synchronises inside these calls; all scratch
- *    memory is the caller's workspace (size from the matching *_workspace_size call).
+ *    memory is the caller's workspace (size from the matching *_workspace_size call), except
+ *    for moe_align_noalloc, whose scratch is a fixed array inside the library (see there).
  *  - Work is enqueued on `stream` and returns immediately; no host reads of device data, so
- *    the calls may be captured in a CUDA graph.
+ *    the calls that take a workspace may be captured in a CUDA graph.
  *  - Argument, shape and alignment errors return an error code synchronously with nothing
  *    enqueued.  A failed kernel launch returns MOE_ERR_CUDA.
  *  - Faults the GPU detects (an expert id outside [0,E), a wait that timed out) are recorded
@@ -85,6 +86,21 @@ size_t moe_align_workspace_size(int T, int k, int E);
 moe_status_t moe_align(const int32_t* topk_ids, int T, int k, int E, int align, int32_t* expert_counts,
                        int32_t* expert_offsets, int32_t* sorted_ids, int32_t* inv_pos, void* ws, size_t ws_bytes,
                        cudaStream_t stream);
+
+/* moe_align_noalloc: the same alignment as moe_align, for callers that cannot allocate device
+ * memory and have no workspace to pass (e.g. a plugin inside a host framework that owns all
+ * device buffers, or a deployment with a device memory budget fixed at start-up).  The pages
+ * describing the method have no counterpart of this call; it exists for those callers.
+ * The scratch lives in a fixed 512 KiB array inside the library (131072 int32, kept on every
+ * GPU that loads the library until the process exits); a call needs ceil(T*k/512)*E of them and
+ * returns MOE_ERR_UNSUPPORTED when that is more.  It allocates nothing.  The first call on a
+ * device looks up the array's device address (cudaGetSymbolAddress) and caches it: make that
+ * first call before any stream capture.  Every call reuses the same array and overwrites each
+ * entry it reads, so earlier contents never leak into a result; calls that overlap on the GPU
+ * race on the array and must be serialised by the caller.  Arguments and outputs otherwise as
+ * moe_align. */
+moe_status_t moe_align_noalloc(const int32_t* topk_ids, int T, int k, int E, int align, int32_t* expert_counts,
+                               int32_t* expert_offsets, int32_t* sorted_ids, int32_t* inv_pos, cudaStream_t stream);
 
 /* ------------------------------------------------------------------ a2..a8: W4A16 layer
  * out[t] = sum_{s<k} topk_w[t,s] * y_{t,s},   y = h . W2[e]^T,   h_j = SiLU(g_j) * g_{I+j},

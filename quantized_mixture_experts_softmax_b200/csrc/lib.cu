@@ -4,3 +4,4 @@
 #include "permute_combine.cu"
 #include "gemm_w4a16.cu"
 #include "api.cu"
+#include "align_noalloc.cu"
