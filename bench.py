@@ -370,7 +370,11 @@ def main():
     ap.add_argument("--workload", choices=sorted(WORKLOADS), default="decode")
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--experts", type=int, default=None,
+                    help="override the expert count (small profiling cases only; not a bench line)")
     args = ap.parse_args()
+    if args.experts:
+        MODEL["E"] = args.experts
 
     if args.impl == "reference":
         rank = int(os.environ.get("RANK", "0"))

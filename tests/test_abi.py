@@ -11,8 +11,8 @@ ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 
 @pytest.fixture(scope="module")
 def native():
-    from quantized_mixture_experts_softmax_b200 import build
-    build.build()
+    import __graft_entry__
+    __graft_entry__.build()
     from quantized_mixture_experts_softmax_b200 import _native
     return _native
 
