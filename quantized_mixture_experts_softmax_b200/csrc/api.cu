@@ -170,7 +170,8 @@ GemmWs carve_gemm(void* ws, int M, int K, int E) {
   w.bytes = c.off + 256;
   return w;
 }
-int pick_nmax(int max_rows_per_expert) { return max_rows_per_expert <= 64 ? 64 : 256; }
+// token-tile height cap: thin variant (w4::kThinN rows) when no expert can exceed 64 rows
+int pick_nmax(int max_rows_per_expert) { return max_rows_per_expert <= 64 ? w4::kThinN : 256; }
 
 bool shape_ok(int T, int H, int I, int E, int k) {
   if (T < 1 || k < 1 || E < k || E > 1024) return false;

@@ -33,10 +33,8 @@ namespace w4 {
 constexpr int BM = 128;  // weight rows per tile (MMA M)
 constexpr int KB = 256;  // K per weight stage
 constexpr int KS = 64;   // K per MMA step (one 128-byte swizzle atom of fp16)
-constexpr int kThreads = 512;
-constexpr int kEpiWarp0 = 4;
-constexpr int kDqWarp0 = 8;
-constexpr int kNumDqWarps = 8;
+constexpr int kEpiWarp0 = 4;  // warps 4-7: epilogue
+constexpr int kDqWarp0 = 8;   // warps 8..: dequantization
 
 __host__ __device__ constexpr int pow2_at_least(int v) {
   int p = 32;
@@ -44,34 +42,84 @@ __host__ __device__ constexpr int pow2_at_least(int v) {
   return p;
 }
 
+// Two variants by token-tile height:
+//  thin (at most kThinN rows, decode-sized experts): the activation tile of each 256-K weight
+//    stage travels in that stage, so it is prefetched as deep as the weights;
+//  wide (up to 256 rows): activations have their own ring of 64-K tiles (a 256-row tile of
+//    256 K would not fit next to the weights).
+// Depths: (weight stages, activation stages [wide only], dequantized-A buffers).
+#ifndef MOE_W4_THIN_N
+#define MOE_W4_THIN_N 16
+#endif
+#ifndef MOE_W4_GT
+#define MOE_W4_GT 5, 0, 6
+#endif
+#ifndef MOE_W4_PT
+#define MOE_W4_PT 8, 0, 8
+#endif
+#ifndef MOE_W4_GW
+#define MOE_W4_GW 2, 2, 2
+#endif
+#ifndef MOE_W4_PW
+#define MOE_W4_PW 4, 3, 2
+#endif
+constexpr int kThinN = MOE_W4_THIN_N;
+struct Depths {
+  int wst, bst, abuf;
+};
+template <bool GATED, bool THIN>
+constexpr Depths depths() {
+  return GATED ? (THIN ? Depths{MOE_W4_GT} : Depths{MOE_W4_GW}) : (THIN ? Depths{MOE_W4_PT} : Depths{MOE_W4_PW});
+}
+
 template <bool GATED, int NMAX>
 struct Cfg {
+  static constexpr bool THIN = NMAX <= kThinN;
+  // thin: the dequantized A operand goes to tensor memory (tcgen05.st by the dequant warps,
+  // read by the MMA as its A operand), which leaves room for a deep A ring; wide: the
+  // accumulators fill tensor memory, so A is staged in shared memory.
+  static constexpr bool A_TMEM = THIN;
   static constexpr int NA = GATED ? 2 : 1;
-  static constexpr int WST = GATED ? (NMAX <= 64 ? 3 : 2) : (NMAX <= 64 ? 8 : 4);
-  static constexpr int BST = GATED ? (NMAX <= 64 ? 4 : 2) : (NMAX <= 64 ? 4 : 3);
-  static constexpr int ABUF = 2;
+  // Dependent tcgen05.mma on one accumulator serialise on the MMA latency when N is small;
+  // the thin variant spreads each matrix's K steps over CH independent accumulators (summed
+  // in the epilogue) so that 4 MMAs are in flight.
+  static constexpr int CH = THIN ? 4 / NA : 1;
+  static constexpr int NDQ = THIN ? 16 : 8;  // dequantization warps
+  static constexpr int THREADS = (kDqWarp0 + NDQ) * 32;
+  static constexpr int WST = depths<GATED, THIN>().wst;
+  static constexpr int BST = THIN ? 0 : depths<GATED, THIN>().bst;
+  static constexpr int ABUF = depths<GATED, THIN>().abuf;
+  static constexpr int NSUB = KB / KS;               // 64-K steps per weight stage
   static constexpr int W_TILE = BM * KB / 2;         // packed INT4 bytes
   static constexpr int S_TILE = BM * (KB / 32) * 2;  // bf16 scales
   static constexpr int A_TILE = BM * KS * 2;         // dequantized fp16 operand
-  static constexpr int B_TILE = NMAX * KS * 2;       // activation operand
-  static constexpr int ACC_COLS = NA * NMAX;
+  static constexpr int B_ATOM = NMAX * KS * 2;       // activation tile of one 64-K step
+  static constexpr int STAGE_W = 0;
+  static constexpr int STAGE_S = NA * W_TILE;
+  static constexpr int STAGE_B = STAGE_S + NA * S_TILE;
+  static constexpr int STAGE = STAGE_B + (THIN ? NSUB * B_ATOM : 0);
+  static constexpr int ACC_COLS = NA * CH * NMAX;
   static constexpr int ACC_BUFS = (2 * ACC_COLS <= 512) ? 2 : 1;
-  static constexpr int TMEM_COLS = pow2_at_least(ACC_BUFS * ACC_COLS);
-  static constexpr int OFF_W = 0;
-  static constexpr int OFF_S = OFF_W + WST * NA * W_TILE;
-  static constexpr int OFF_A = OFF_S + WST * NA * S_TILE;
-  static constexpr int OFF_B = OFF_A + ABUF * NA * A_TILE;
-  static constexpr int OFF_BAR = OFF_B + BST * B_TILE;
+  static constexpr int A_COLS = KS / 2;                 // one 64-K fp16 row = 32 TMEM columns
+  static constexpr int A_COL0 = ACC_BUFS * ACC_COLS;    // first TMEM column of the A ring
+  static constexpr int TMEM_COLS = pow2_at_least(A_COL0 + (A_TMEM ? ABUF * NA * A_COLS : 0));
+  static constexpr int OFF_A = WST * STAGE;
+  static constexpr int OFF_B = OFF_A + (A_TMEM ? 0 : ABUF * NA * A_TILE);  // wide activation ring
+  static constexpr int OFF_BAR = OFF_B + BST * B_ATOM;
   static constexpr int NUM_BARS = 2 * WST + 2 * BST + 2 * ABUF + 2 * ACC_BUFS + 1;
   static constexpr int OFF_MISC = OFF_BAR + NUM_BARS * 8;
   static constexpr int OFF_PREFIX = OFF_MISC + 16;
-  static_assert(OFF_A % 1024 == 0 && OFF_B % 1024 == 0, "swizzled tiles need 1024-byte alignment");
-  static_assert(ACC_BUFS * ACC_COLS <= 512, "TMEM has 512 columns");
+  static_assert(STAGE % 1024 == 0 && STAGE_B % 1024 == 0 && OFF_A % 1024 == 0 && OFF_B % 1024 == 0,
+                "swizzled tiles need 1024-byte alignment");
+  static_assert(A_COL0 + (A_TMEM ? ABUF * NA * A_COLS : 0) <= 512, "TMEM has 512 columns");
   static constexpr size_t smem_bytes(int E) { return (size_t)OFF_PREFIX + 4 * (size_t)(E + 1) + 1024; }
+  static_assert(smem_bytes(1024) <= 232448, "shared memory budget");
+  static_assert(!THIN || A_TMEM, "the thin variant keeps A in tensor memory");
 };
 
 struct Params {
   int K, E, rows_per_expert, I, m_tiles;
+  int scales_tma;  // 1: scales arrive by TMA (K % 256 == 0), else by cp.async
   const uint16_t* w_s;
   TileSched sched;
   void* out;
@@ -159,16 +207,17 @@ __device__ __forceinline__ int interleave_pos(int j) {
 }
 
 template <bool GATED, int NMAX>
-__global__ void __launch_bounds__(kThreads, 1)
-    w4a16_gemm_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CUtensorMap tm_b,
-                      const Params p) {
+__global__ void __launch_bounds__(Cfg<GATED, NMAX>::THREADS, 1)
+    w4a16_gemm_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CUtensorMap tm_s,
+                      const __grid_constant__ CUtensorMap tm_b, const Params p) {
   using C = Cfg<GATED, NMAX>;
-  constexpr int NA = C::NA, WST = C::WST, BST = C::BST, ABUF = C::ABUF, ACCB = C::ACC_BUFS;
+  constexpr bool THIN = C::THIN;
+  constexpr int NA = C::NA, WST = C::WST, BST = C::BST, ABUF = C::ABUF, ACCB = C::ACC_BUFS, NSUB = C::NSUB;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint64_t* full_w = reinterpret_cast<uint64_t*>(smem + C::OFF_BAR);
   uint64_t* empty_w = full_w + WST;
-  uint64_t* full_b = empty_w + WST;
+  uint64_t* full_b = empty_w + WST;  // wide variant only
   uint64_t* empty_b = full_b + BST;
   uint64_t* a_full = empty_b + BST;
   uint64_t* a_empty = a_full + ABUF;
@@ -185,15 +234,18 @@ __global__ void __launch_bounds__(kThreads, 1)
   for (int i = threadIdx.x; i <= p.E; i += blockDim.x) sprefix[i] = __ldg(p.sched.tile_prefix + i);
   if (threadIdx.x == 0) {
     for (int i = 0; i < WST; ++i) {
-      mbar_init(&full_w[i], 1 + 32);  // expect_tx arrival + one cp.async arrival per producer lane
-      mbar_init(&empty_w[i], kNumDqWarps);
+      // full: the expect_tx arrival (+ one cp.async arrival per producer lane when scales
+      // come by cp.async); empty: the dequant warps (+ the MMA commit when the stage also
+      // holds the activation tile)
+      mbar_init(&full_w[i], p.scales_tma ? 1 : 1 + 32);
+      mbar_init(&empty_w[i], C::NDQ + (THIN ? 1 : 0));
     }
     for (int i = 0; i < BST; ++i) {
       mbar_init(&full_b[i], 1);
       mbar_init(&empty_b[i], 1);
     }
     for (int i = 0; i < ABUF; ++i) {
-      mbar_init(&a_full[i], kNumDqWarps);
+      mbar_init(&a_full[i], C::NDQ);
       mbar_init(&a_empty[i], 1);
     }
     for (int i = 0; i < ACCB; ++i) {
@@ -206,6 +258,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
   if (warp == 0 && lane == 0) {
     prefetch_tmap(&tm_w);
+    if (p.scales_tma) prefetch_tmap(&tm_s);
     prefetch_tmap(&tm_b);
   }
   if (warp == 1) {
@@ -219,11 +272,11 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int total = p.m_tiles * sprefix[p.E];
   const int K = p.K;
   const int nkb = ceil_div(K, KB);
-  const int nks = K / KS;
 
   if (warp == 0) {
-    // ---------------------------------------------------------------- weight producer
-    const uint64_t pol = policy_evict_first();
+    // ---------------------------------------------------------------- weight (+ activation) producer
+    const uint64_t pol_w = policy_evict_first();
+    const uint64_t pol_b = policy_evict_last();
     const int kg = K / 32;
     int ws = 0, issued = 0;
     uint32_t ph = 0;
@@ -235,26 +288,40 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int kb = 0; kb < nkb; ++kb) {
         ok = __all_sync(0xffffffffu, mbar_wait(&empty_w[ws], ph ^ 1u, abort_flag, lim));
         if (!ok) break;
+        uint8_t* st = smem + ws * C::STAGE;
+        const int nsub = min(NSUB, (K - kb * KB) / KS);
         if (lane == 0) {
-          mbar_arrive_expect_tx(&full_w[ws], NA * C::W_TILE);
-          tma_load_2d_hint(smem + C::OFF_W + (ws * NA + 0) * C::W_TILE, &tm_w, &full_w[ws], kb * (KB / 8), row_g, pol);
-          if (GATED)
-            tma_load_2d_hint(smem + C::OFF_W + (ws * NA + 1) * C::W_TILE, &tm_w, &full_w[ws], kb * (KB / 8), row_u,
-                             pol);
-        }
-        const int ng = min(8, kg - kb * 8);  // 4 or 8: K is a multiple of 128
-#pragma unroll
-        for (int mat = 0; mat < NA; ++mat) {
-          const int row0 = mat ? row_u : row_g;
-#pragma unroll
-          for (int rr = lane; rr < BM; rr += 32) {
-            const uint16_t* src = p.w_s + (size_t)(row0 + rr) * kg + kb * 8;
-            uint8_t* dst = smem + C::OFF_S + (ws * NA + mat) * C::S_TILE + rr * 16;
-            cp_async_8(dst, src);
-            if (ng == 8) cp_async_8(dst + 8, src + 4);
+          uint32_t bytes = NA * C::W_TILE + (p.scales_tma ? NA * C::S_TILE : 0);
+          if (THIN) bytes += (uint32_t)(nsub * I.nmma * KS * 2);
+          mbar_arrive_expect_tx(&full_w[ws], bytes);
+          tma_load_2d_hint(st + C::STAGE_W, &tm_w, &full_w[ws], kb * (KB / 8), row_g, pol_w);
+          if (GATED) tma_load_2d_hint(st + C::STAGE_W + C::W_TILE, &tm_w, &full_w[ws], kb * (KB / 8), row_u, pol_w);
+          if (p.scales_tma) {
+            tma_load_2d_hint(st + C::STAGE_S, &tm_s, &full_w[ws], kb * (KB / 32), row_g, pol_w);
+            if (GATED) tma_load_2d_hint(st + C::STAGE_S + C::S_TILE, &tm_s, &full_w[ws], kb * (KB / 32), row_u, pol_w);
+          }
+          if (THIN) {
+            for (int j = 0; j < nsub; ++j)
+              for (int r = 0; r < I.nmma; r += 16)
+                tma_load_2d_hint(st + C::STAGE_B + j * C::B_ATOM + r * 128, &tm_b, &full_w[ws], kb * KB + j * KS,
+                                 I.r0 + r, pol_b);
           }
         }
-        cp_async_arrive_noinc(&full_w[ws]);
+        if (!p.scales_tma) {
+          const int ng = min(8, kg - kb * 8);  // 4 or 8: K is a multiple of 128
+#pragma unroll
+          for (int mat = 0; mat < NA; ++mat) {
+            const int row0 = mat ? row_u : row_g;
+#pragma unroll
+            for (int rr = lane; rr < BM; rr += 32) {
+              const uint16_t* src = p.w_s + (size_t)(row0 + rr) * kg + kb * 8;
+              uint8_t* dst = st + C::STAGE_S + mat * C::S_TILE + rr * 16;
+              cp_async_8(dst, src);
+              if (ng == 8) cp_async_8(dst + 8, src + 4);
+            }
+          }
+          cp_async_arrive_noinc(&full_w[ws]);
+        }
         ++issued;
         if (++ws == WST) {
           ws = 0;
@@ -267,38 +334,64 @@ __global__ void __launch_bounds__(kThreads, 1)
   } else if (warp == 1) {
     // ---------------------------------------------------------------- MMA issuer
     if (lane == 0) {
-      int ab = 0, bs = 0, acc = 0;
-      uint32_t ph_a = 0, ph_b = 0, ph_acc = 0;
+      int ab = 0, bs = 0, acc = 0, ws = 0;
+      uint32_t ph_a = 0, ph_b = 0, ph_acc = 0, ph_w = 0;
       bool ok = true;
       for (int it = blockIdx.x; it < total && ok; it += gridDim.x) {
         const Item I = decode_item(it, sprefix, p);
         const uint32_t idesc = make_idesc(BM, I.nmma, 0, 0);
         if (!(ok = mbar_wait(&acc_empty[acc], ph_acc ^ 1u, abort_flag, lim))) break;
         tc_fence_after();
-        const uint32_t d0 = tmem_base + (uint32_t)(acc * C::ACC_COLS);
-        const uint32_t d1 = d0 + NMAX;
-        for (int ks = 0; ks < nks; ++ks) {
-          if (!(ok = mbar_wait(&a_full[ab], ph_a, abort_flag, lim))) break;
-          if (!(ok = mbar_wait(&full_b[bs], ph_b, abort_flag, lim))) break;
-          tc_fence_after();
-          const uint64_t a0 = sw128_kmajor_desc(smem_u32(smem + C::OFF_A + (ab * NA + 0) * C::A_TILE));
-          const uint64_t a1 = sw128_kmajor_desc(smem_u32(smem + C::OFF_A + (ab * NA + (NA - 1)) * C::A_TILE));
-          const uint64_t b = sw128_kmajor_desc(smem_u32(smem + C::OFF_B + bs * C::B_TILE));
+        const uint32_t d0 = tmem_base + (uint32_t)(acc * C::ACC_COLS);  // [matrix][chain][NMAX] columns
+        const uint32_t d1 = d0 + C::CH * NMAX;
+        for (int kb = 0; kb < nkb && ok; ++kb) {
+          const int nsub = min(NSUB, (K - kb * KB) / KS);
+          if (THIN && !(ok = mbar_wait(&full_w[ws], ph_w, abort_flag, lim))) break;
+          for (int j = 0; j < nsub; ++j) {
+            if (!(ok = mbar_wait(&a_full[ab], ph_a, abort_flag, lim))) break;
+            if (!THIN && !(ok = mbar_wait(&full_b[bs], ph_b, abort_flag, lim))) break;
+            tc_fence_after();
+            const uint8_t* bt = THIN ? smem + ws * C::STAGE + C::STAGE_B + j * C::B_ATOM : smem + C::OFF_B + bs * C::B_ATOM;
+            const uint64_t b = sw128_kmajor_desc(smem_u32(bt));
+            if constexpr (C::A_TMEM) {
+              constexpr int CH = C::CH;
+              const uint32_t a0 = tmem_base + (uint32_t)(C::A_COL0 + ab * NA * C::A_COLS);
 #pragma unroll
-          for (int kk = 0; kk < KS / 16; ++kk) {
-            const uint32_t accum = (ks | kk) != 0;
-            umma_f16(d0, a0 + 2 * kk, b + 2 * kk, idesc, accum);  // +32 bytes along K
-            if (GATED) umma_f16(d1, a1 + 2 * kk, b + 2 * kk, idesc, accum);
+              for (int kk = 0; kk < KS / 16; ++kk) {
+                const uint32_t accum = (kb | j | (kk / CH)) != 0;  // each chain starts fresh at K = 0
+                const uint32_t dc = d0 + (uint32_t)((kk % CH) * NMAX);
+                umma_f16_ts(dc, a0 + 8 * kk, b + 2 * kk, idesc, accum);  // 16 K = 8 columns / 32 bytes
+                if (GATED) umma_f16_ts(dc + CH * NMAX, a0 + C::A_COLS + 8 * kk, b + 2 * kk, idesc, accum);
+              }
+            } else {
+              const uint64_t a0 = sw128_kmajor_desc(smem_u32(smem + C::OFF_A + (ab * NA + 0) * C::A_TILE));
+              const uint64_t a1 = sw128_kmajor_desc(smem_u32(smem + C::OFF_A + (ab * NA + (NA - 1)) * C::A_TILE));
+#pragma unroll
+              for (int kk = 0; kk < KS / 16; ++kk) {
+                const uint32_t accum = (kb | j | kk) != 0;
+                umma_f16(d0, a0 + 2 * kk, b + 2 * kk, idesc, accum);  // +32 bytes along K
+                if (GATED) umma_f16(d1, a1 + 2 * kk, b + 2 * kk, idesc, accum);
+              }
+            }
+            umma_commit(&a_empty[ab]);
+            if (++ab == ABUF) {
+              ab = 0;
+              ph_a ^= 1u;
+            }
+            if (!THIN) {
+              umma_commit(&empty_b[bs]);
+              if (++bs == BST) {
+                bs = 0;
+                ph_b ^= 1u;
+              }
+            }
           }
-          umma_commit(&a_empty[ab]);
-          umma_commit(&empty_b[bs]);
-          if (++ab == ABUF) {
-            ab = 0;
-            ph_a ^= 1u;
-          }
-          if (++bs == BST) {
-            bs = 0;
-            ph_b ^= 1u;
+          if (THIN && ok) {
+            umma_commit(&empty_w[ws]);  // the stage's activation tile has been read
+            if (++ws == WST) {
+              ws = 0;
+              ph_w ^= 1u;
+            }
           }
         }
         if (!ok) break;
@@ -312,9 +405,11 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_wait_plain(drain, 0, lim);
     }
   } else if (warp == 2) {
-    // ---------------------------------------------------------------- activation producer
-    if (lane == 0) {
+    // ---------------------------------------------------------------- activation producer (wide variant)
+    if constexpr (!THIN) {
+     if (lane == 0) {
       const uint64_t pol = policy_evict_last();
+      const int nks = K / KS;
       int bs = 0, issued = 0;
       uint32_t ph = 0;
       bool ok = true;
@@ -324,7 +419,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (!(ok = mbar_wait(&empty_b[bs], ph ^ 1u, abort_flag, lim))) break;
           mbar_arrive_expect_tx(&full_b[bs], (uint32_t)(I.nmma * KS * 2));
           for (int r = 0; r < I.nmma; r += 16)
-            tma_load_2d_hint(smem + C::OFF_B + bs * C::B_TILE + r * 128, &tm_b, &full_b[bs], ks * KS, I.r0 + r, pol);
+            tma_load_2d_hint(smem + C::OFF_B + bs * C::B_ATOM + r * 128, &tm_b, &full_b[bs], ks * KS, I.r0 + r, pol);
           ++issued;
           if (++bs == BST) {
             bs = 0;
@@ -333,6 +428,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
       }
       for (int i = max(0, issued - BST); i < issued; ++i) mbar_wait_plain(&full_b[i % BST], (i / BST) & 1, lim);
+     }
     }
   } else if (warp >= kEpiWarp0 && warp < kEpiWarp0 + 4) {
     // ---------------------------------------------------------------- epilogue
@@ -349,8 +445,20 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int c0 = 0; c0 < I.nmma; c0 += 16) {
         uint32_t g[16], u[16];
         tmem_ld16(tb + c0, g);
-        if (GATED) tmem_ld16(tb + NMAX + c0, u);
+        if (GATED) tmem_ld16(tb + C::CH * NMAX + c0, u);
         tmem_ld_wait();
+#pragma unroll
+        for (int c = 1; c < C::CH; ++c) {  // sum the independent K chains
+          uint32_t g2[16], u2[16];
+          tmem_ld16(tb + c * NMAX + c0, g2);
+          if (GATED) tmem_ld16(tb + (C::CH + c) * NMAX + c0, u2);
+          tmem_ld_wait();
+#pragma unroll
+          for (int i = 0; i < 16; ++i) {
+            g[i] = __float_as_uint(__uint_as_float(g[i]) + __uint_as_float(g2[i]));
+            if (GATED) u[i] = __float_as_uint(__uint_as_float(u[i]) + __uint_as_float(u2[i]));
+          }
+        }
         const int nv = min(16, I.nvalid - c0);
         if (GATED) {
           __half* out = reinterpret_cast<__half*>(p.out) + (size_t)(I.r0 + c0) * p.out_ld + interleave_pos(col);
@@ -382,54 +490,139 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
     }
   } else if (warp >= kDqWarp0) {
-    // ---------------------------------------------------------------- dequantization
-    const int dt = threadIdx.x - kDqWarp0 * 32;  // 0..255
-    const int mat = GATED ? (dt >> 7) : 0;
-    const int half = GATED ? 0 : (dt >> 7);
-    const int row = dt & 127;
-    const int sw = row & 7;
-    int ws = 0, ab = 0;
-    uint32_t ph_w = 0, ph_a = 0;
-    bool ok = true;
-    for (int it = blockIdx.x; it < total && ok; it += gridDim.x) {
-      for (int kb = 0; kb < nkb && ok; ++kb) {
-        ok = __all_sync(0xffffffffu, mbar_wait(&full_w[ws], ph_w, abort_flag, lim));
-        if (!ok) break;
-        const uint32_t wrow = smem_u32(smem + C::OFF_W + (ws * NA + mat) * C::W_TILE + row * 128);
-        const uint4 sc = ld_shared_v4(smem_u32(smem + C::OFF_S + (ws * NA + mat) * C::S_TILE + row * 16));
-        const int nsub = min(KB / KS, (K - kb * KB) / KS);
+    if constexpr (THIN) {
+      // ---------------------------------------------------------------- dequantization -> TMEM
+      // 16 warps; warp dw writes TMEM lanes 32*(dw%4).. (its rows).  GATED: warps 0-7 gate,
+      // 8-15 up, each thread one row and one 32-K half of every 64-K step.  Plain: each thread
+      // one row and one 16-K quarter of every step.
+      const int dw = warp - kDqWarp0;
+      const int row = (dw & 3) * 32 + lane;
+      const int sw = row & 7;
+      const int mat = GATED ? (dw >> 3) : 0;
+      const int part = GATED ? ((dw >> 2) & 1) : (dw >> 2);  // K half (GATED) or quarter (plain)
+      const uint32_t lane_base = tmem_base + ((uint32_t)((dw & 3) * 32) << 16);
+      int ws = 0, ab = 0;
+      uint32_t ph_w = 0, ph_a = 0;
+      bool ok = true;
+      for (int it = blockIdx.x; it < total && ok; it += gridDim.x) {
+        for (int kb = 0; kb < nkb && ok; ++kb) {
+          ok = __all_sync(0xffffffffu, mbar_wait(&full_w[ws], ph_w, abort_flag, lim));
+          if (!ok) break;
+          const uint8_t* st = smem + ws * C::STAGE;
+          const uint8_t* wrow = st + C::STAGE_W + mat * C::W_TILE + row * 128;
+          const uint4 sc = *reinterpret_cast<const uint4*>(st + C::STAGE_S + mat * C::S_TILE + row * 16);
+          // this thread's packed words of every step of the stage
+          uint4 wv[NSUB];
+          uint2 wq[NSUB];
 #pragma unroll
-        for (int j = 0; j < KB / KS; ++j) {
-          if (j < nsub) {
-            ok = __all_sync(0xffffffffu, mbar_wait(&a_empty[ab], ph_a ^ 1u, abort_flag, lim));
-            if (!ok) break;
-            const uint32_t arow = smem_u32(smem + C::OFF_A + (ab * NA + mat) * C::A_TILE + row * 128);
-#pragma unroll
-            for (int q = 0; q < 2; ++q) {
-              if (GATED || q == half) {
-                const uint4 wv = ld_shared_v4(wrow + (uint32_t)(((2 * j + q) ^ sw) << 4));
-                const __half2 s2 = scale_h2(sc, 2 * j + q);
-                st_shared_v4(arow + (uint32_t)(((4 * q + 0) ^ sw) << 4), dequant_word(wv.x, s2));
-                st_shared_v4(arow + (uint32_t)(((4 * q + 1) ^ sw) << 4), dequant_word(wv.y, s2));
-                st_shared_v4(arow + (uint32_t)(((4 * q + 2) ^ sw) << 4), dequant_word(wv.z, s2));
-                st_shared_v4(arow + (uint32_t)(((4 * q + 3) ^ sw) << 4), dequant_word(wv.w, s2));
-              }
-            }
-            fence_proxy_async_smem();  // generic-proxy smem writes -> visible to the tensor core
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&a_full[ab]);
-            if (++ab == ABUF) {
-              ab = 0;
-              ph_a ^= 1u;
+          for (int j = 0; j < NSUB; ++j) {
+            if constexpr (GATED) {
+              wv[j] = *reinterpret_cast<const uint4*>(wrow + (((2 * j + part) ^ sw) << 4));
+            } else {
+              wq[j] = *reinterpret_cast<const uint2*>(wrow + (((2 * j + (part >> 1)) ^ sw) << 4) + 8 * (part & 1));
             }
           }
+          const int nsub = min(NSUB, (K - kb * KB) / KS);
+#pragma unroll
+          for (int j = 0; j < NSUB; ++j) {
+            if (j < nsub) {
+              ok = __all_sync(0xffffffffu, mbar_wait(&a_empty[ab], ph_a ^ 1u, abort_flag, lim));
+              if (!ok) break;
+              tc_fence_after();  // the MMAs that last read this A slot have completed
+              const uint32_t col = (uint32_t)(C::A_COL0 + (ab * NA + mat) * C::A_COLS);
+              if constexpr (GATED) {
+                const __half2 s2 = scale_h2(sc, 2 * j + part);
+                const uint4 d0 = dequant_word(wv[j].x, s2), d1 = dequant_word(wv[j].y, s2);
+                const uint4 d2 = dequant_word(wv[j].z, s2), d3 = dequant_word(wv[j].w, s2);
+                const uint32_t r[16] = {d0.x, d0.y, d0.z, d0.w, d1.x, d1.y, d1.z, d1.w,
+                                        d2.x, d2.y, d2.z, d2.w, d3.x, d3.y, d3.z, d3.w};
+                tmem_st16(lane_base + col + 16 * part, r);
+              } else {
+                const __half2 s2 = scale_h2(sc, 2 * j + (part >> 1));
+                const uint4 d0 = dequant_word(wq[j].x, s2), d1 = dequant_word(wq[j].y, s2);
+                const uint32_t r[8] = {d0.x, d0.y, d0.z, d0.w, d1.x, d1.y, d1.z, d1.w};
+                tmem_st8(lane_base + col + 8 * part, r);
+              }
+              tmem_st_wait();
+              tc_fence_before();
+              __syncwarp();
+              if (lane == 0) mbar_arrive(&a_full[ab]);
+              if (++ab == ABUF) {
+                ab = 0;
+                ph_a ^= 1u;
+              }
+            }
+          }
+          if (!ok) break;
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&empty_w[ws]);  // every word read from the stage is consumed
+          if (++ws == WST) {
+            ws = 0;
+            ph_w ^= 1u;
+          }
         }
-        if (!ok) break;
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&empty_w[ws]);
-        if (++ws == WST) {
-          ws = 0;
-          ph_w ^= 1u;
+      }
+    } else {
+      // ---------------------------------------------------------------- dequantization -> SMEM
+      // 8 warps.  GATED: thread = one row of the gate (warps 8-11) or up (warps 12-15) tile,
+      // all 64 K of each step; plain: thread = one row, half of each 64-K step.
+      const int dt = threadIdx.x - kDqWarp0 * 32;  // 0..255
+      const int mat = GATED ? (dt >> 7) : 0;
+      const int half = GATED ? 0 : (dt >> 7);
+      const int row = dt & 127;
+      const int sw = row & 7;
+      constexpr int CHK = GATED ? 8 : 4;  // 16-byte chunks of packed words this thread takes per stage
+      int ws = 0, ab = 0;
+      uint32_t ph_w = 0, ph_a = 0;
+      bool ok = true;
+      for (int it = blockIdx.x; it < total && ok; it += gridDim.x) {
+        for (int kb = 0; kb < nkb && ok; ++kb) {
+          ok = __all_sync(0xffffffffu, mbar_wait(&full_w[ws], ph_w, abort_flag, lim));
+          if (!ok) break;
+          const uint8_t* st = smem + ws * C::STAGE;
+          const uint8_t* wrow = st + C::STAGE_W + mat * C::W_TILE + row * 128;
+          const uint4 sc = *reinterpret_cast<const uint4*>(st + C::STAGE_S + mat * C::S_TILE + row * 16);
+          uint4 wv[CHK];
+#pragma unroll
+          for (int c = 0; c < CHK; ++c) {
+            const int lc = GATED ? c : 2 * c + half;  // logical 16-byte chunk (32 K) of the 128-byte row
+            wv[c] = *reinterpret_cast<const uint4*>(wrow + ((lc ^ sw) << 4));
+          }
+          const int nsub = min(NSUB, (K - kb * KB) / KS);
+#pragma unroll
+          for (int j = 0; j < NSUB; ++j) {
+            if (j < nsub) {
+              ok = __all_sync(0xffffffffu, mbar_wait(&a_empty[ab], ph_a ^ 1u, abort_flag, lim));
+              if (!ok) break;
+              uint8_t* arow = smem + C::OFF_A + (ab * NA + mat) * C::A_TILE + row * 128;
+#pragma unroll
+              for (int q = 0; q < 2; ++q) {
+                if (GATED || q == half) {
+                  const uint4 w = GATED ? wv[2 * j + q] : wv[j];
+                  const __half2 s2 = scale_h2(sc, 2 * j + q);
+                  *reinterpret_cast<uint4*>(arow + (((4 * q + 0) ^ sw) << 4)) = dequant_word(w.x, s2);
+                  *reinterpret_cast<uint4*>(arow + (((4 * q + 1) ^ sw) << 4)) = dequant_word(w.y, s2);
+                  *reinterpret_cast<uint4*>(arow + (((4 * q + 2) ^ sw) << 4)) = dequant_word(w.z, s2);
+                  *reinterpret_cast<uint4*>(arow + (((4 * q + 3) ^ sw) << 4)) = dequant_word(w.w, s2);
+                }
+              }
+              fence_proxy_async_smem();  // generic-proxy smem writes -> visible to the tensor core
+              __syncwarp();
+              if (lane == 0) mbar_arrive(&a_full[ab]);
+              if (++ab == ABUF) {
+                ab = 0;
+                ph_a ^= 1u;
+              }
+            }
+          }
+          if (!ok) break;
+          // release the stage only after every word loaded from it has been consumed
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&empty_w[ws]);
+          if (++ws == WST) {
+            ws = 0;
+            ph_w ^= 1u;
+          }
         }
       }
     }
@@ -446,13 +639,21 @@ __global__ void __launch_bounds__(kThreads, 1)
 template <bool GATED, int NMAX>
 cudaError_t launch_t(const W4GemmProblem& pr, cudaStream_t s) {
   using C = Cfg<GATED, NMAX>;
-  CUtensorMap tm_w, tm_b;
+  CUtensorMap tm_w, tm_s, tm_b;
   const uint64_t wrows = (uint64_t)pr.E * pr.rows_per_expert;
   if (encode_tmap_2d(&tm_w, pr.w_q, CU_TENSOR_MAP_DATA_TYPE_INT32, pr.K / 8, wrows, (uint64_t)pr.K / 2, KB / 8, BM,
                      CU_TENSOR_MAP_SWIZZLE_128B) != CUDA_SUCCESS)
     return cudaErrorInvalidValue;
-  if (encode_tmap_2d(&tm_b, pr.act, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, pr.K, (uint64_t)pr.act_rows, (uint64_t)pr.K * 2, KS, 16,
-                     CU_TENSOR_MAP_SWIZZLE_128B) != CUDA_SUCCESS)
+  const int scales_tma = (pr.K % KB) == 0;  // scale rows are then a multiple of 16 bytes
+  if (scales_tma) {
+    if (encode_tmap_2d(&tm_s, pr.w_s, CU_TENSOR_MAP_DATA_TYPE_UINT16, pr.K / 32, wrows, (uint64_t)pr.K / 16, KB / 32,
+                       BM, CU_TENSOR_MAP_SWIZZLE_NONE) != CUDA_SUCCESS)
+      return cudaErrorInvalidValue;
+  } else {
+    tm_s = tm_w;  // unused
+  }
+  if (encode_tmap_2d(&tm_b, pr.act, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, pr.K, (uint64_t)pr.act_rows, (uint64_t)pr.K * 2,
+                     KS, 16, CU_TENSOR_MAP_SWIZZLE_128B) != CUDA_SUCCESS)
     return cudaErrorInvalidValue;
   Params p;
   p.K = pr.K;
@@ -460,6 +661,7 @@ cudaError_t launch_t(const W4GemmProblem& pr, cudaStream_t s) {
   p.rows_per_expert = pr.rows_per_expert;
   p.I = pr.I;
   p.m_tiles = GATED ? pr.I / BM : pr.rows_per_expert / BM;
+  p.scales_tma = scales_tma;
   p.w_s = pr.w_s;
   p.sched = pr.sched;
   p.out = pr.out;
@@ -472,7 +674,7 @@ cudaError_t launch_t(const W4GemmProblem& pr, cudaStream_t s) {
   if (err != cudaSuccess) return err;
   const char* name = GATED ? "w4a16_gemm_gate_up" : "w4a16_gemm_down";
   timing_before(name, s);
-  kern<<<sm_count(), kThreads, smem, s>>>(tm_w, tm_b, p);
+  kern<<<sm_count(), C::THREADS, smem, s>>>(tm_w, tm_s, tm_b, p);
   timing_after(name, s);
   return cudaGetLastError();
 }
@@ -480,11 +682,12 @@ cudaError_t launch_t(const W4GemmProblem& pr, cudaStream_t s) {
 }  // namespace w4
 
 cudaError_t launch_w4a16_gemm(const W4GemmProblem& p, cudaStream_t s) {
+  constexpr int THIN = w4::kThinN;
   if (p.gated) {
-    if (p.nmax <= 64) return w4::launch_t<true, 64>(p, s);
+    if (p.nmax <= THIN) return w4::launch_t<true, THIN>(p, s);
     return w4::launch_t<true, 256>(p, s);
   }
-  if (p.nmax <= 64) return w4::launch_t<false, 64>(p, s);
+  if (p.nmax <= THIN) return w4::launch_t<false, THIN>(p, s);
   return w4::launch_t<false, 256>(p, s);
 }
 
