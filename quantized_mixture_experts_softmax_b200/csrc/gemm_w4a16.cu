@@ -52,10 +52,10 @@ __host__ __device__ constexpr int pow2_at_least(int v) {
 #define MOE_W4_THIN_N 16
 #endif
 #ifndef MOE_W4_GT
-#define MOE_W4_GT 5, 0, 6
+#define MOE_W4_GT 5, 0, 3
 #endif
 #ifndef MOE_W4_PT
-#define MOE_W4_PT 8, 0, 8
+#define MOE_W4_PT 8, 0, 6
 #endif
 #ifndef MOE_W4_GW
 #define MOE_W4_GW 2, 2, 2
@@ -101,8 +101,12 @@ struct Cfg {
   static constexpr int ACC_COLS = NA * CH * NMAX;
   static constexpr int ACC_BUFS = (2 * ACC_COLS <= 512) ? 2 : 1;
   static constexpr int A_COLS = KS / 2;                 // one 64-K fp16 row = 32 TMEM columns
+  // thin: an A slot holds SPS consecutive 64-K steps of every matrix, handed over with one
+  // barrier round trip and one commit
+  static constexpr int SPS = A_TMEM ? 2 : 1;
+  static constexpr int SLOT_COLS = NA * SPS * A_COLS;   // [matrix][step][32 columns]
   static constexpr int A_COL0 = ACC_BUFS * ACC_COLS;    // first TMEM column of the A ring
-  static constexpr int TMEM_COLS = pow2_at_least(A_COL0 + (A_TMEM ? ABUF * NA * A_COLS : 0));
+  static constexpr int TMEM_COLS = pow2_at_least(A_COL0 + (A_TMEM ? ABUF * SLOT_COLS : 0));
   static constexpr int OFF_A = WST * STAGE;
   static constexpr int OFF_B = OFF_A + (A_TMEM ? 0 : ABUF * NA * A_TILE);  // wide activation ring
   static constexpr int OFF_BAR = OFF_B + BST * B_ATOM;
@@ -111,7 +115,8 @@ struct Cfg {
   static constexpr int OFF_PREFIX = OFF_MISC + 16;
   static_assert(STAGE % 1024 == 0 && STAGE_B % 1024 == 0 && OFF_A % 1024 == 0 && OFF_B % 1024 == 0,
                 "swizzled tiles need 1024-byte alignment");
-  static_assert(A_COL0 + (A_TMEM ? ABUF * NA * A_COLS : 0) <= 512, "TMEM has 512 columns");
+  static_assert(A_COL0 + (A_TMEM ? ABUF * SLOT_COLS : 0) <= 512, "TMEM has 512 columns");
+  static_assert(NSUB % SPS == 0, "whole slots per stage");
   static constexpr size_t smem_bytes(int E) { return (size_t)OFF_PREFIX + 4 * (size_t)(E + 1) + 1024; }
   static_assert(smem_bytes(1024) <= 232448, "shared memory budget");
   static_assert(!THIN || A_TMEM, "the thin variant keeps A in tensor memory");
@@ -347,23 +352,28 @@ __global__ void __launch_bounds__(Cfg<GATED, NMAX>::THREADS, 1)
         for (int kb = 0; kb < nkb && ok; ++kb) {
           const int nsub = min(NSUB, (K - kb * KB) / KS);
           if (THIN && !(ok = mbar_wait(&full_w[ws], ph_w, abort_flag, lim))) break;
-          for (int j = 0; j < nsub; ++j) {
+          for (int j = 0; j < nsub; j += C::SPS) {
             if (!(ok = mbar_wait(&a_full[ab], ph_a, abort_flag, lim))) break;
             if (!THIN && !(ok = mbar_wait(&full_b[bs], ph_b, abort_flag, lim))) break;
             tc_fence_after();
-            const uint8_t* bt = THIN ? smem + ws * C::STAGE + C::STAGE_B + j * C::B_ATOM : smem + C::OFF_B + bs * C::B_ATOM;
-            const uint64_t b = sw128_kmajor_desc(smem_u32(bt));
             if constexpr (C::A_TMEM) {
               constexpr int CH = C::CH;
-              const uint32_t a0 = tmem_base + (uint32_t)(C::A_COL0 + ab * NA * C::A_COLS);
+              const uint32_t slot = tmem_base + (uint32_t)(C::A_COL0 + ab * C::SLOT_COLS);
 #pragma unroll
-              for (int kk = 0; kk < KS / 16; ++kk) {
-                const uint32_t accum = (kb | j | (kk / CH)) != 0;  // each chain starts fresh at K = 0
-                const uint32_t dc = d0 + (uint32_t)((kk % CH) * NMAX);
-                umma_f16_ts(dc, a0 + 8 * kk, b + 2 * kk, idesc, accum);  // 16 K = 8 columns / 32 bytes
-                if (GATED) umma_f16_ts(dc + CH * NMAX, a0 + C::A_COLS + 8 * kk, b + 2 * kk, idesc, accum);
+              for (int s2 = 0; s2 < C::SPS; ++s2) {
+                const uint64_t b = sw128_kmajor_desc(smem_u32(smem + ws * C::STAGE + C::STAGE_B + (j + s2) * C::B_ATOM));
+#pragma unroll
+                for (int kk = 0; kk < KS / 16; ++kk) {
+                  const uint32_t accum = (kb | j | s2 | (kk / CH)) != 0;  // each chain starts fresh at K = 0
+                  const uint32_t dc = d0 + (uint32_t)((kk % CH) * NMAX);
+                  const uint32_t a = slot + (uint32_t)(s2 * C::A_COLS + 8 * kk);  // 16 K = 8 columns
+                  umma_f16_ts(dc, a, b + 2 * kk, idesc, accum);
+                  if (GATED) umma_f16_ts(dc + CH * NMAX, a + C::SPS * C::A_COLS, b + 2 * kk, idesc, accum);
+                }
               }
             } else {
+              const uint8_t* bt = THIN ? smem + ws * C::STAGE + C::STAGE_B + j * C::B_ATOM : smem + C::OFF_B + bs * C::B_ATOM;
+              const uint64_t b = sw128_kmajor_desc(smem_u32(bt));
               const uint64_t a0 = sw128_kmajor_desc(smem_u32(smem + C::OFF_A + (ab * NA + 0) * C::A_TILE));
               const uint64_t a1 = sw128_kmajor_desc(smem_u32(smem + C::OFF_A + (ab * NA + (NA - 1)) * C::A_TILE));
 #pragma unroll
@@ -524,24 +534,29 @@ __global__ void __launch_bounds__(Cfg<GATED, NMAX>::THREADS, 1)
           }
           const int nsub = min(NSUB, (K - kb * KB) / KS);
 #pragma unroll
-          for (int j = 0; j < NSUB; ++j) {
-            if (j < nsub) {
+          for (int j0 = 0; j0 < NSUB; j0 += C::SPS) {
+            if (j0 < nsub) {
               ok = __all_sync(0xffffffffu, mbar_wait(&a_empty[ab], ph_a ^ 1u, abort_flag, lim));
               if (!ok) break;
               tc_fence_after();  // the MMAs that last read this A slot have completed
-              const uint32_t col = (uint32_t)(C::A_COL0 + (ab * NA + mat) * C::A_COLS);
-              if constexpr (GATED) {
-                const __half2 s2 = scale_h2(sc, 2 * j + part);
-                const uint4 d0 = dequant_word(wv[j].x, s2), d1 = dequant_word(wv[j].y, s2);
-                const uint4 d2 = dequant_word(wv[j].z, s2), d3 = dequant_word(wv[j].w, s2);
-                const uint32_t r[16] = {d0.x, d0.y, d0.z, d0.w, d1.x, d1.y, d1.z, d1.w,
-                                        d2.x, d2.y, d2.z, d2.w, d3.x, d3.y, d3.z, d3.w};
-                tmem_st16(lane_base + col + 16 * part, r);
-              } else {
-                const __half2 s2 = scale_h2(sc, 2 * j + (part >> 1));
-                const uint4 d0 = dequant_word(wq[j].x, s2), d1 = dequant_word(wq[j].y, s2);
-                const uint32_t r[8] = {d0.x, d0.y, d0.z, d0.w, d1.x, d1.y, d1.z, d1.w};
-                tmem_st8(lane_base + col + 8 * part, r);
+              const uint32_t slot = (uint32_t)(C::A_COL0 + ab * C::SLOT_COLS + mat * C::SPS * C::A_COLS);
+#pragma unroll
+              for (int s2 = 0; s2 < C::SPS; ++s2) {
+                const int j = j0 + s2;
+                const uint32_t col = slot + (uint32_t)(s2 * C::A_COLS);
+                if constexpr (GATED) {
+                  const __half2 sc2 = scale_h2(sc, 2 * j + part);
+                  const uint4 d0 = dequant_word(wv[j].x, sc2), d1 = dequant_word(wv[j].y, sc2);
+                  const uint4 d2 = dequant_word(wv[j].z, sc2), d3 = dequant_word(wv[j].w, sc2);
+                  const uint32_t r[16] = {d0.x, d0.y, d0.z, d0.w, d1.x, d1.y, d1.z, d1.w,
+                                          d2.x, d2.y, d2.z, d2.w, d3.x, d3.y, d3.z, d3.w};
+                  tmem_st16(lane_base + col + 16 * part, r);
+                } else {
+                  const __half2 sc2 = scale_h2(sc, 2 * j + (part >> 1));
+                  const uint4 d0 = dequant_word(wq[j].x, sc2), d1 = dequant_word(wq[j].y, sc2);
+                  const uint32_t r[8] = {d0.x, d0.y, d0.z, d0.w, d1.x, d1.y, d1.z, d1.w};
+                  tmem_st8(lane_base + col + 8 * part, r);
+                }
               }
               tmem_st_wait();
               tc_fence_before();
