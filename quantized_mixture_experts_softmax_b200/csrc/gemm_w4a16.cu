@@ -84,7 +84,13 @@ struct Cfg {
   // the thin variant spreads each matrix's K steps over CH independent accumulators (summed
   // in the epilogue) so that 4 MMAs are in flight.
   static constexpr int CH = THIN ? 4 / NA : 1;
-  static constexpr int NDQ = THIN ? 16 : 8;  // dequantization warps
+#ifndef MOE_W4_THIN_DQ
+#define MOE_W4_THIN_DQ 8
+#endif
+  static constexpr int NDQ = THIN ? MOE_W4_THIN_DQ : 8;  // dequantization warps
+  // thin: each thread dequantizes one row and 1/PARTS of every 64-K step
+  static constexpr int PARTS = THIN ? NDQ / (4 * NA) : 1;
+  static_assert(!THIN || (PARTS >= 1 && 8 % PARTS == 0 && NDQ == 4 * NA * PARTS), "thin dequant split");
   static constexpr int THREADS = (kDqWarp0 + NDQ) * 32;
   static constexpr int WST = depths<GATED, THIN>().wst;
   static constexpr int BST = THIN ? 0 : depths<GATED, THIN>().bst;
@@ -508,8 +514,10 @@ __global__ void __launch_bounds__(Cfg<GATED, NMAX>::THREADS, 1)
       const int dw = warp - kDqWarp0;
       const int row = (dw & 3) * 32 + lane;
       const int sw = row & 7;
-      const int mat = GATED ? (dw >> 3) : 0;
-      const int part = GATED ? ((dw >> 2) & 1) : (dw >> 2);  // K half (GATED) or quarter (plain)
+      constexpr int PARTS = C::PARTS;
+      constexpr int WPS = 8 / PARTS;  // packed words of each 64-K step this thread takes
+      const int mat = GATED ? (dw / (4 * PARTS)) : 0;
+      const int part = (dw >> 2) % PARTS;  // which 1/PARTS of the step
       const uint32_t lane_base = tmem_base + ((uint32_t)((dw & 3) * 32) << 16);
       int ws = 0, ab = 0;
       uint32_t ph_w = 0, ph_a = 0;
@@ -521,15 +529,26 @@ __global__ void __launch_bounds__(Cfg<GATED, NMAX>::THREADS, 1)
           const uint8_t* st = smem + ws * C::STAGE;
           const uint8_t* wrow = st + C::STAGE_W + mat * C::W_TILE + row * 128;
           const uint4 sc = *reinterpret_cast<const uint4*>(st + C::STAGE_S + mat * C::S_TILE + row * 16);
-          // this thread's packed words of every step of the stage
-          uint4 wv[NSUB];
-          uint2 wq[NSUB];
+          // this thread's packed words of every step of the stage: step j = bytes 32j..32j+31
+          // of the row (before the swizzle), of which this thread takes words
+          // part*WPS .. part*WPS+WPS-1
+          uint32_t wv[NSUB][WPS];
 #pragma unroll
           for (int j = 0; j < NSUB; ++j) {
-            if constexpr (GATED) {
-              wv[j] = *reinterpret_cast<const uint4*>(wrow + (((2 * j + part) ^ sw) << 4));
-            } else {
-              wq[j] = *reinterpret_cast<const uint2*>(wrow + (((2 * j + (part >> 1)) ^ sw) << 4) + 8 * (part & 1));
+#pragma unroll
+            for (int c = 0; c < WPS; c += 4 > WPS ? WPS : 4) {
+              const int w0 = part * WPS + c;              // first word within the step (0..7)
+              const int lc = 2 * j + (w0 >> 2);           // logical 16-byte chunk
+              const uint8_t* src = wrow + ((lc ^ sw) << 4) + 4 * (w0 & 3);
+              if constexpr (WPS >= 4) {
+                const uint4 v = *reinterpret_cast<const uint4*>(src);
+                wv[j][c] = v.x, wv[j][c + 1] = v.y, wv[j][c + 2] = v.z, wv[j][c + 3] = v.w;
+              } else if constexpr (WPS == 2) {
+                const uint2 v = *reinterpret_cast<const uint2*>(src);
+                wv[j][c] = v.x, wv[j][c + 1] = v.y;
+              } else {
+                wv[j][c] = *reinterpret_cast<const uint32_t*>(src);
+              }
             }
           }
           const int nsub = min(NSUB, (K - kb * KB) / KS);
@@ -543,20 +562,20 @@ __global__ void __launch_bounds__(Cfg<GATED, NMAX>::THREADS, 1)
 #pragma unroll
               for (int s2 = 0; s2 < C::SPS; ++s2) {
                 const int j = j0 + s2;
-                const uint32_t col = slot + (uint32_t)(s2 * C::A_COLS);
-                if constexpr (GATED) {
-                  const __half2 sc2 = scale_h2(sc, 2 * j + part);
-                  const uint4 d0 = dequant_word(wv[j].x, sc2), d1 = dequant_word(wv[j].y, sc2);
-                  const uint4 d2 = dequant_word(wv[j].z, sc2), d3 = dequant_word(wv[j].w, sc2);
-                  const uint32_t r[16] = {d0.x, d0.y, d0.z, d0.w, d1.x, d1.y, d1.z, d1.w,
-                                          d2.x, d2.y, d2.z, d2.w, d3.x, d3.y, d3.z, d3.w};
-                  tmem_st16(lane_base + col + 16 * part, r);
-                } else {
-                  const __half2 sc2 = scale_h2(sc, 2 * j + (part >> 1));
-                  const uint4 d0 = dequant_word(wq[j].x, sc2), d1 = dequant_word(wq[j].y, sc2);
-                  const uint32_t r[8] = {d0.x, d0.y, d0.z, d0.w, d1.x, d1.y, d1.z, d1.w};
-                  tmem_st8(lane_base + col + 8 * part, r);
+                const uint32_t col = slot + (uint32_t)(s2 * C::A_COLS + part * WPS * 4);
+                uint32_t r[WPS * 4];
+#pragma unroll
+                for (int w = 0; w < WPS; ++w) {
+                  const __half2 sc2 = scale_h2(sc, 2 * j + ((part * WPS + w) >> 2));  // 32 K per scale
+                  const uint4 d = dequant_word(wv[j][w], sc2);
+                  r[4 * w + 0] = d.x, r[4 * w + 1] = d.y, r[4 * w + 2] = d.z, r[4 * w + 3] = d.w;
                 }
+                if constexpr (WPS == 8)
+                  tmem_st32(lane_base + col, r);
+                else if constexpr (WPS == 4)
+                  tmem_st16(lane_base + col, r);
+                else
+                  tmem_st8(lane_base + col, r);
               }
               tmem_st_wait();
               tc_fence_before();
