@@ -171,6 +171,31 @@ GemmWs carve_gemm(void* ws, int M, int K, int E) {
   return w;
 }
 // token-tile height cap: thin variant (w4::kThinN rows) when no expert can exceed 64 rows
+struct F8Ws {
+  int32_t *counts, *offsets, *sorted, *inv, *blockcnt, *tile_prefix, *chunk;
+  uint8_t *x_perm, *h;
+  float *xs_t, *hs_t, *y;
+  size_t bytes;
+};
+F8Ws carve_fp8_forward(void* ws, int T, int H, int I, int E, int k) {
+  Carver c(ws);
+  F8Ws w;
+  const size_t P = (size_t)T * k;
+  w.counts = c.take<int32_t>(E);
+  w.offsets = c.take<int32_t>(E + 1);
+  w.sorted = c.take<int32_t>(P);
+  w.inv = c.take<int32_t>(P);
+  w.blockcnt = c.take<int32_t>((size_t)align_blocks(T, k) * E);
+  w.tile_prefix = c.take<int32_t>(E + 1);
+  w.chunk = c.take<int32_t>(E);
+  w.x_perm = c.take<uint8_t>(P * H);
+  w.xs_t = c.take<float>((size_t)(H / 128) * P);
+  w.h = c.take<uint8_t>(P * I);
+  w.hs_t = c.take<float>((size_t)(I / 128) * P);
+  w.y = c.take<float>(P * H);
+  w.bytes = c.off + 256;
+  return w;
+}
 int pick_nmax(int max_rows_per_expert) { return max_rows_per_expert <= 64 ? w4::kThinN : 256; }
 
 bool shape_ok(int T, int H, int I, int E, int k) {
@@ -272,13 +297,37 @@ moe_status_t moe_w4a16_forward(const moe_w4a16_args* a, void* ws, size_t ws_byte
 }
 
 size_t moe_blockfp8_workspace_size(int T, int H, int I, int E, int k) {
-  (void)T, (void)H, (void)I, (void)E, (void)k;
-  return 0;
+  if (!shape_ok(T, H, I, E, k)) return 0;
+  return carve_fp8_forward(nullptr, T, H, I, E, k).bytes;
 }
 
 moe_status_t moe_blockfp8_forward(const moe_blockfp8_args* a, void* ws, size_t ws_bytes, cudaStream_t stream) {
-  (void)a, (void)ws, (void)ws_bytes, (void)stream;
-  return MOE_ERR_UNSUPPORTED;
+  if (!a) return MOE_ERR_INVALID_ARG;
+  if (!shape_ok(a->T, a->H, a->I, a->E, a->k)) return MOE_ERR_UNSUPPORTED;
+  if (!aligned(a->x, 16) || !aligned(a->xs, 4) || !aligned(a->topk_ids, 4) || !aligned(a->topk_w, 4) ||
+      !aligned(a->w13, 16) || !aligned(a->w13_s, 4) || !aligned(a->w2, 16) || !aligned(a->w2_s, 4) ||
+      !aligned(a->out, 16) || !aligned(ws, 256))
+    return MOE_ERR_INVALID_ARG;
+  const int T = a->T, H = a->H, I = a->I, E = a->E, k = a->k;
+  if (ws_bytes < moe_blockfp8_workspace_size(T, H, I, E, k)) return MOE_ERR_WORKSPACE;
+  if (moe_status_t st = check_device()) return st;
+  const F8Ws w = carve_fp8_forward(ws, T, H, I, E, k);
+  const int P = T * k;
+  const int nmax = 32;  // the FP8 GEMM's token tile
+  cudaError_t e = launch_align(a->topk_ids, T, k, E, 1, w.counts, w.offsets, w.sorted, w.inv, w.blockcnt, nmax,
+                               w.tile_prefix, w.chunk, stream);
+  if (e == cudaSuccess) e = launch_permute_fp8(a->x, a->xs, w.inv, T, k, H, w.x_perm, w.xs_t, P, stream);
+  const TileSched sched{w.offsets, w.counts, w.tile_prefix, w.chunk};
+  if (e == cudaSuccess) {
+    F8GemmProblem g{a->w13, a->w13_s, w.x_perm, w.xs_t, P, H, E, 2 * I, true, I, sched, w.h, I, w.hs_t};
+    e = launch_fp8_gemm(g, stream);
+  }
+  if (e == cudaSuccess) {
+    F8GemmProblem g{a->w2, a->w2_s, w.h, w.hs_t, P, I, E, H, false, 0, sched, w.y, H, nullptr};
+    e = launch_fp8_gemm(g, stream);
+  }
+  if (e == cudaSuccess) e = launch_combine(w.y, w.inv, a->topk_w, T, k, H, a->out, a->out_fp32, stream);
+  return e == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
 }
 
 size_t moe_w4a16_gemm_workspace_size(int M, int K, int N, int E) {

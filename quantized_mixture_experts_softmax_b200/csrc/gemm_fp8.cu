@@ -1,0 +1,358 @@
+// a9: block-FP8 grouped expert GEMM (e4m3 x e4m3 on tcgen05 kind::f8f6f4, fp32 promotion).
+//
+// The format (the Helion article, "Scope: Hopper and quantized formats"): activations carry one
+// fp32 scale per 1x128 group of K, weights one fp32 scale per 128x128 block.  A 128-K block of
+// the reduction therefore has a single weight scale per 128-row weight tile and one activation
+// scale per token, so each block's partial product is computed on the tensor cores in its own
+// TMEM tile and promoted on the CUDA cores:
+//     acc[row][tok] += P_kb[row][tok] * (w_scale[tile][kb] * x_scale[tok][kb]).
+//
+// One persistent CTA per SM over the same (expert, 128-row weight tile, token tile) work list as
+// the W4A16 GEMM, weights swapped into the MMA's M slot.  Warp roles (256 threads):
+//   warp 0      TMA producer: e4m3 weight tiles (128 rows x 128 K, 128-byte swizzle; gate and up
+//               tiles for the gate/up GEMM) and the token tile's activations, one stage per
+//               128-K block;
+//   warp 1      TMEM allocator and single-thread MMA issuer: four K=32 MMAs per matrix per block
+//               into a double-buffered partial-product tile;
+//   warps 4-7   promotion and epilogue: each thread owns one weight row and keeps its tokens'
+//               fp32 accumulators in registers.  The gate/up GEMM ends with h = SiLU(gate) * up,
+//               requantized per (token, 128-column group) - the tile's 128 rows are exactly one
+//               group - to e4m3 with s = max(amax, 1e-10) / 448; the down GEMM stores fp32.
+#include <cuda_fp8.h>
+
+#include "common.cuh"
+#include "internal.h"
+
+namespace moe {
+namespace f8 {
+
+constexpr int BM = 128;   // weight rows per tile (MMA M)
+constexpr int KB = 128;   // K per stage = one scale block
+constexpr int NMAX = 32;  // token rows per tile
+constexpr int kThreads = 256;
+constexpr int kEpiWarp0 = 4;
+
+template <bool GATED>
+struct Cfg {
+  static constexpr int NA = GATED ? 2 : 1;
+  static constexpr int W_TILE = BM * KB;    // e4m3 bytes
+  static constexpr int B_TILE = NMAX * KB;  // activation bytes
+  static constexpr int STAGE = NA * W_TILE + B_TILE;
+  static constexpr int ST = GATED ? 6 : 10;
+  static constexpr int P_COLS = NA * NMAX;  // one partial-product tile: [matrix][NMAX] columns
+  static constexpr int TMEM_COLS = 2 * P_COLS <= 32 ? 32 : (2 * P_COLS <= 64 ? 64 : 128);
+  static constexpr int OFF_BAR = ST * STAGE;
+  static constexpr int NUM_BARS = 2 * ST + 4 + 2;
+  static constexpr int OFF_MISC = OFF_BAR + NUM_BARS * 8;
+  static constexpr int OFF_RED = OFF_MISC + 16;              // [4 warps][NMAX] amax partials
+  static constexpr int OFF_PREFIX = OFF_RED + 4 * NMAX * 4;
+  static_assert(STAGE % 1024 == 0, "swizzled tiles need 1024-byte alignment");
+  static constexpr size_t smem_bytes(int E) { return (size_t)OFF_PREFIX + 4 * (size_t)(E + 1) + 1024; }
+  static_assert(smem_bytes(1024) <= 232448, "shared memory budget");
+};
+
+struct Params {
+  int K, E, rows_per_expert, I, m_tiles;
+  const float* w_scale;  // [E, rows_per_expert/128, K/128]
+  const float* x_scale;  // transposed activation scales [K/128, act_rows]
+  int act_rows;
+  TileSched sched;
+  void* out;  // GATED: e4m3 h [act_rows, I]; else fp32 y [act_rows, out_ld]
+  int out_ld;
+  float* h_scale;  // GATED: transposed scales of h [I/128, act_rows]
+  uint64_t wait_limit;
+};
+
+struct Item {
+  int e, m, r0, nvalid, nmma;
+};
+
+__device__ __forceinline__ Item decode_item(int it, const int* __restrict__ sprefix, const Params& p) {
+  Item I;
+  const int tile = it / p.m_tiles;
+  int lo = 0, hi = p.E;  // sprefix[lo] <= tile < sprefix[hi]
+  while (hi - lo > 1) {
+    const int mid = (lo + hi) >> 1;
+    if (sprefix[mid] <= tile)
+      lo = mid;
+    else
+      hi = mid;
+  }
+  I.e = lo;
+  const int nt = sprefix[lo + 1] - sprefix[lo];
+  const int local = it - p.m_tiles * sprefix[lo];
+  I.m = local / nt;
+  const int t = local - I.m * nt;
+  const int ch = __ldg(p.sched.chunk + lo);
+  const int cnt = __ldg(p.sched.row_count + lo);
+  I.r0 = __ldg(p.sched.row_start + lo) + t * ch;
+  I.nvalid = min(ch, cnt - t * ch);
+  I.nmma = (I.nvalid + 15) & ~15;
+  return I;
+}
+
+// Bounded barrier among the 4 epilogue warps (an mbarrier of count 4, alternating phases).
+__device__ __forceinline__ bool epi_sync(uint64_t* bar, uint32_t& phase, volatile int* abort, uint64_t lim) {
+  __syncwarp();
+  if ((threadIdx.x & 31) == 0) mbar_arrive(bar);
+  const bool ok = __all_sync(0xffffffffu, mbar_wait(bar, phase, abort, lim));
+  phase ^= 1u;
+  return ok;
+}
+
+template <bool GATED>
+__global__ void __launch_bounds__(kThreads, 1)
+    fp8_gemm_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CUtensorMap tm_b,
+                    const Params p) {
+  using C = Cfg<GATED>;
+  constexpr int NA = C::NA, ST = C::ST;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + C::OFF_BAR);
+  uint64_t* empty = full + ST;
+  uint64_t* p_full = empty + ST;
+  uint64_t* p_empty = p_full + 2;
+  uint64_t* drain = p_empty + 2;
+  uint64_t* epi_bar = drain + 1;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::OFF_MISC);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::OFF_MISC + 4);
+  float* red = reinterpret_cast<float*>(smem + C::OFF_RED);
+  int* sprefix = reinterpret_cast<int*>(smem + C::OFF_PREFIX);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const uint64_t lim = p.wait_limit;
+
+  for (int i = threadIdx.x; i <= p.E; i += blockDim.x) sprefix[i] = __ldg(p.sched.tile_prefix + i);
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < ST; ++i) {
+      mbar_init(&full[i], 1);
+      mbar_init(&empty[i], 1);
+    }
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&p_full[i], 1);
+      mbar_init(&p_empty[i], 4);
+    }
+    mbar_init(drain, 1);
+    mbar_init(epi_bar, 4);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 0 && lane == 0) {
+    prefetch_tmap(&tm_w);
+    prefetch_tmap(&tm_b);
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_slot, C::TMEM_COLS);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+  const int total = p.m_tiles * sprefix[p.E];
+  const int nkb = p.K / KB;
+
+  if (warp == 0) {
+    // ---------------------------------------------------------------- producer
+    if (lane == 0) {
+      const uint64_t pol_w = policy_evict_first();
+      const uint64_t pol_b = policy_evict_last();
+      int s = 0, issued = 0;
+      uint32_t ph = 0;
+      bool ok = true;
+      for (int it = blockIdx.x; it < total && ok; it += gridDim.x) {
+        const Item I = decode_item(it, sprefix, p);
+        const int row_g = I.e * p.rows_per_expert + I.m * BM;
+        const int row_u = row_g + p.I;
+        for (int kb = 0; kb < nkb; ++kb) {
+          if (!(ok = mbar_wait(&empty[s], ph ^ 1u, abort_flag, lim))) break;
+          uint8_t* st = smem + s * C::STAGE;
+          mbar_arrive_expect_tx(&full[s], (uint32_t)(NA * C::W_TILE + I.nmma * KB));
+          tma_load_2d_hint(st, &tm_w, &full[s], kb * KB, row_g, pol_w);
+          if (GATED) tma_load_2d_hint(st + C::W_TILE, &tm_w, &full[s], kb * KB, row_u, pol_w);
+          for (int r = 0; r < I.nmma; r += 16)
+            tma_load_2d_hint(st + NA * C::W_TILE + r * 128, &tm_b, &full[s], kb * KB, I.r0 + r, pol_b);
+          ++issued;
+          if (++s == ST) {
+            s = 0;
+            ph ^= 1u;
+          }
+        }
+      }
+      for (int i = max(0, issued - ST); i < issued; ++i) mbar_wait_plain(&full[i % ST], (i / ST) & 1, lim);
+    }
+  } else if (warp == 1) {
+    // ---------------------------------------------------------------- MMA issuer
+    if (lane == 0) {
+      int s = 0, pb = 0;
+      uint32_t ph = 0, ph_p = 0;
+      bool ok = true;
+      for (int it = blockIdx.x; it < total && ok; it += gridDim.x) {
+        const Item I = decode_item(it, sprefix, p);
+        const uint32_t idesc = make_idesc(BM, I.nmma, 0, 0);  // e4m3 x e4m3 -> fp32
+        for (int kb = 0; kb < nkb; ++kb) {
+          if (!(ok = mbar_wait(&full[s], ph, abort_flag, lim))) break;
+          if (!(ok = mbar_wait(&p_empty[pb], ph_p ^ 1u, abort_flag, lim))) break;
+          tc_fence_after();
+          const uint8_t* st = smem + s * C::STAGE;
+          const uint64_t a0 = sw128_kmajor_desc(smem_u32(st));
+          const uint64_t a1 = sw128_kmajor_desc(smem_u32(st + (NA - 1) * C::W_TILE));
+          const uint64_t b = sw128_kmajor_desc(smem_u32(st + NA * C::W_TILE));
+          const uint32_t d = tmem_base + (uint32_t)(pb * C::P_COLS);
+#pragma unroll
+          for (int kk = 0; kk < KB / 32; ++kk) {  // K = 32 e4m3 = 32 bytes per MMA
+            umma_f8(d, a0 + 2 * kk, b + 2 * kk, idesc, kk != 0);
+            if (GATED) umma_f8(d + NMAX, a1 + 2 * kk, b + 2 * kk, idesc, kk != 0);
+          }
+          umma_commit(&p_full[pb]);
+          umma_commit(&empty[s]);
+          if (++s == ST) {
+            s = 0;
+            ph ^= 1u;
+          }
+          if (++pb == 2) {
+            pb = 0;
+            ph_p ^= 1u;
+          }
+        }
+      }
+      umma_commit(drain);
+      mbar_wait_plain(drain, 0, lim);
+    }
+  } else if (warp >= kEpiWarp0) {
+    // ---------------------------------------------------------------- promotion + epilogue
+    const int ew = warp - kEpiWarp0;  // == warp % 4: TMEM lanes 32*ew..32*ew+31
+    const int mrow = ew * 32 + lane;
+    const int GK = p.K / KB;
+    int pb = 0;
+    uint32_t ph_p = 0, ph_e = 0;
+    bool ok = true;
+    for (int it = blockIdx.x; it < total && ok; it += gridDim.x) {
+      const Item I = decode_item(it, sprefix, p);
+      float ag[NMAX], au[NMAX];
+#pragma unroll
+      for (int c = 0; c < NMAX; ++c) ag[c] = au[c] = 0.f;
+      const float* wsg = p.w_scale + ((size_t)I.e * (p.rows_per_expert / BM) + I.m) * GK;
+      const float* wsu = GATED ? wsg + (size_t)(p.I / BM) * GK : wsg;
+      for (int kb = 0; kb < nkb; ++kb) {
+        // this block's per-token activation scales: lane c holds token c's
+        const float xs_l = (lane < I.nvalid) ? __ldg(p.x_scale + (size_t)kb * p.act_rows + I.r0 + lane) : 0.f;
+        const float sg = __ldg(wsg + kb), su = GATED ? __ldg(wsu + kb) : 0.f;
+        ok = __all_sync(0xffffffffu, mbar_wait(&p_full[pb], ph_p, abort_flag, lim));
+        if (!ok) break;
+        tc_fence_after();
+        const uint32_t tb = tmem_base + ((uint32_t)(ew * 32) << 16) + (uint32_t)(pb * C::P_COLS);
+        uint32_t pg[16], pu[16];
+#pragma unroll
+        for (int c0 = 0; c0 < NMAX; c0 += 16) {
+          if (c0 < I.nmma) {
+            tmem_ld16(tb + c0, pg);
+            if (GATED) tmem_ld16(tb + NMAX + c0, pu);
+            tmem_ld_wait();
+#pragma unroll
+            for (int i = 0; i < 16; ++i) {
+              const float xs = __shfl_sync(0xffffffffu, xs_l, c0 + i);
+              ag[c0 + i] = fmaf(__uint_as_float(pg[i]), sg * xs, ag[c0 + i]);
+              if (GATED) au[c0 + i] = fmaf(__uint_as_float(pu[i]), su * xs, au[c0 + i]);
+            }
+          }
+        }
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&p_empty[pb]);
+        if (++pb == 2) {
+          pb = 0;
+          ph_p ^= 1u;
+        }
+      }
+      if (!ok) break;
+      if constexpr (GATED) {
+        // h = SiLU(gate) * up; requantize each token's 128 values of this tile (one 1x128 group)
+        float amax[NMAX];
+#pragma unroll
+        for (int c = 0; c < NMAX; ++c) {
+          const float h = ag[c] / (1.0f + __expf(-ag[c])) * au[c];
+          ag[c] = h;
+          float m = fabsf(h);
+#pragma unroll
+          for (int off = 16; off; off >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, off));
+          amax[c] = m;
+        }
+        if (lane == 0)
+#pragma unroll
+          for (int c = 0; c < NMAX; ++c) red[ew * NMAX + c] = amax[c];
+        if (!(ok = epi_sync(epi_bar, ph_e, abort_flag, lim))) break;
+        uint8_t* hq = reinterpret_cast<uint8_t*>(p.out);
+        const int j = I.m * BM + mrow;
+#pragma unroll
+        for (int c = 0; c < NMAX; ++c) {
+          if (c < I.nvalid) {
+            const float a = fmaxf(fmaxf(red[c], red[NMAX + c]), fmaxf(red[2 * NMAX + c], red[3 * NMAX + c]));
+            const float sc = __fdiv_rn(fmaxf(a, 1e-10f), 448.0f);
+            const __nv_fp8_e4m3 q(__fdiv_rn(ag[c], sc));  // round to nearest even, saturating
+            hq[(size_t)(I.r0 + c) * p.out_ld + j] = *reinterpret_cast<const uint8_t*>(&q);
+            if (mrow == 0) p.h_scale[(size_t)I.m * p.act_rows + I.r0 + c] = sc;
+          }
+        }
+        if (!(ok = epi_sync(epi_bar, ph_e, abort_flag, lim))) break;  // red[] is reused by the next item
+      } else {
+        float* y = reinterpret_cast<float*>(p.out);
+        const int n = I.m * BM + mrow;
+#pragma unroll
+        for (int c = 0; c < NMAX; ++c)
+          if (c < I.nvalid) y[(size_t)(I.r0 + c) * p.out_ld + n] = ag[c];
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem_base, C::TMEM_COLS);
+  }
+}
+
+template <bool GATED>
+cudaError_t launch_t(const F8GemmProblem& pr, cudaStream_t s) {
+  using C = Cfg<GATED>;
+  CUtensorMap tm_w, tm_b;
+  const uint64_t wrows = (uint64_t)pr.E * pr.rows_per_expert;
+  if (encode_tmap_2d(&tm_w, pr.w, CU_TENSOR_MAP_DATA_TYPE_UINT8, pr.K, wrows, (uint64_t)pr.K, KB, BM,
+                     CU_TENSOR_MAP_SWIZZLE_128B) != CUDA_SUCCESS)
+    return cudaErrorInvalidValue;
+  if (encode_tmap_2d(&tm_b, pr.act, CU_TENSOR_MAP_DATA_TYPE_UINT8, pr.K, (uint64_t)pr.act_rows, (uint64_t)pr.K, KB,
+                     16, CU_TENSOR_MAP_SWIZZLE_128B) != CUDA_SUCCESS)
+    return cudaErrorInvalidValue;
+  Params p;
+  p.K = pr.K;
+  p.E = pr.E;
+  p.rows_per_expert = pr.rows_per_expert;
+  p.I = pr.I;
+  p.m_tiles = GATED ? pr.I / BM : pr.rows_per_expert / BM;
+  p.w_scale = pr.w_scale;
+  p.x_scale = pr.x_scale;
+  p.act_rows = pr.act_rows;
+  p.sched = pr.sched;
+  p.out = pr.out;
+  p.out_ld = pr.out_ld;
+  p.h_scale = pr.h_scale;
+  p.wait_limit = wait_limit_ns();
+  const size_t smem = C::smem_bytes(pr.E);
+  auto kern = fp8_gemm_kernel<GATED>;
+  cudaError_t err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (err != cudaSuccess) return err;
+  const char* name = GATED ? "fp8_gemm_gate_up" : "fp8_gemm_down";
+  timing_before(name, s);
+  kern<<<sm_count(), kThreads, smem, s>>>(tm_w, tm_b, p);
+  timing_after(name, s);
+  return cudaGetLastError();
+}
+
+}  // namespace f8
+
+cudaError_t launch_fp8_gemm(const F8GemmProblem& p, cudaStream_t s) {
+  return p.gated ? f8::launch_t<true>(p, s) : f8::launch_t<false>(p, s);
+}
+
+}  // namespace moe

@@ -60,6 +60,25 @@ struct W4GemmProblem {
 };
 cudaError_t launch_w4a16_gemm(const W4GemmProblem& p, cudaStream_t s);
 
+// block-FP8 grouped GEMM (gemm_fp8.cu)
+struct F8GemmProblem {
+  const uint8_t* w;        // e4m3 [E, rows_per_expert, K]
+  const float* w_scale;    // [E, rows_per_expert/128, K/128]
+  const uint8_t* act;      // e4m3 [act_rows, K]
+  const float* x_scale;    // transposed activation scales [K/128, act_rows]
+  int act_rows;
+  int K, E, rows_per_expert;
+  bool gated;              // gate rows [0, I), up rows [I, 2I); output e4m3 h [*, I] + h_scale
+  int I;
+  TileSched sched;
+  void* out;
+  int out_ld;
+  float* h_scale;          // gated: [I/128, act_rows]
+};
+cudaError_t launch_fp8_gemm(const F8GemmProblem& p, cudaStream_t s);
+cudaError_t launch_permute_fp8(const uint8_t* x, const float* xs, const int32_t* inv_pos, int T, int k, int H,
+                               uint8_t* x_perm, float* xs_t, int P, cudaStream_t s);
+
 // driver entry point for tensor maps (api.cu)
 // 2-D tiled tensor map over a row-major [rows, cols] tensor at `base` (zero fill out of bounds).
 CUresult encode_tmap_2d(CUtensorMap* map, const void* base, CUtensorMapDataType dt, uint64_t cols, uint64_t rows,

@@ -3,5 +3,6 @@
 #include "route_align.cu"
 #include "permute_combine.cu"
 #include "gemm_w4a16.cu"
+#include "gemm_fp8.cu"
 #include "api.cu"
 #include "align_noalloc.cu"

@@ -56,6 +56,33 @@ cudaError_t launch_permute_w4(const uint16_t* x_bf16, const int32_t* inv_pos, in
   return cudaGetLastError();
 }
 
+// one warp per (token, slot) pair: x_perm[r] = x[p / k] (e4m3 bytes), xs_t[g][r] = xs[p / k][g]
+__global__ void __launch_bounds__(256) permute_fp8_kernel(const uint4* __restrict__ x, const float* __restrict__ xs,
+                                                          const int32_t* __restrict__ inv_pos, int Pn, int k, int H,
+                                                          uint4* __restrict__ x_perm, float* __restrict__ xs_t,
+                                                          int P) {
+  const int p = (int)((blockIdx.x * blockDim.x + threadIdx.x) >> 5);
+  const int lane = threadIdx.x & 31;
+  if (p >= Pn) return;
+  const int r = inv_pos[p];
+  if (r < 0) return;
+  const int t = p / k;
+  const uint4* src = x + (size_t)t * (H / 16);
+  uint4* dst = x_perm + (size_t)r * (H / 16);
+  for (int c = lane; c < H / 16; c += 32) dst[c] = __ldg(src + c);
+  for (int g = lane; g < H / 128; g += 32) xs_t[(size_t)g * P + r] = __ldg(xs + (size_t)t * (H / 128) + g);
+}
+
+cudaError_t launch_permute_fp8(const uint8_t* x, const float* xs, const int32_t* inv_pos, int T, int k, int H,
+                               uint8_t* x_perm, float* xs_t, int P, cudaStream_t s) {
+  const int Pn = T * k;
+  timing_before("permute_fp8", s);
+  permute_fp8_kernel<<<ceil_div(Pn, 8), 256, 0, s>>>(reinterpret_cast<const uint4*>(x), xs, inv_pos, Pn, k, H,
+                                                    reinterpret_cast<uint4*>(x_perm), xs_t, P);
+  timing_after("permute_fp8", s);
+  return cudaGetLastError();
+}
+
 __global__ void __launch_bounds__(256) convert_rows_kernel(const uint4* __restrict__ a, int a_is_bf16, size_t n8,
                                                            uint4* __restrict__ out) {
   for (size_t i = blockIdx.x * (size_t)blockDim.x + threadIdx.x; i < n8; i += (size_t)gridDim.x * blockDim.x) {
