@@ -34,9 +34,12 @@ import numpy as np  # noqa: E402
 METRIC = "routed-MoE layer µs, TFLOPS and HBM GB/s (% roofline) at decode T=64 and prefill T=8192"
 MODEL = dict(H=7168, I=2048, E=384, k=8)
 WORKLOADS = {
-    "decode": dict(T=64, zipf=0.0, steps=400, warmup=20),
-    "prefill": dict(T=8192, zipf=1.1, steps=40, warmup=5),
+    "decode": dict(kind="w4a16", T=64, zipf=0.0, steps=400, warmup=20),
+    "prefill": dict(kind="w4a16", T=8192, zipf=1.1, steps=40, warmup=5),
 }
+for _t in (1, 16, 64, 512, 4096):  # block-FP8 layer, 256 experts
+    WORKLOADS[f"fp8_t{_t}"] = dict(kind="fp8", T=_t, zipf=0.0, steps=200 if _t <= 512 else 60, warmup=10)
+FP8_MODEL = dict(H=7168, I=2048, E=256, k=8)
 W13_BYTES_PER_EXPERT = 2 * 2048 * 7168 // 2 + 2 * 2048 * (7168 // 32) * 2   # INT4 words + bf16 scales
 W2_BYTES_PER_EXPERT = 7168 * 2048 // 2 + 7168 * (2048 // 32) * 2
 
@@ -159,8 +162,37 @@ def make_model(seed: int):
     return out
 
 
-def make_inputs(seed: int, T: int, zipf: float):
+def make_model_fp8(seed: int):
+    """All 256 block-FP8 experts generated on the host by the seeded generator, copied to HBM."""
+    import torch
     import synth
+    H, I, E = FP8_MODEL["H"], FP8_MODEL["I"], FP8_MODEL["E"]
+    lo, hi = synth.FP8_SCALE_RANGE
+    out = {}
+    specs = [("w13", (E, 2 * I, H), torch.uint8, "w13_8"), ("w13_s", (E, 2 * I // 128, H // 128), torch.float32, "w13_8s"),
+             ("w2", (E, H, I), torch.uint8, "w2_8"), ("w2_s", (E, H // 128, I // 128), torch.float32, "w2_8s")]
+    for name, shape, dt, tid in specs:
+        d = torch.empty(shape, dtype=dt, device="cuda")
+        per = int(np.prod(shape[1:]))
+        chunk = 16
+        stage = torch.empty((chunk, *shape[1:]), dtype=dt, pin_memory=True)
+        for e0 in range(0, E, chunk):
+            n = min(chunk, E - e0)
+            buf = stage[:n]
+            if dt == torch.uint8:
+                synth.fill_normal_e4m3(seed, synth.TID[tid], e0 * per, buf)
+            else:
+                synth.fill_uniform_f32(seed, synth.TID[tid], e0 * per, buf, lo, hi)
+            d[e0:e0 + n].copy_(buf)
+        out[name] = d
+    return out
+
+
+def make_inputs(seed: int, T: int, zipf: float, kind: str = "w4a16"):
+    import synth
+    if kind == "fp8":
+        xq, xs = synth.x_e4m3(seed, T, FP8_MODEL["H"])
+        return (xq, xs), synth.logits(seed, T, FP8_MODEL["E"], zipf_s=zipf)
     x = synth.x_bf16(seed, T, MODEL["H"])
     lg = synth.logits(seed, T, MODEL["E"], zipf_s=zipf)
     return x, lg
@@ -171,23 +203,38 @@ def run_ours(args, world, rank):
     import quantized_mixture_experts_softmax_b200 as moe
 
     wl = WORKLOADS[args.workload]
-    T, H, I, E, k = wl["T"], MODEL["H"], MODEL["I"], MODEL["E"], MODEL["k"]
+    kind = wl["kind"]
+    M = FP8_MODEL if kind == "fp8" else MODEL
+    T, H, I, E, k = wl["T"], M["H"], M["I"], M["E"], M["k"]
     steps = args.steps if args.steps is not None else wl["steps"]
     warmup = args.warmup if args.warmup is not None else wl["warmup"]
     warmup = max(3, warmup)
     seed = 0
-    W = make_model(seed)
-    x_h, lg_h = make_inputs(seed, T, wl["zipf"])
-    x = torch.from_numpy(x_h).cuda().view(torch.bfloat16)
+    W = make_model_fp8(seed) if kind == "fp8" else make_model(seed)
+    x_h, lg_h = make_inputs(seed, T, wl["zipf"], kind)
     lg = torch.from_numpy(lg_h).cuda()
     ids = torch.empty(T, k, dtype=torch.int32, device="cuda")
     tw = torch.empty(T, k, dtype=torch.float32, device="cuda")
     out = torch.empty(T, H, dtype=torch.bfloat16, device="cuda")
-    ws = torch.empty(moe.moe_w4a16_workspace_size(T, H, I, E, k), dtype=torch.uint8, device="cuda")
+    if kind == "fp8":
+        x = torch.from_numpy(x_h[0]).cuda()
+        xs = torch.from_numpy(x_h[1]).cuda()
+        ws = torch.empty(moe.moe_blockfp8_workspace_size(T, H, I, E, k), dtype=torch.uint8, device="cuda")
+
+        def forward(xx, xxs):
+            moe.moe_blockfp8_forward(xx, xxs, ids, tw, W["w13"], W["w13_s"], W["w2"], W["w2_s"], out=out,
+                                     workspace=ws)
+    else:
+        x = torch.from_numpy(x_h).cuda().view(torch.bfloat16)
+        xs = None
+        ws = torch.empty(moe.moe_w4a16_workspace_size(T, H, I, E, k), dtype=torch.uint8, device="cuda")
+
+        def forward(xx, xxs):
+            moe.moe_w4a16_forward(xx, ids, tw, W["w13_q"], W["w13_s"], W["w2_q"], W["w2_s"], out=out, workspace=ws)
 
     def step():
         moe.moe_route(lg, k, topk_ids=ids, topk_w=tw)
-        moe.moe_w4a16_forward(x, ids, tw, W["w13_q"], W["w13_s"], W["w2_q"], W["w2_s"], out=out, workspace=ws)
+        forward(x, xs)
 
     for _ in range(warmup):
         step()
@@ -218,18 +265,30 @@ def run_ours(args, world, rank):
     clocks = clk.summary()
 
     # ---- end to end through the C ABI with host buffers (pinned), copies inside the region
-    x_pin = torch.from_numpy(x_h).pin_memory()
     lg_pin = torch.from_numpy(lg_h).pin_memory()
     out_pin = torch.empty(T, H, dtype=torch.bfloat16).pin_memory()
-    x_d = torch.empty(T, H, dtype=torch.int16, device="cuda")
     lg_d = torch.empty(T, E, dtype=torch.float32, device="cuda")
+    if kind == "fp8":
+        x_pin = torch.from_numpy(x_h[0]).pin_memory()
+        xs_pin = torch.from_numpy(x_h[1]).pin_memory()
+        x_d = torch.empty_like(x)
+        xs_d = torch.empty_like(xs)
+        h2d = T * H + T * (H // 128) * 4 + T * E * 4
+    else:
+        x_pin = torch.from_numpy(x_h).pin_memory()
+        xs_pin = None
+        x_d = torch.empty(T, H, dtype=torch.int16, device="cuda")
+        xs_d = None
+        h2d = T * H * 2 + T * E * 4
+    d2h = T * H * 2
 
     def e2e_step():
-        x_d.copy_(x_pin.view(torch.int16), non_blocking=True)
+        x_d.copy_(x_pin.view(x_d.dtype), non_blocking=True)
+        if xs_d is not None:
+            xs_d.copy_(xs_pin, non_blocking=True)
         lg_d.copy_(lg_pin, non_blocking=True)
         moe.moe_route(lg_d, k, topk_ids=ids, topk_w=tw)
-        moe.moe_w4a16_forward(x_d.view(torch.bfloat16), ids, tw, W["w13_q"], W["w13_s"], W["w2_q"], W["w2_s"],
-                              out=out, workspace=ws)
+        forward(x_d if kind == "fp8" else x_d.view(torch.bfloat16), xs_d)
         out_pin.copy_(out, non_blocking=True)
 
     for _ in range(3):
@@ -244,51 +303,65 @@ def run_ours(args, world, rank):
     torch.cuda.synchronize()
     barrier(world)
     ms_e2e = max_over_ranks(ev0.elapsed_time(ev1), world) / e2e_steps
-    h2d = T * H * 2 + T * E * 4
-    d2h = T * H * 2
 
     # ---- roofline of the dominant kernel
     peaks = load_peaks()
     P = T * k
     flops = 6.0 * P * H * I
-    layer_bytes = active * (W13_BYTES_PER_EXPERT + W2_BYTES_PER_EXPERT) + 2 * T * H * 2 + T * E * 4
+    if kind == "fp8":
+        w13_b = 2 * I * H + (2 * I // 128) * (H // 128) * 4
+        w2_b = H * I + (H // 128) * (I // 128) * 4
+        act_in, act_mid, y_b = P * H, P * I, P * H * 4
+        x_in = T * H + T * (H // 128) * 4
+    else:
+        w13_b, w2_b = W13_BYTES_PER_EXPERT, W2_BYTES_PER_EXPERT
+        act_in, act_mid, y_b = P * H * 2, P * I * 2, P * H * 4
+        x_in = T * H * 2
+    layer_bytes = active * (w13_b + w2_b) + x_in + T * H * 2 + T * E * 4
+    # tensor peak for the contraction's own operand type: fp16 runs at the measured bf16 rate,
+    # e4m3 at twice it (the nominal dense fp8 : bf16 ratio)
+    t_peak = peaks["bf16"] * (2.0 if kind == "fp8" else 1.0)
+    t_peak_src = peaks["src"] + (" bf16 GEMM x 2 (nominal fp8:bf16)" if kind == "fp8" else " bf16 GEMM, burst")
     top = max(kern.items(), key=lambda kv: kv[1][0]) if kern else None
     roof = None
     if top is not None:
         name, (ms_k, n_k) = top
         per_launch_s = ms_k / n_k / 1e3
-        if name == "w4a16_gemm_gate_up":
-            alg_bytes = active * W13_BYTES_PER_EXPERT + P * H * 2 + P * I * 2
+        if name.endswith("gate_up"):
+            alg_bytes = active * w13_b + act_in + act_mid
             alg_flops = 2.0 * P * H * 2 * I
-        elif name == "w4a16_gemm_down":
-            alg_bytes = active * W2_BYTES_PER_EXPERT + P * I * 2 + P * H * 4
+        elif name.endswith("down"):
+            alg_bytes = active * w2_b + act_mid + y_b
             alg_flops = 2.0 * P * I * H
         else:
             alg_bytes, alg_flops = None, None
-        if args.workload == "decode" and alg_bytes:
+        hbm_bound = alg_bytes is not None and (alg_flops / alg_bytes) < (t_peak * 1e3 / peaks["hbm"])
+        if alg_bytes and hbm_bound:
             ach = alg_bytes / per_launch_s / 1e9
             roof = dict(kernel=name, bound="hbm", achieved=round(ach, 1), peak=peaks["hbm"], unit="GB/s",
-                        frac=round(ach / peaks["hbm"], 4), traffic=None, peak_source=peaks["src"],
+                        frac=round(ach / peaks["hbm"], 4), traffic=None, peak_source=peaks["src"] + " (copy, burst)",
                         algorithmic_bytes_per_launch=int(alg_bytes), launch_ms=round(per_launch_s * 1e3, 4))
         elif alg_flops:
             ach = alg_flops / per_launch_s / 1e12
-            roof = dict(kernel=name, bound="tensor", achieved=round(ach, 1), peak=peaks["bf16"], unit="TFLOP/s",
-                        frac=round(ach / peaks["bf16"], 4), traffic=None, peak_source=peaks["src"],
+            roof = dict(kernel=name, bound="tensor", achieved=round(ach, 1), peak=t_peak, unit="TFLOP/s",
+                        frac=round(ach / t_peak, 4), traffic=None, peak_source=t_peak_src,
                         algorithmic_flops_per_launch=alg_flops, launch_ms=round(per_launch_s * 1e3, 4))
     launches = sum(n for (_, n) in kern.values())
     res = {
         "metric": METRIC, "value": round(ms_step * 1e3 / world, 2), "unit": "µs/layer",
         "n_gpus": world, "steps": steps, "warmup": warmup, "ms_per_step": round(ms_step, 4),
-        "higher_is_better": False, "scaling": "weak", "vs_baseline": None, "dtype": "w4a16 (fp16 MMA, fp32 acc)",
-        "data": "synthetic (seeded counter-based generator; random-init INT4 weights)",
-        "config": {"workload": f"{args.workload} W4A16 MoE layer T={T} H={H} I={I} E={E} top-{k}",
+        "higher_is_better": False, "scaling": "weak", "vs_baseline": None,
+        "dtype": "e4m3 (fp32 acc)" if kind == "fp8" else "w4a16 (fp16 MMA, fp32 acc)",
+        "data": "synthetic (seeded counter-based generator; random-init quantized weights)",
+        "config": {"workload": f"{args.workload} {'block-FP8' if kind == 'fp8' else 'W4A16'} MoE layer T={T} "
+                               f"H={H} I={I} E={E} top-{k}",
                    "T": T, "H": H, "I": I, "E": E, "k": k, "active_experts": active,
                    "parallelism": "replicas" if world > 1 else "single GPU",
-                   "l2": "no flush: >6.9 GB of expert weights streamed per step (L2 126 MB)"},
+                   "l2": "no flush: the active experts' weights streamed per step exceed the 126 MB L2"},
         "layer": {"us": round(ms_step * 1e3, 2), "tflops": round(flops / (ms_step * 1e-3) / 1e12, 2),
                   "hbm_gbs": round(layer_bytes / (ms_step * 1e-3) / 1e9, 1),
                   "hbm_frac": round(layer_bytes / (ms_step * 1e-3) / 1e9 / peaks["hbm"], 4),
-                  "tensor_frac": round(flops / (ms_step * 1e-3) / 1e12 / peaks["bf16"], 4),
+                  "tensor_frac": round(flops / (ms_step * 1e-3) / 1e12 / t_peak, 4),
                   "algorithmic_bytes": int(layer_bytes), "flops": flops},
         "kernels_ms_per_step": {n: round(v[0] / steps, 4) for n, v in sorted(kern.items(), key=lambda kv: -kv[1][0])},
         "e2e": {"value": round(ms_e2e * 1e3, 2), "unit": "µs/layer", "h2d_bytes_per_step": h2d,
@@ -297,43 +370,40 @@ def run_ours(args, world, rank):
         "roofline": roof,
         "clocks": clocks,
     }
-    return res, (x_h, lg_h, T)
+    return res, (x_h, lg_h, T, kind)
 
 
-def oracle_sample_time(x_h, lg_h, T, budget_s=15.0):
+def oracle_sample_time(x_h, lg_h, T, kind="w4a16", budget_s=15.0):
     """CPU oracle on a bounded token sample of the same workload -> (us per layer, sample, cores)."""
     import oracle
     import synth
-    k = MODEL["k"]
+    M = FP8_MODEL if kind == "fp8" else MODEL
+    k = M["k"]
     ids, w, _ = oracle.route(lg_h, k)
     cores = oracle.nthreads()
-    n_probe = max(1, min(T, cores))
-    # weights of the experts the probe tokens use (the generator regenerates any slice)
-    t0 = time.time()
-    tok = np.arange(n_probe, dtype=np.int32)
-    used = np.unique(ids[tok])
-    W = synth.w4a16_weights(0, MODEL["H"], MODEL["I"], used)
-    remap = {int(e): i for i, e in enumerate(used)}
-    ids_l = np.vectorize(lambda e: remap.get(int(e), 0))(ids[tok]).astype(np.int32)
-    gen_s = time.time() - t0
-    t0 = time.time()
-    oracle.w4a16_tokens(x_h[tok], ids_l, w[tok], W["w13_q"], W["w13_s"], W["w2_q"], W["w2_s"])
-    probe = time.time() - t0
-    per_tok = probe / n_probe  # wall time per token with all cores busy
-    n = int(min(T, max(n_probe, budget_s / max(per_tok, 1e-9))))
-    if n > n_probe:
+
+    def run(n):
         tok = np.arange(n, dtype=np.int32)
         used = np.unique(ids[tok])
-        W = synth.w4a16_weights(0, MODEL["H"], MODEL["I"], used)
         remap = {int(e): i for i, e in enumerate(used)}
         ids_l = np.vectorize(lambda e: remap.get(int(e), 0))(ids[tok]).astype(np.int32)
-        t0 = time.time()
-        oracle.w4a16_tokens(x_h[tok], ids_l, w[tok], W["w13_q"], W["w13_s"], W["w2_q"], W["w2_s"])
-        el = time.time() - t0
-    else:
-        el = probe
+        if kind == "fp8":
+            Wt = synth.fp8_weights(0, M["H"], M["I"], used)
+            t0 = time.time()
+            oracle.fp8_tokens(x_h[0][tok], x_h[1][tok], ids_l, w[tok], Wt["w13"], Wt["w13_s"], Wt["w2"], Wt["w2_s"])
+        else:
+            Wt = synth.w4a16_weights(0, M["H"], M["I"], used)
+            t0 = time.time()
+            oracle.w4a16_tokens(x_h[tok], ids_l, w[tok], Wt["w13_q"], Wt["w13_s"], Wt["w2_q"], Wt["w2_s"])
+        return time.time() - t0
+
+    n_probe = max(1, min(T, cores))
+    probe = run(n_probe)
+    per_tok = probe / n_probe  # wall time per token with all cores busy
+    n = int(min(T, max(n_probe, budget_s / max(per_tok, 1e-9))))
+    el = run(n) if n > n_probe else probe
     us_layer = el / n * T * 1e6
-    return us_layer, f"{n} of {T} tokens (all 8 experts each), extrapolated linearly to {T}", cores, gen_s
+    return us_layer, f"{n} of {T} tokens (all {k} experts each), extrapolated linearly to {T}", cores, 0.0
 
 
 def run_reference(args, world, rank):
@@ -341,11 +411,11 @@ def run_reference(args, world, rank):
     T = wl["T"]
     steps = args.steps if args.steps is not None else 3
     warmup = args.warmup if args.warmup is not None else 1
-    x_h, lg_h = make_inputs(0, T, wl["zipf"])
+    x_h, lg_h = make_inputs(0, T, wl["zipf"], wl["kind"])
     vals = []
     sample = cores = None
     for i in range(warmup + steps):
-        us, sample, cores, _ = oracle_sample_time(x_h, lg_h, T, budget_s=8.0)
+        us, sample, cores, _ = oracle_sample_time(x_h, lg_h, T, wl["kind"], budget_s=8.0)
         if i >= warmup:
             vals.append(us)
     v = statistics.median(vals)
@@ -353,8 +423,8 @@ def run_reference(args, world, rank):
         "metric": METRIC, "value": round(v, 1), "unit": "µs/layer", "n_gpus": world, "steps": steps,
         "warmup": warmup, "ms_per_step": round(v / 1e3, 3), "higher_is_better": False, "scaling": "weak",
         "vs_baseline": None, "dtype": "f64 (oracle)", "data": "synthetic",
-        "config": {"workload": f"{args.workload} W4A16 MoE layer T={T} H={MODEL['H']} I={MODEL['I']} "
-                               f"E={MODEL['E']} top-{MODEL['k']}"},
+        "config": {"workload": f"{args.workload} {'block-FP8' if wl['kind'] == 'fp8' else 'W4A16'} MoE layer "
+                               f"T={T}"},
         "impl": "reference",
         "cpu_baseline": {"value": round(v, 1), "unit": "µs/layer", "cores": cores, "kind": "oracle",
                          "sample": sample},
@@ -375,6 +445,7 @@ def main():
     args = ap.parse_args()
     if args.experts:
         MODEL["E"] = args.experts
+        FP8_MODEL["E"] = args.experts
 
     if args.impl == "reference":
         rank = int(os.environ.get("RANK", "0"))
@@ -384,9 +455,9 @@ def main():
         return
 
     world, rank, _ = dist_init()
-    res, (x_h, lg_h, T) = run_ours(args, world, rank)
+    res, (x_h, lg_h, T, kind) = run_ours(args, world, rank)
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        us, sample, cores, _ = oracle_sample_time(x_h, lg_h, T)
+        us, sample, cores, _ = oracle_sample_time(x_h, lg_h, T, kind)
         res["cpu_baseline"] = {"value": round(us, 1), "unit": "µs/layer", "cores": cores, "kind": "oracle",
                                "sample": sample}
     if rank == 0:
