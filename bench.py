@@ -442,10 +442,14 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--experts", type=int, default=None,
                     help="override the expert count (small profiling cases only; not a bench line)")
+    ap.add_argument("--tokens", type=int, default=None,
+                    help="override the workload's token count (small profiling cases only; not a bench line)")
     args = ap.parse_args()
     if args.experts:
         MODEL["E"] = args.experts
         FP8_MODEL["E"] = args.experts
+    if args.tokens:
+        WORKLOADS[args.workload] = dict(WORKLOADS[args.workload], T=args.tokens)
 
     if args.impl == "reference":
         rank = int(os.environ.get("RANK", "0"))

@@ -132,15 +132,32 @@ void timing_after(const char*, cudaStream_t s) {
 
 // ------------------------------------------------------------------ workspace layouts
 namespace {
+// Decode-sized problems (no expert can get more than 64 rows) run on the int8 tensor-core GEMM
+// with activations as 16-bit fixed-point planes; larger ones on the fp16 GEMM.
+bool use_i8(int max_rows_per_expert) { return max_rows_per_expert <= 64; }
+
+// 16-bit fixed-point planes of an activation matrix [rows, K]
+struct Planes {
+  int8_t* x;      // [2*rows, K]: hi and lo rows interleaved
+  int32_t* meta;  // [rows, meta_words_per_row(K)]: group sums and block scales
+};
+Planes take_planes(Carver& c, size_t rows, int K) {
+  Planes q;
+  q.x = c.take<int8_t>(2 * rows * K);
+  q.meta = c.take<int32_t>(rows * meta_words_per_row(K));
+  return q;
+}
+
 struct FwdWs {
   int32_t *counts, *offsets, *sorted, *inv, *blockcnt, *tile_prefix, *chunk;
-  __half *x_perm, *h;
+  __half *x_perm, *h;  // fp16 path
+  Planes xq, hq;       // int8 path
   float* y;
   size_t bytes;
 };
 FwdWs carve_w4_forward(void* ws, int T, int H, int I, int E, int k) {
   Carver c(ws);
-  FwdWs w;
+  FwdWs w{};
   const size_t P = (size_t)T * k;
   w.counts = c.take<int32_t>(E);
   w.offsets = c.take<int32_t>(E + 1);
@@ -149,24 +166,33 @@ FwdWs carve_w4_forward(void* ws, int T, int H, int I, int E, int k) {
   w.blockcnt = c.take<int32_t>((size_t)align_blocks(T, k) * E);
   w.tile_prefix = c.take<int32_t>(E + 1);
   w.chunk = c.take<int32_t>(E);
-  w.x_perm = c.take<__half>(P * H);
-  w.h = c.take<__half>(P * I);
+  if (use_i8(T)) {
+    w.xq = take_planes(c, P, H);
+    w.hq = take_planes(c, P, I);
+  } else {
+    w.x_perm = c.take<__half>(P * H);
+    w.h = c.take<__half>(P * I);
+  }
   w.y = c.take<float>(P * H);
   w.bytes = c.off + 256;
   return w;
 }
 struct GemmWs {
   int32_t *row_count, *tile_prefix, *chunk;
-  __half* a;
+  __half* a;  // fp16 path
+  Planes aq;  // int8 path
   size_t bytes;
 };
 GemmWs carve_gemm(void* ws, int M, int K, int E) {
   Carver c(ws);
-  GemmWs w;
+  GemmWs w{};
   w.row_count = c.take<int32_t>(E);
   w.tile_prefix = c.take<int32_t>(E + 1);
   w.chunk = c.take<int32_t>(E);
-  w.a = c.take<__half>((size_t)M * K);
+  if (use_i8(M))
+    w.aq = take_planes(c, M, K);
+  else
+    w.a = c.take<__half>((size_t)M * K);
   w.bytes = c.off + 256;
   return w;
 }
@@ -196,7 +222,7 @@ F8Ws carve_fp8_forward(void* ws, int T, int H, int I, int E, int k) {
   w.bytes = c.off + 256;
   return w;
 }
-int pick_nmax(int max_rows_per_expert) { return max_rows_per_expert <= 64 ? w4::kThinN : 256; }
+int pick_nmax(int max_rows_per_expert) { return use_i8(max_rows_per_expert) ? kI8TileRows : 256; }
 
 bool shape_ok(int T, int H, int I, int E, int k) {
   if (T < 1 || k < 1 || E < k || E > 1024) return false;
@@ -280,8 +306,24 @@ moe_status_t moe_w4a16_forward(const moe_w4a16_args* a, void* ws, size_t ws_byte
   const int P = T * k;
   cudaError_t e = launch_align(a->topk_ids, T, k, E, 1, w.counts, w.offsets, w.sorted, w.inv, w.blockcnt, nmax,
                                w.tile_prefix, w.chunk, stream);
-  if (e == cudaSuccess) e = launch_permute_w4(static_cast<const uint16_t*>(a->x), w.inv, T, k, H, w.x_perm, stream);
   const TileSched sched{w.offsets, w.counts, w.tile_prefix, w.chunk};
+  if (use_i8(T)) {
+    if (e == cudaSuccess)
+      e = launch_planes(static_cast<const uint16_t*>(a->x), 1, w.inv, P, k, H, w.xq.x, w.xq.meta, stream);
+    if (e == cudaSuccess) {
+      W4I8Problem g{a->w13_q, static_cast<const uint16_t*>(a->w13_s), w.xq.x, w.xq.meta, P, H, E, 2 * I, true, I,
+                    sched, OUT_PLANES, w.hq.x, w.hq.meta, I};
+      e = launch_w4i8_gemm(g, stream);
+    }
+    if (e == cudaSuccess) {
+      W4I8Problem g{a->w2_q, static_cast<const uint16_t*>(a->w2_s), w.hq.x, w.hq.meta, P, I, E, H, false, 0, sched,
+                    OUT_F32, w.y, nullptr, H};
+      e = launch_w4i8_gemm(g, stream);
+    }
+    if (e == cudaSuccess) e = launch_combine(w.y, w.inv, a->topk_w, T, k, H, a->out, a->out_fp32, stream);
+    return e == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
+  }
+  if (e == cudaSuccess) e = launch_permute_w4(static_cast<const uint16_t*>(a->x), w.inv, T, k, H, w.x_perm, stream);
   if (e == cudaSuccess) {
     W4GemmProblem g{a->w13_q, static_cast<const uint16_t*>(a->w13_s), w.x_perm, P, H, E, 2 * I, true, I, sched, nmax,
                     w.h, I, OUT_H_F16_INTERLEAVED};
@@ -348,9 +390,19 @@ moe_status_t moe_w4a16_gemm(const void* a, int a_is_bf16, const int32_t* w_q, co
   const GemmWs w = carve_gemm(ws, M, K, E);
   const int nmax = pick_nmax(M);
   cudaError_t e = launch_sched_from_offsets(expert_offsets, E, M, nmax, w.row_count, w.tile_prefix, w.chunk, stream);
+  const TileSched sched{expert_offsets, w.row_count, w.tile_prefix, w.chunk};
+  if (use_i8(M)) {
+    if (e == cudaSuccess)
+      e = launch_planes(static_cast<const uint16_t*>(a), a_is_bf16, nullptr, M, 1, K, w.aq.x, w.aq.meta, stream);
+    if (e == cudaSuccess) {
+      W4I8Problem g{w_q, static_cast<const uint16_t*>(w_s), w.aq.x, w.aq.meta, M, K, E, N, false, 0, sched,
+                    out_fp32 ? OUT_F32 : OUT_BF16, out, nullptr, N};
+      e = launch_w4i8_gemm(g, stream);
+    }
+    return e == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
+  }
   if (e == cudaSuccess) e = launch_convert_rows(static_cast<const uint16_t*>(a), a_is_bf16, M, K, w.a, stream);
   if (e == cudaSuccess) {
-    const TileSched sched{expert_offsets, w.row_count, w.tile_prefix, w.chunk};
     W4GemmProblem g{w_q, static_cast<const uint16_t*>(w_s), w.a, M, K, E, N, false, 0, sched, nmax, out, N,
                     out_fp32 ? OUT_F32 : OUT_BF16};
     e = launch_w4a16_gemm(g, stream);

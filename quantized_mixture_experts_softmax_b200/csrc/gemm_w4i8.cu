@@ -1,0 +1,650 @@
+// a5-a7 for decode-sized experts: W4A16 grouped GEMM on the int8 tensor cores.
+//
+// With few tokens per expert the tensor core's cost is set by how many weights one MMA covers
+// (a 128-row MMA with N <= 64 takes the same time whatever N is).  An fp16 weight operand
+// covers 128x16 weights per instruction; here the INT4 weights go to the tensor core as
+// exact unsigned 8-bit integers n = q + 8 (one AND/XOR per four weights, no floating-point
+// dequantization), so one kind::i8 MMA covers 128x32 weights - exactly one scale group of
+// the format (the Chord article, second paragraph: one BF16 scale per 32 weights).
+//
+// The 16-bit activations enter as 16-bit fixed point: per (token, 128-K block) a scale
+// s = amax / 32639 and integers X = rint(x / s) split into two signed 8-bit planes
+// X = 256*hi + lo, interleaved along N (tile row 2c = hi of token c, 2c+1 = its lo; 8 tokens
+// give N = 16, the smallest N of a 128-row MMA).  For one
+// token t and one weight row r, one MMA per 32-K group g gives D_hi and D_lo exactly in int32:
+//     sum_{k in g} q[r][k] * X[t][k] = 256*D_hi + D_lo - 8*C[t][g],   C[t][g] = sum_{k in g} X[t][k],
+// which the promotion warps scale by the group's weight scale and the block's activation
+// scale and accumulate in fp32.  They read from tensor memory only the columns of the tile's
+// live tokens (2, 4, 8 or 16 columns of each MMA's 16), batched under one wait; the tokens' group sums and
+// block scales arrive with the stage (one TMA box of the meta words), as do the weight scales.  The gate/up kernel ends with
+// h = SiLU(gate) * up written straight back in the same fixed-point planes (one scale per
+// token per 128-row tile) for the down kernel.
+//
+// Work list, swap (weights in the MMA's M slot) and persistence as in the fp16 GEMM.  Warps
+// (512 threads): 0 producer (TMA of the INT4 words, weight scales, activation planes and meta
+// words of the token tile per 256-K stage; cp.async for scale rows not 16-byte aligned), 1 TMEM allocator + MMA issuer, 4-7 promotion and epilogue, 8-15 unpacking INT4
+// words into u8 rows of tensor memory (the MMA's A operand).
+#include "common.cuh"
+#include "internal.h"
+
+namespace moe {
+namespace w4i8 {
+
+constexpr int BM = 128;          // weight rows per tile
+constexpr int KB = 256;          // K per stage
+constexpr int G = 32;            // K per scale group = K per MMA
+constexpr int NG = KB / G;       // groups per stage
+constexpr int NT = kI8TileRows;  // token rows per tile (each gives a hi and a lo plane row)
+constexpr int DC = 2 * NT;       // D columns of one MMA (N)
+constexpr int SG = 4;            // groups per D slot
+constexpr int kThreads = 512;
+constexpr int kEpiWarp0 = 4;
+constexpr int kUnpackWarp0 = 8;
+constexpr int kNumUnpack = 8;
+static_assert(NT == 8, "the promotion code handles up to 8 tokens per tile");
+
+template <bool GATED>
+struct Cfg {
+  static constexpr int NA = GATED ? 2 : 1;
+  static constexpr int W_TILE = BM * KB / 2;   // INT4 bytes
+  static constexpr int B_ATOM = 2 * NT * 128;  // one 128-K atom of the 2*NT plane rows
+  static constexpr int STAGE_B = NA * W_TILE;
+  static constexpr int META = STAGE_B + (KB / 128) * B_ATOM;  // [NT tokens][kMetaWords] int32
+  static constexpr int META_BYTES = NT * kMetaWords * 4;
+  static constexpr int SCL = META + 1024;            // [NA][BM rows][NG] bf16 weight scales
+  static constexpr int S_TILE = BM * NG * 2;
+  static constexpr int STAGE = SCL + NA * S_TILE;
+  static_assert(META_BYTES <= 1024, "meta box fits its slot");
+  static constexpr int ST = GATED ? 5 : 9;
+  // TMEM: D ring of SG-group slots [group][matrix][DC int32 columns], A ring of whole-stage
+  // slots [matrix][group][8 columns] (a 32-K row of u8 = 8 columns)
+  static constexpr int D_SLOT = SG * NA * DC;
+  static constexpr int DSLOTS = GATED ? 2 : 4;
+  static constexpr int A_SLOT = NA * NG * 8;
+  static constexpr int ASLOTS = GATED ? 2 : 4;
+  static constexpr int A_COL0 = DSLOTS * D_SLOT;
+  static_assert(A_COL0 + ASLOTS * A_SLOT <= 512, "TMEM has 512 columns");
+  static constexpr int OFF_BAR = ST * STAGE;
+  static constexpr int NUM_BARS = 2 * ST + 2 * ASLOTS + 2 * DSLOTS + 2;
+  static constexpr int OFF_MISC = OFF_BAR + NUM_BARS * 8;
+  static constexpr int OFF_RED = OFF_MISC + 16;  // [4 warps][NT] amax partials
+  static constexpr int OFF_PREFIX = OFF_RED + 4 * NT * 4;
+  static_assert(STAGE % 1024 == 0 && STAGE_B % 1024 == 0, "swizzled tiles need 1024-byte alignment");
+  static constexpr size_t smem_bytes(int E) { return (size_t)OFF_PREFIX + 4 * (size_t)(E + 1) + 1024; }
+  static_assert(smem_bytes(1024) <= 232448, "shared memory budget");
+};
+
+struct Params {
+  int K, E, rows_per_expert, I, m_tiles;
+  const uint16_t* w_s;   // bf16 [E*rows_per_expert, K/32]
+  int scales_tma;        // 1: weight scales by TMA (K % 256 == 0), else by cp.async
+  TileSched sched;
+  int out_kind;          // OUT_PLANES (gated), OUT_F32, OUT_BF16
+  void* out;             // planes int8 [2*rows, out_ld]; else fp32/bf16 [rows, out_ld]
+  int32_t* out_meta;     // planes: meta words of h
+  int out_ld;
+  uint64_t wait_limit;
+};
+
+struct Item {
+  int e, m, r0, nvalid;
+};
+
+__device__ __forceinline__ Item decode_item(int it, const int* __restrict__ sprefix, const Params& p) {
+  Item I;
+  const int tile = it / p.m_tiles;
+  int lo = 0, hi = p.E;  // sprefix[lo] <= tile < sprefix[hi]
+  while (hi - lo > 1) {
+    const int mid = (lo + hi) >> 1;
+    if (sprefix[mid] <= tile)
+      lo = mid;
+    else
+      hi = mid;
+  }
+  I.e = lo;
+  const int nt = sprefix[lo + 1] - sprefix[lo];
+  const int local = it - p.m_tiles * sprefix[lo];
+  I.m = local / nt;
+  const int t = local - I.m * nt;
+  const int ch = __ldg(p.sched.chunk + lo);
+  const int cnt = __ldg(p.sched.row_count + lo);
+  I.r0 = __ldg(p.sched.row_start + lo) + t * ch;
+  I.nvalid = min(ch, cnt - t * ch);
+  return I;
+}
+
+// D[tmem] = A[tmem] * B[smem]^T, u8 x s8 -> s32, D overwritten (no accumulation)
+__device__ __forceinline__ void umma_i8_ts(uint32_t d, uint32_t a, uint64_t b, uint32_t idesc) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::i8 [%0], [%1], %2, %3, p;\n\t}\n" ::"r"(d),
+      "r"(a), "l"(b), "r"(idesc), "r"(0u)
+      : "memory");
+}
+
+// 32 lanes x NC consecutive 32-bit columns of tensor memory (NC = 2, 4, 8, 16)
+template <int NC>
+__device__ __forceinline__ void tmem_ldn(uint32_t taddr, uint32_t (&r)[NC]);
+template <>
+__device__ __forceinline__ void tmem_ldn<2>(uint32_t taddr, uint32_t (&r)[2]) {
+  asm volatile("tcgen05.ld.sync.aligned.32x32b.x2.b32 {%0, %1}, [%2];" : "=r"(r[0]), "=r"(r[1]) : "r"(taddr) : "memory");
+}
+template <>
+__device__ __forceinline__ void tmem_ldn<4>(uint32_t taddr, uint32_t (&r)[4]) {
+  asm volatile("tcgen05.ld.sync.aligned.32x32b.x4.b32 {%0, %1, %2, %3}, [%4];"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+               : "r"(taddr)
+               : "memory");
+}
+template <>
+__device__ __forceinline__ void tmem_ldn<8>(uint32_t taddr, uint32_t (&r)[8]) {
+  asm volatile("tcgen05.ld.sync.aligned.32x32b.x8.b32 {%0, %1, %2, %3, %4, %5, %6, %7}, [%8];"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7])
+               : "r"(taddr)
+               : "memory");
+}
+template <>
+__device__ __forceinline__ void tmem_ldn<16>(uint32_t taddr, uint32_t (&r)[16]) {
+  tmem_ld16(taddr, r);
+}
+// Bounded barrier among the 4 epilogue warps (an mbarrier of count 4, alternating phases).
+__device__ __forceinline__ bool epi_sync(uint64_t* bar, uint32_t& phase, volatile int* abort, uint64_t lim) {
+  __syncwarp();
+  if ((threadIdx.x & 31) == 0) mbar_arrive(bar);
+  const bool ok = __all_sync(0xffffffffu, mbar_wait(bar, phase, abort, lim));
+  phase ^= 1u;
+  return ok;
+}
+
+// position of K offset j inside its group of 8 in the plane layout: (0,2,4,6,1,3,5,7)
+__device__ __forceinline__ int plane_pos(int j) {
+  const int r = j & 7;
+  return (j & ~7) | ((r & 1) ? 4 + (r >> 1) : (r >> 1));
+}
+
+// fp32 accumulators of one epilogue thread's gate (or only) and up rows, per live token
+template <int NP>
+struct Promo {
+  float ag[NP], au[NP];
+};
+
+// Tokens [0, NP) of one D slot (groups g0 .. g0+SG-1 x NA matrices): loads their 2*NP columns
+// of every (group, matrix) in batches of at most 32 registers, one wait per batch.  swg/swu:
+// weight scales of this thread's rows per group; meta: the stage's meta words per token.
+template <int NA, int NP>
+__device__ __forceinline__ void promote_slot(uint32_t slot_addr, int nv, const int* meta, int g0,
+                                             const float (&swg)[SG], const float (&swu)[SG], Promo<NP>& P) {
+  constexpr int NC = 2 * NP, U = SG * NA;
+  constexpr int PER = (32 / NC) < U ? (32 / NC) : U;
+#pragma unroll
+  for (int b0 = 0; b0 < U; b0 += PER) {
+    uint32_t d[PER][NC];
+#pragma unroll
+    for (int u = 0; u < PER; ++u) tmem_ldn<NC>(slot_addr + (uint32_t)((b0 + u) * DC), d[u]);
+    tmem_ld_wait();
+#pragma unroll
+    for (int u = 0; u < PER; ++u) {
+      const int unit = b0 + u, gg = unit / NA, mat = unit % NA;
+      const float sw = mat ? swu[gg] : swg[gg];
+#pragma unroll
+      for (int c = 0; c < NP; ++c) {
+        if (c < nv) {
+          const int csum = meta[c * kMetaWords + g0 + gg];
+          const float xsc = __int_as_float(meta[c * kMetaWords + 8 + ((g0 + gg) >> 2)]);
+          const int gi = (int)d[u][2 * c] * 256 + (int)d[u][2 * c + 1] - 8 * csum;  // sum_k q*X exactly
+          if (mat)
+            P.au[c] = fmaf((float)gi, sw * xsc, P.au[c]);
+          else
+            P.ag[c] = fmaf((float)gi, sw * xsc, P.ag[c]);
+        }
+      }
+    }
+  }
+}
+
+// bf16 number g (0..7) of eight packed in a uint4, as fp32
+__device__ __forceinline__ float bf16_at(const uint4& v, int g) {
+  const uint32_t word = (g >> 1) == 0 ? v.x : (g >> 1) == 1 ? v.y : (g >> 1) == 2 ? v.z : v.w;
+  return __uint_as_float((g & 1) ? (word & 0xFFFF0000u) : (word << 16));
+}
+
+// The K loop of one work item for the promotion warps, specialised on the live-token bound NP.
+template <bool GATED, int NP>
+__device__ __forceinline__ bool promote_item(const Params& p, const Item& I, int mrow, int lane, uint32_t lane_base,
+                                             const uint8_t* smem, int& s, uint32_t& ph, uint64_t* full,
+                                             uint64_t* empty, int& ds, uint32_t& ph_d, uint64_t* d_full,
+                                             uint64_t* d_empty, volatile int* abort_flag, Promo<NP>& P) {
+  using C = Cfg<GATED>;
+  constexpr int NA = C::NA, DSL = C::DSLOTS, ST = C::ST;
+  const int K = p.K, nkb = ceil_div(K, KB), nv = I.nvalid;
+  const uint64_t lim = p.wait_limit;
+  for (int kb = 0; kb < nkb; ++kb) {
+    const int ng = min(KB, K - kb * KB) / G;
+    // the stage's meta words and weight scales (their copies completed long before; this wait
+    // also orders the reads after them)
+    if (!__all_sync(0xffffffffu, mbar_wait(&full[s], ph, abort_flag, lim))) return false;
+    const uint8_t* st = smem + s * C::STAGE;
+    const int* meta = reinterpret_cast<const int*>(st + C::META);
+    const uint4 sgv = *reinterpret_cast<const uint4*>(st + C::SCL + mrow * 16);
+    const uint4 suv = GATED ? *reinterpret_cast<const uint4*>(st + C::SCL + C::S_TILE + mrow * 16) : sgv;
+#pragma unroll
+    for (int g0 = 0; g0 < NG; g0 += SG) {  // unrolled: scale registers are indexed statically
+      if (g0 >= ng) break;
+      if (!__all_sync(0xffffffffu, mbar_wait(&d_full[ds], ph_d, abort_flag, lim))) return false;
+      tc_fence_after();
+      float swg[SG], swu[SG];
+#pragma unroll
+      for (int gg = 0; gg < SG; ++gg) {
+        swg[gg] = bf16_at(sgv, g0 + gg);
+        swu[gg] = bf16_at(suv, g0 + gg);
+      }
+      promote_slot<NA, NP>(lane_base + (uint32_t)(ds * C::D_SLOT), nv, meta, g0, swg, swu, P);
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&d_empty[ds]);
+      if (++ds == DSL) {
+        ds = 0;
+        ph_d ^= 1u;
+      }
+    }
+    __syncwarp();
+    if (lane == 0) mbar_arrive(&empty[s]);  // meta words read
+    if (++s == ST) {
+      s = 0;
+      ph ^= 1u;
+    }
+  }
+  return true;
+}
+
+// One work item of the promotion warps: the K loop, then the epilogue (GATED: h = SiLU(gate)
+// * up as fixed-point planes with one scale per (token, tile); else fp32 or bf16 rows).
+template <bool GATED, int NP>
+__device__ __forceinline__ bool epi_item(const Params& p, const Item& I, int ew, int lane, uint32_t lane_base,
+                                         const uint8_t* smem, int& s, uint32_t& ph, uint64_t* full, uint64_t* empty,
+                                         int& ds, uint32_t& ph_d, uint64_t* d_full, uint64_t* d_empty,
+                                         float* red, uint64_t* epi_bar, uint32_t& ph_e, volatile int* abort_flag) {
+  const int mrow = ew * 32 + lane, nv = I.nvalid;
+  Promo<NP> P;
+#pragma unroll
+  for (int c = 0; c < NP; ++c) P.ag[c] = P.au[c] = 0.f;
+  if (!promote_item<GATED, NP>(p, I, mrow, lane, lane_base, smem, s, ph, full, empty, ds, ph_d, d_full, d_empty,
+                               abort_flag, P))
+    return false;
+  if constexpr (GATED) {
+#pragma unroll
+    for (int c = 0; c < NP; ++c) {
+      const float h = P.ag[c] / (1.0f + __expf(-P.ag[c])) * P.au[c];
+      P.ag[c] = h;
+      float m = fabsf(h);
+#pragma unroll
+      for (int off = 16; off; off >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, off));
+      if (lane == 0) red[ew * NT + c] = m;
+    }
+    if (!epi_sync(epi_bar, ph_e, abort_flag, p.wait_limit)) return false;
+    const int j = I.m * BM + mrow;
+    const int pos = plane_pos(j);
+    const int mw_h = meta_words_per_row(p.I);
+    int8_t* planes = reinterpret_cast<int8_t*>(p.out);
+#pragma unroll
+    for (int c = 0; c < NP; ++c) {
+      if (c < nv) {
+        const float a = fmaxf(fmaxf(red[c], red[NT + c]), fmaxf(red[2 * NT + c], red[3 * NT + c]));
+        const float sc = fmaxf(a, 1e-30f) * (1.0f / 32639.0f);
+        const int X = __float2int_rn(__fdiv_rn(P.ag[c], sc));
+        const int h8 = (X + 128) >> 8;
+        const size_t o = (size_t)(2 * (I.r0 + c)) * p.out_ld + pos;
+        planes[o] = (int8_t)h8;
+        planes[o + p.out_ld] = (int8_t)(X - 256 * h8);
+        int sum = X;  // the 32 rows of this warp are one 32-group of h's K
+#pragma unroll
+        for (int off = 16; off; off >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, off);
+        // h's meta: stage I.m / 2, group (I.m & 1) * 4 + ew, block scale 8 + (I.m & 1)
+        int32_t* m = p.out_meta + (size_t)(I.r0 + c) * mw_h + (I.m >> 1) * kMetaWords;
+        if (lane == 0) m[(I.m & 1) * 4 + ew] = sum;
+        if (mrow == 0) m[8 + (I.m & 1)] = __float_as_int(sc);
+      }
+    }
+    return epi_sync(epi_bar, ph_e, abort_flag, p.wait_limit);  // red[] is reused by the next item
+  } else {
+    const int n = I.m * BM + mrow;
+    if (p.out_kind == OUT_F32) {
+      float* y = reinterpret_cast<float*>(p.out);
+#pragma unroll
+      for (int c = 0; c < NP; ++c)
+        if (c < nv) y[(size_t)(I.r0 + c) * p.out_ld + n] = P.ag[c];
+    } else {
+      __nv_bfloat16* y = reinterpret_cast<__nv_bfloat16*>(p.out);
+#pragma unroll
+      for (int c = 0; c < NP; ++c)
+        if (c < nv) y[(size_t)(I.r0 + c) * p.out_ld + n] = __float2bfloat16_rn(P.ag[c]);
+    }
+    return true;
+  }
+}
+
+template <bool GATED>
+__global__ void __launch_bounds__(kThreads, 1)
+    w4i8_gemm_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CUtensorMap tm_x,
+                     const __grid_constant__ CUtensorMap tm_m, const __grid_constant__ CUtensorMap tm_s,
+                     const Params p) {
+  using C = Cfg<GATED>;
+  constexpr int NA = C::NA, ST = C::ST, ASL = C::ASLOTS, DSL = C::DSLOTS;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + C::OFF_BAR);
+  uint64_t* empty = full + ST;
+  uint64_t* a_full = empty + ST;
+  uint64_t* a_empty = a_full + ASL;
+  uint64_t* d_full = a_empty + ASL;
+  uint64_t* d_empty = d_full + DSL;
+  uint64_t* drain = d_empty + DSL;
+  uint64_t* epi_bar = drain + 1;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::OFF_MISC);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::OFF_MISC + 4);
+  float* red = reinterpret_cast<float*>(smem + C::OFF_RED);
+  int* sprefix = reinterpret_cast<int*>(smem + C::OFF_PREFIX);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const uint64_t lim = p.wait_limit;
+
+  for (int i = threadIdx.x; i <= p.E; i += blockDim.x) sprefix[i] = __ldg(p.sched.tile_prefix + i);
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < ST; ++i) {
+      mbar_init(&full[i], p.scales_tma ? 1 : 1 + 32);
+      mbar_init(&empty[i], kNumUnpack + 1 + 4);  // unpack warps (words), MMA commit (planes), epilogue (meta)
+    }
+    for (int i = 0; i < ASL; ++i) {
+      mbar_init(&a_full[i], kNumUnpack);
+      mbar_init(&a_empty[i], 1);
+    }
+    for (int i = 0; i < DSL; ++i) {
+      mbar_init(&d_full[i], 1);
+      mbar_init(&d_empty[i], 4);
+    }
+    mbar_init(drain, 1);
+    mbar_init(epi_bar, 4);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 0 && lane == 0) {
+    prefetch_tmap(&tm_w);
+    prefetch_tmap(&tm_x);
+    prefetch_tmap(&tm_m);
+    if (p.scales_tma) prefetch_tmap(&tm_s);
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_slot, 512);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+  const int total = p.m_tiles * sprefix[p.E];
+  const int K = p.K;
+  const int nkb = ceil_div(K, KB);
+
+  if (warp == 0) {
+    // ---------------------------------------------------------------- producer
+    const uint64_t pol_w = policy_evict_first();
+    const uint64_t pol_b = policy_evict_last();
+    const int kg = K / G;
+    int s = 0, issued = 0;
+    uint32_t ph = 0;
+    bool ok = true;
+    for (int it = blockIdx.x; it < total && ok; it += gridDim.x) {
+      const Item I = decode_item(it, sprefix, p);
+      const int row_g = I.e * p.rows_per_expert + I.m * BM;
+      const int row_u = row_g + p.I;
+      for (int kb = 0; kb < nkb; ++kb) {
+        if (!(ok = __all_sync(0xffffffffu, mbar_wait(&empty[s], ph ^ 1u, abort_flag, lim)))) break;
+        uint8_t* st = smem + s * C::STAGE;
+        const int natom = min(KB, K - kb * KB) / 128;  // 2, or 1 for a half stage
+        if (lane == 0) {
+          uint32_t bytes = NA * C::W_TILE + natom * C::B_ATOM + C::META_BYTES;
+          if (p.scales_tma) bytes += NA * C::S_TILE;
+          mbar_arrive_expect_tx(&full[s], bytes);
+          tma_load_2d_hint(st, &tm_w, &full[s], kb * (KB / 8), row_g, pol_w);
+          if (GATED) tma_load_2d_hint(st + C::W_TILE, &tm_w, &full[s], kb * (KB / 8), row_u, pol_w);
+          for (int a = 0; a < natom; ++a)
+            tma_load_2d_hint(st + C::STAGE_B + a * C::B_ATOM, &tm_x, &full[s], kb * KB + a * 128, 2 * I.r0, pol_b);
+          tma_load_2d_hint(st + C::META, &tm_m, &full[s], kb * kMetaWords, I.r0, pol_b);
+          if (p.scales_tma) {
+            tma_load_2d_hint(st + C::SCL, &tm_s, &full[s], kb * NG, row_g, pol_w);
+            if (GATED) tma_load_2d_hint(st + C::SCL + C::S_TILE, &tm_s, &full[s], kb * NG, row_u, pol_w);
+          }
+        }
+        if (!p.scales_tma) {  // scale rows 8-byte aligned: 8 or 4 bf16 per row by cp.async
+#pragma unroll
+          for (int mat = 0; mat < NA; ++mat) {
+            const int row0 = mat ? row_u : row_g;
+            for (int rr = lane; rr < BM; rr += 32) {
+              const uint16_t* src = p.w_s + (size_t)(row0 + rr) * kg + kb * NG;
+              uint8_t* dst = st + C::SCL + mat * C::S_TILE + rr * 16;
+              cp_async_8(dst, src);
+              if (natom == 2) cp_async_8(dst + 8, src + 4);
+            }
+          }
+          cp_async_arrive_noinc(&full[s]);
+        }
+        ++issued;
+        if (++s == ST) {
+          s = 0;
+          ph ^= 1u;
+        }
+      }
+    }
+    if (lane == 0)
+      for (int i = max(0, issued - ST); i < issued; ++i) mbar_wait_plain(&full[i % ST], (i / ST) & 1, lim);
+  } else if (warp == 1) {
+    // ---------------------------------------------------------------- MMA issuer
+    if (lane == 0) {
+      // u8 A x s8 B -> s32, M = 128, N = DC (NT tokens x (hi, lo))
+      const uint32_t idesc = (2u << 4) | (0u << 7) | (1u << 10) | ((uint32_t)(DC >> 3) << 17) |
+                             ((uint32_t)(BM >> 4) << 24);
+      int s = 0, as = 0, ds = 0;
+      uint32_t ph = 0, ph_a = 0, ph_d = 0;
+      bool ok = true;
+      for (int it = blockIdx.x; it < total && ok; it += gridDim.x) {
+        for (int kb = 0; kb < nkb && ok; ++kb) {
+          const int ng = min(KB, K - kb * KB) / G;
+          if (!(ok = mbar_wait(&full[s], ph, abort_flag, lim))) break;
+          if (!(ok = mbar_wait(&a_full[as], ph_a, abort_flag, lim))) break;
+          const uint8_t* st = smem + s * C::STAGE;
+          const uint32_t a_slot = tmem_base + (uint32_t)(C::A_COL0 + as * C::A_SLOT);
+          for (int g0 = 0; g0 < ng; g0 += SG) {
+            if (!(ok = mbar_wait(&d_empty[ds], ph_d ^ 1u, abort_flag, lim))) break;
+            tc_fence_after();
+#pragma unroll
+            for (int gg = 0; gg < SG; ++gg) {
+              const int g = g0 + gg;
+              const uint64_t b = sw128_kmajor_desc(smem_u32(st + C::STAGE_B + (g >> 2) * C::B_ATOM)) + 2 * (g & 3);
+#pragma unroll
+              for (int mat = 0; mat < NA; ++mat) {
+                const uint32_t d = tmem_base + (uint32_t)(ds * C::D_SLOT + (gg * NA + mat) * DC);
+                umma_i8_ts(d, a_slot + (uint32_t)(mat * NG * 8 + g * 8), b, idesc);
+              }
+            }
+            umma_commit(&d_full[ds]);
+            if (++ds == DSL) {
+              ds = 0;
+              ph_d ^= 1u;
+            }
+          }
+          if (!ok) break;
+          umma_commit(&a_empty[as]);
+          umma_commit(&empty[s]);
+          if (++as == ASL) {
+            as = 0;
+            ph_a ^= 1u;
+          }
+          if (++s == ST) {
+            s = 0;
+            ph ^= 1u;
+          }
+        }
+      }
+      umma_commit(drain);
+      mbar_wait_plain(drain, 0, lim);
+    }
+  } else if (warp >= kEpiWarp0 && warp < kEpiWarp0 + 4) {
+    // ---------------------------------------------------------------- promotion + epilogue
+    const int ew = warp - kEpiWarp0;  // == warp % 4: TMEM lanes 32*ew..
+    const uint32_t lane_base = tmem_base + ((uint32_t)(ew * 32) << 16);
+    int ds = 0, s = 0;
+    uint32_t ph_d = 0, ph_e = 0, ph = 0;
+    bool ok = true;
+    for (int it = blockIdx.x; it < total && ok; it += gridDim.x) {
+      const Item I = decode_item(it, sprefix, p);
+      const int nv = I.nvalid;
+#define MOE_EPI_ITEM(NP_)                                                                                           \
+  epi_item<GATED, NP_>(p, I, ew, lane, lane_base, smem, s, ph, full, empty, ds, ph_d, d_full, d_empty, red, epi_bar, \
+                       ph_e, abort_flag)
+      if (nv <= 1)
+        ok = MOE_EPI_ITEM(1);
+      else if (nv <= 2)
+        ok = MOE_EPI_ITEM(2);
+      else if (nv <= 4)
+        ok = MOE_EPI_ITEM(4);
+      else
+        ok = MOE_EPI_ITEM(8);
+#undef MOE_EPI_ITEM
+    }
+  } else if (warp >= kUnpackWarp0) {
+    // ---------------------------------------------------------------- INT4 -> u8 rows of TMEM
+    // GATED: warps 8-11 gate rows, 12-15 up rows, a thread = a row, the whole stage;
+    // plain: a thread = a row and one 128-K half of the stage.
+    const int uw = warp - kUnpackWarp0;
+    const int row = (uw & 3) * 32 + lane;
+    const int sw = row & 7;
+    const int mat = GATED ? (uw >> 2) : 0;
+    const int half = GATED ? 0 : (uw >> 2);
+    constexpr int CHK = GATED ? 8 : 4;  // 16-byte chunks (32 K each) this thread unpacks per stage
+    const uint32_t lane_base = tmem_base + ((uint32_t)((uw & 3) * 32) << 16);
+    int s = 0, as = 0;
+    uint32_t ph = 0, ph_a = 0;
+    bool ok = true;
+    for (int it = blockIdx.x; it < total && ok; it += gridDim.x) {
+      for (int kb = 0; kb < nkb && ok; ++kb) {
+        const int ng = min(KB, K - kb * KB) / G;
+        ok = __all_sync(0xffffffffu, mbar_wait(&full[s], ph, abort_flag, lim));
+        if (!ok) break;
+        const uint8_t* wrow = smem + s * C::STAGE + mat * C::W_TILE + row * 128;
+        uint4 wv[CHK];
+#pragma unroll
+        for (int c = 0; c < CHK; ++c) {
+          const int lc = GATED ? c : 4 * half + c;  // logical 16-byte chunk = 32-K group
+          wv[c] = *reinterpret_cast<const uint4*>(wrow + ((lc ^ sw) << 4));
+        }
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&empty[s]);  // words are in registers
+        if (++s == ST) {
+          s = 0;
+          ph ^= 1u;
+        }
+        ok = __all_sync(0xffffffffu, mbar_wait(&a_empty[as], ph_a ^ 1u, abort_flag, lim));
+        if (!ok) break;
+        tc_fence_after();
+        // group g's 32 K = 4 words -> 8 columns of 4 bytes; word w gives K offsets
+        // (0,2,4,6) then (1,3,5,7) as offset-binary bytes n = q + 8
+        uint32_t r[CHK * 8];
+#pragma unroll
+        for (int c = 0; c < CHK; ++c) {
+          const uint32_t w4[4] = {wv[c].x, wv[c].y, wv[c].z, wv[c].w};
+#pragma unroll
+          for (int w = 0; w < 4; ++w) {
+            const uint32_t n = w4[w] ^ 0x88888888u;
+            r[c * 8 + 2 * w] = n & 0x0F0F0F0Fu;
+            r[c * 8 + 2 * w + 1] = (n >> 4) & 0x0F0F0F0Fu;
+          }
+        }
+        const uint32_t col0 = (uint32_t)(C::A_COL0 + as * C::A_SLOT + mat * NG * 8 + (GATED ? 0 : half * 32));
+        if constexpr (GATED) {
+          uint32_t r0[32], r1[32];
+#pragma unroll
+          for (int i = 0; i < 32; ++i) r0[i] = r[i], r1[i] = r[32 + i];
+          tmem_st32(lane_base + col0, r0);
+          if (ng > 4) tmem_st32(lane_base + col0 + 32, r1);
+        } else {
+          uint32_t r0[32];
+#pragma unroll
+          for (int i = 0; i < 32; ++i) r0[i] = r[i];
+          if (ng > 4 * half) tmem_st32(lane_base + col0, r0);
+        }
+        tmem_st_wait();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&a_full[as]);
+        if (++as == ASL) {
+          as = 0;
+          ph_a ^= 1u;
+        }
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem_base, 512);
+  }
+}
+
+template <bool GATED>
+cudaError_t launch_t(const W4I8Problem& pr, cudaStream_t s) {
+  using C = Cfg<GATED>;
+  CUtensorMap tm_w, tm_x, tm_m, tm_s;
+  const uint64_t wrows = (uint64_t)pr.E * pr.rows_per_expert;
+  if (encode_tmap_2d(&tm_w, pr.w_q, CU_TENSOR_MAP_DATA_TYPE_INT32, pr.K / 8, wrows, (uint64_t)pr.K / 2, KB / 8, BM,
+                     CU_TENSOR_MAP_SWIZZLE_128B) != CUDA_SUCCESS)
+    return cudaErrorInvalidValue;
+  if (encode_tmap_2d(&tm_x, pr.act, CU_TENSOR_MAP_DATA_TYPE_UINT8, pr.K, 2 * (uint64_t)pr.act_rows, (uint64_t)pr.K,
+                     128, 2 * NT, CU_TENSOR_MAP_SWIZZLE_128B) != CUDA_SUCCESS)
+    return cudaErrorInvalidValue;
+  const int mw = meta_words_per_row(pr.K);
+  if (encode_tmap_2d(&tm_m, pr.act_meta, CU_TENSOR_MAP_DATA_TYPE_INT32, mw, (uint64_t)pr.act_rows, (uint64_t)mw * 4,
+                     kMetaWords, NT, CU_TENSOR_MAP_SWIZZLE_NONE) != CUDA_SUCCESS)
+    return cudaErrorInvalidValue;
+  const int scales_tma = (pr.K % KB) == 0;  // scale rows are then a multiple of 16 bytes
+  if (scales_tma) {
+    if (encode_tmap_2d(&tm_s, pr.w_s, CU_TENSOR_MAP_DATA_TYPE_UINT16, pr.K / G, wrows, (uint64_t)pr.K / 16, NG, BM,
+                       CU_TENSOR_MAP_SWIZZLE_NONE) != CUDA_SUCCESS)
+      return cudaErrorInvalidValue;
+  } else {
+    tm_s = tm_w;  // unused
+  }
+  Params p;
+  p.K = pr.K;
+  p.scales_tma = scales_tma;
+  p.E = pr.E;
+  p.rows_per_expert = pr.rows_per_expert;
+  p.I = pr.I;
+  p.m_tiles = GATED ? pr.I / BM : pr.rows_per_expert / BM;
+  p.w_s = pr.w_s;
+  p.sched = pr.sched;
+  p.out_kind = pr.out_kind;
+  p.out = pr.out;
+  p.out_meta = pr.out_meta;
+  p.out_ld = pr.out_ld;
+  p.wait_limit = wait_limit_ns();
+  const size_t smem = C::smem_bytes(pr.E);
+  auto kern = w4i8_gemm_kernel<GATED>;
+  cudaError_t err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (err != cudaSuccess) return err;
+  const char* name = GATED ? "w4a16_gemm_gate_up" : "w4a16_gemm_down";
+  timing_before(name, s);
+  kern<<<sm_count(), kThreads, smem, s>>>(tm_w, tm_x, tm_m, tm_s, p);
+  timing_after(name, s);
+  return cudaGetLastError();
+}
+
+}  // namespace w4i8
+
+cudaError_t launch_w4i8_gemm(const W4I8Problem& p, cudaStream_t s) {
+  return p.gated ? w4i8::launch_t<true>(p, s) : w4i8::launch_t<false>(p, s);
+}
+
+}  // namespace moe

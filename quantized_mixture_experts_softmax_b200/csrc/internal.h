@@ -43,7 +43,7 @@ cudaError_t launch_combine(const float* y_perm, const int32_t* inv_pos, const fl
                            void* out, int out_fp32, cudaStream_t s);
 
 // W4A16 grouped GEMM (gemm_w4a16.cu)
-enum OutKind { OUT_H_F16_INTERLEAVED = 0, OUT_F32 = 1, OUT_BF16 = 2 };
+enum OutKind { OUT_H_F16_INTERLEAVED = 0, OUT_F32 = 1, OUT_BF16 = 2, OUT_PLANES = 3 };
 struct W4GemmProblem {
   const int32_t* w_q;  // [E, rows_per_expert, K/8]
   const uint16_t* w_s; // [E, rows_per_expert, K/32]
@@ -59,6 +59,36 @@ struct W4GemmProblem {
   OutKind out_kind;
 };
 cudaError_t launch_w4a16_gemm(const W4GemmProblem& p, cudaStream_t s);
+
+// W4A16 grouped GEMM for decode-sized experts on the int8 tensor cores (gemm_w4i8.cu).
+// Activations as 16-bit fixed-point planes: per (row, 128-K block) scale s, X = rint(x/s)
+// = 256*hi + lo.  Plane matrix int8 [2*rows, K]: row 2r holds hi of row r, row 2r+1 its lo,
+// with K in the order (0,2,4,6,1,3,5,7) inside every 8-group.  Meta int32 [rows, ceil(K/256),
+// 12]: per 256-K stage the sums of X over its eight 32-K groups, then the scales of its two
+// 128-K blocks (fp32 bits), then two unused words.
+constexpr int kMetaWords = 12;
+__host__ __device__ inline int meta_words_per_row(int K) { return (K + 255) / 256 * kMetaWords; }
+struct W4I8Problem {
+  const int32_t* w_q;   // [E, rows_per_expert, K/8]
+  const uint16_t* w_s;  // [E, rows_per_expert, K/32]
+  const int8_t* act;    // planes [2*act_rows, K]
+  const int32_t* act_meta;
+  int act_rows;
+  int K, E, rows_per_expert;
+  bool gated;  // output planes of h [2*act_rows, I]
+  int I;
+  TileSched sched;
+  OutKind out_kind;  // OUT_PLANES (gated), OUT_F32 or OUT_BF16
+  void* out;
+  int32_t* out_meta;  // planes only: meta of h
+  int out_ld;         // OUT_F32/OUT_BF16: elements per output row (planes: I)
+};
+constexpr int kI8TileRows = 8;  // token rows per tile of the int8 GEMM
+cudaError_t launch_w4i8_gemm(const W4I8Problem& p, cudaStream_t s);
+// Planes of the K-vectors x_src: plane row r takes source row r (inv_pos == null, k == 1),
+// or for every pair p plane row inv_pos[p] takes source row p / k.
+cudaError_t launch_planes(const uint16_t* a, int a_is_bf16, const int32_t* inv_pos, int n_pairs, int k, int K,
+                          int8_t* planes, int32_t* meta, cudaStream_t s);
 
 // block-FP8 grouped GEMM (gemm_fp8.cu)
 struct F8GemmProblem {

@@ -4,5 +4,6 @@
 #include "permute_combine.cu"
 #include "gemm_w4a16.cu"
 #include "gemm_fp8.cu"
+#include "gemm_w4i8.cu"
 #include "api.cu"
 #include "align_noalloc.cu"

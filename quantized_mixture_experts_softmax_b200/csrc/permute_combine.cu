@@ -83,6 +83,86 @@ cudaError_t launch_permute_fp8(const uint8_t* x, const float* xs, const int32_t*
   return cudaGetLastError();
 }
 
+// 16-bit fixed-point planes of activation rows.  16 threads per (row, 128-K block), 8 K
+// elements each: s = max(amax, 1e-30) / 32639, X = rint(x / s) = 256*hi + lo with hi =
+// floor((X + 128) / 256) in [-127, 127] and lo in [-128, 127]; hi goes to plane row 2r, lo to
+// 2r+1, bytes in the order (0,2,4,6,1,3,5,7) of each 8-group (the order in which a packed INT4
+// word unpacks); the sum of X over every 32-K group (for the MMA's offset correction) and the
+// block scales go to the row's meta words.
+__global__ void __launch_bounds__(256) planes_kernel(const uint4* __restrict__ a, int a_is_bf16,
+                                                     const int32_t* __restrict__ inv_pos, int n_pairs, int k, int K,
+                                                     uint2* __restrict__ planes, int32_t* __restrict__ meta) {
+  const int nblk = K / 128;
+  const size_t unit = (blockIdx.x * (size_t)blockDim.x + threadIdx.x) >> 4;  // (pair, block)
+  const int i = threadIdx.x & 15;                                             // 8-group within the block
+  const bool live = unit < (size_t)n_pairs * nblk;
+  const int p = live ? (int)(unit / nblk) : 0;
+  const int blk = live ? (int)(unit % nblk) : 0;
+  const int r = live ? (inv_pos ? inv_pos[p] : p) : -1;
+  const int src = p / k;
+  float x[8];
+  float amax = 0.f;
+  if (live && r >= 0) {
+    const uint4 v = __ldg(a + ((size_t)src * K + blk * 128 + 8 * i) / 8);
+    const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      if (a_is_bf16) {
+        x[2 * j] = __uint_as_float(w[j] << 16);
+        x[2 * j + 1] = __uint_as_float(w[j] & 0xFFFF0000u);
+      } else {
+        const __half2 h = *reinterpret_cast<const __half2*>(&w[j]);
+        x[2 * j] = __low2float(h);
+        x[2 * j + 1] = __high2float(h);
+      }
+    }
+#pragma unroll
+    for (int j = 0; j < 8; ++j) amax = fmaxf(amax, fabsf(x[j]));
+  } else {
+#pragma unroll
+    for (int j = 0; j < 8; ++j) x[j] = 0.f;
+  }
+#pragma unroll
+  for (int off = 8; off; off >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, off));  // 16 lanes
+  const float sc = fmaxf(amax, 1e-30f) * (1.0f / 32639.0f);
+  int X[8], sum = 0;
+#pragma unroll
+  for (int j = 0; j < 8; ++j) {
+    X[j] = __float2int_rn(__fdiv_rn(x[j], sc));
+    sum += X[j];
+  }
+  sum += __shfl_xor_sync(0xffffffffu, sum, 1);
+  sum += __shfl_xor_sync(0xffffffffu, sum, 2);  // 4 threads = one 32-K group
+  if (!live || r < 0) return;
+  constexpr int ord[8] = {0, 2, 4, 6, 1, 3, 5, 7};
+  uint32_t hb[2] = {0, 0}, lb[2] = {0, 0};
+#pragma unroll
+  for (int q = 0; q < 8; ++q) {
+    const int v = X[ord[q]];
+    const int h8 = (v + 128) >> 8;
+    const int l8 = v - 256 * h8;
+    hb[q >> 2] |= (uint32_t)(h8 & 0xFF) << (8 * (q & 3));
+    lb[q >> 2] |= (uint32_t)(l8 & 0xFF) << (8 * (q & 3));
+  }
+  const size_t o = ((size_t)(2 * r) * K + blk * 128 + 8 * i) / 8;
+  planes[o] = make_uint2(hb[0], hb[1]);
+  planes[o + K / 8] = make_uint2(lb[0], lb[1]);
+  int32_t* m = meta + (size_t)r * meta_words_per_row(K) + (blk >> 1) * kMetaWords;
+  if ((i & 3) == 0) m[(blk & 1) * 4 + (i >> 2)] = sum;
+  if (i == 0) m[8 + (blk & 1)] = __float_as_int(sc);
+}
+
+cudaError_t launch_planes(const uint16_t* a, int a_is_bf16, const int32_t* inv_pos, int n_pairs, int k, int K,
+                          int8_t* planes, int32_t* meta, cudaStream_t s) {
+  const size_t threads = (size_t)n_pairs * (K / 128) * 16;
+  timing_before("planes", s);
+  planes_kernel<<<(unsigned)((threads + 255) / 256), 256, 0, s>>>(reinterpret_cast<const uint4*>(a), a_is_bf16,
+                                                                  inv_pos, n_pairs, k, K, reinterpret_cast<uint2*>(planes),
+                                                                  meta);
+  timing_after("planes", s);
+  return cudaGetLastError();
+}
+
 __global__ void __launch_bounds__(256) convert_rows_kernel(const uint4* __restrict__ a, int a_is_bf16, size_t n8,
                                                            uint4* __restrict__ out) {
   for (size_t i = blockIdx.x * (size_t)blockDim.x + threadIdx.x; i < n8; i += (size_t)gridDim.x * blockDim.x) {

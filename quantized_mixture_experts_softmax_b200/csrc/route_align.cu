@@ -132,7 +132,8 @@ __device__ __forceinline__ int block_exclusive_scan(int v, int* warp_tot, int* t
   return r;
 }
 
-// token tiles of an expert with `c` rows, at most `nmax` rows each, balanced, rows a multiple of 16
+// token tiles of an expert with `c` rows, at most `nmax` rows each, balanced, rows a multiple of
+// min(nmax, 16)
 __device__ __forceinline__ void expert_tiles(int c, int nmax, int* nt, int* ch) {
   if (c <= 0) {
     *nt = 0;
@@ -140,8 +141,9 @@ __device__ __forceinline__ void expert_tiles(int c, int nmax, int* nt, int* ch) 
     return;
   }
   const int nt0 = (c + nmax - 1) / nmax;
+  const int q = nmax < 16 ? nmax : 16;
   int chunk = (c + nt0 - 1) / nt0;
-  chunk = (chunk + 15) / 16 * 16;
+  chunk = (chunk + q - 1) / q * q;
   *ch = chunk;
   *nt = (c + chunk - 1) / chunk;
 }
