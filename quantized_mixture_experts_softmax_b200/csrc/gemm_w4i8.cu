@@ -8,22 +8,29 @@
 // the format (the Chord article, second paragraph: one BF16 scale per 32 weights).
 //
 // The 16-bit activations enter as 16-bit fixed point: per (token, 128-K block) a scale
-// s = amax / 32639 and integers X = rint(x / s) split into two signed 8-bit planes
+// s = amax / 16383 and integers X = rint(x / s) split into two signed 8-bit planes
 // X = 256*hi + lo, interleaved along N (tile row 2c = hi of token c, 2c+1 = its lo; 8 tokens
 // give N = 16, the smallest N of a 128-row MMA).  For one
 // token t and one weight row r, one MMA per 32-K group g gives D_hi and D_lo exactly in int32:
 //     sum_{k in g} q[r][k] * X[t][k] = 256*D_hi + D_lo - 8*C[t][g],   C[t][g] = sum_{k in g} X[t][k],
-// which the promotion warps scale by the group's weight scale and the block's activation
-// scale and accumulate in fp32.  They read from tensor memory only the columns of the tile's
-// live tokens (2, 4, 8 or 16 columns of each MMA's 16), batched under one wait; the tokens' group sums and
-// block scales arrive with the stage (one TMA box of the meta words), as do the weight scales.  The gate/up kernel ends with
-// h = SiLU(gate) * up written straight back in the same fixed-point planes (one scale per
-// token per 128-row tile) for the down kernel.
+// (|sum| < 2^22, so adding it to the bits of 1.5 * 2^23 converts it to fp32 exactly), which the
+// promotion warps scale by the group's weight scale and the block's activation scale and
+// accumulate in fp32.  They read from tensor memory only the columns of the tile's live
+// tokens (2, 4, 8 or 16 columns of each MMA's 16), batched under one wait; the tokens' group
+// sums and block scales arrive with the stage (one TMA box of the meta words), as do the weight
+// scales.  The gate/up kernel ends with h = SiLU(gate) * up written straight back in the same
+// fixed-point planes (one scale per token per 128-row tile) for the down kernel.
+//
+// The MMA-issuing thread never waits on an mbarrier: a wait (or any shared-memory access) by
+// the thread that has MMAs in flight stalls until they drain, idling the tensor core for
+// hundreds of cycles per wait.  A scheduler warp does the waits and releases the MMA warp
+// through a named barrier with an AND reduction (which also carries a timeout or abort).
 //
 // Work list, swap (weights in the MMA's M slot) and persistence as in the fp16 GEMM.  Warps
 // (512 threads): 0 producer (TMA of the INT4 words, weight scales, activation planes and meta
-// words of the token tile per 256-K stage; cp.async for scale rows not 16-byte aligned), 1 TMEM allocator + MMA issuer, 4-7 promotion and epilogue, 8-15 unpacking INT4
-// words into u8 rows of tensor memory (the MMA's A operand).
+// words of the token tile per 256-K stage; cp.async for scale rows not 16-byte aligned),
+// 1 TMEM allocator + MMA issuer, 2 MMA scheduler, 4-7 promotion and epilogue, 8-15 unpacking
+// INT4 words into u8 rows of tensor memory (the MMA's A operand).
 #include "common.cuh"
 #include "internal.h"
 
@@ -38,6 +45,9 @@ constexpr int NT = kI8TileRows;  // token rows per tile (each gives a hi and a l
 constexpr int DC = 2 * NT;       // D columns of one MMA (N)
 constexpr int SG = 4;            // groups per D slot
 constexpr int kThreads = 512;
+constexpr int kMmaWarp = 1;
+constexpr int kSchedWarp = 2;
+constexpr int kMmaBarrier = 1;  // named barrier of the MMA and scheduler warps (0 is __syncthreads)
 constexpr int kEpiWarp0 = 4;
 constexpr int kUnpackWarp0 = 8;
 constexpr int kNumUnpack = 8;
@@ -59,7 +69,7 @@ struct Cfg {
   // TMEM: D ring of SG-group slots [group][matrix][DC int32 columns], A ring of whole-stage
   // slots [matrix][group][8 columns] (a 32-K row of u8 = 8 columns)
   static constexpr int D_SLOT = SG * NA * DC;
-  static constexpr int DSLOTS = GATED ? 2 : 4;
+  static constexpr int DSLOTS = 256 / D_SLOT;
   static constexpr int A_SLOT = NA * NG * 8;
   static constexpr int ASLOTS = GATED ? 2 : 4;
   static constexpr int A_COL0 = DSLOTS * D_SLOT;
@@ -111,6 +121,20 @@ __device__ __forceinline__ Item decode_item(int it, const int* __restrict__ spre
   I.r0 = __ldg(p.sched.row_start + lo) + t * ch;
   I.nvalid = min(ch, cnt - t * ch);
   return I;
+}
+
+// Named barrier `id` over `n` threads that also returns the AND of every thread's `in`.
+__device__ __forceinline__ bool bar_red_and(int id, int n, bool in) {
+  uint32_t r;
+  asm volatile(
+      "{\n\t.reg .pred pi, po;\n\t"
+      "setp.ne.u32 pi, %1, 0;\n\t"
+      "bar.red.and.pred po, %2, %3, pi;\n\t"
+      "selp.u32 %0, 1, 0, po;\n\t}\n"
+      : "=r"(r)
+      : "r"((uint32_t)in), "r"(id), "r"(n)
+      : "memory");
+  return r != 0;
 }
 
 // D[tmem] = A[tmem] * B[smem]^T, u8 x s8 -> s32, D overwritten (no accumulation)
@@ -173,7 +197,7 @@ struct Promo {
 // of every (group, matrix) in batches of at most 32 registers, one wait per batch.  swg/swu:
 // weight scales of this thread's rows per group; meta: the stage's meta words per token.
 template <int NA, int NP>
-__device__ __forceinline__ void promote_slot(uint32_t slot_addr, int nv, const int* meta, int g0,
+__device__ __forceinline__ void promote_slot(uint32_t slot_addr, const int* meta, int g0,
                                              const float (&swg)[SG], const float (&swu)[SG], Promo<NP>& P) {
   constexpr int NC = 2 * NP, U = SG * NA;
   constexpr int PER = (32 / NC) < U ? (32 / NC) : U;
@@ -187,17 +211,18 @@ __device__ __forceinline__ void promote_slot(uint32_t slot_addr, int nv, const i
     for (int u = 0; u < PER; ++u) {
       const int unit = b0 + u, gg = unit / NA, mat = unit % NA;
       const float sw = mat ? swu[gg] : swg[gg];
+      // all NP columns are promoted: those of tokens >= nv hold finite values of other rows and
+      // are never stored
 #pragma unroll
       for (int c = 0; c < NP; ++c) {
-        if (c < nv) {
-          const int csum = meta[c * kMetaWords + g0 + gg];
-          const float xsc = __int_as_float(meta[c * kMetaWords + 8 + ((g0 + gg) >> 2)]);
-          const int gi = (int)d[u][2 * c] * 256 + (int)d[u][2 * c + 1] - 8 * csum;  // sum_k q*X exactly
-          if (mat)
-            P.au[c] = fmaf((float)gi, sw * xsc, P.au[c]);
-          else
-            P.ag[c] = fmaf((float)gi, sw * xsc, P.ag[c]);
-        }
+        const int bias = meta[c * kMetaWords + g0 + gg];  // kFixBias - 8 * C[c][g]
+        const float xsc = __int_as_float(meta[c * kMetaWords + 8 + ((g0 + gg) >> 2)]);
+        const int t = (int)d[u][2 * c] * 256 + (int)d[u][2 * c + 1] + bias;
+        const float v = __int_as_float(t) - kFixBiasF;  // sum_k q*X, exactly
+        if (mat)
+          P.au[c] = fmaf(v, sw * xsc, P.au[c]);
+        else
+          P.ag[c] = fmaf(v, sw * xsc, P.ag[c]);
       }
     }
   }
@@ -217,7 +242,7 @@ __device__ __forceinline__ bool promote_item(const Params& p, const Item& I, int
                                              uint64_t* d_empty, volatile int* abort_flag, Promo<NP>& P) {
   using C = Cfg<GATED>;
   constexpr int NA = C::NA, DSL = C::DSLOTS, ST = C::ST;
-  const int K = p.K, nkb = ceil_div(K, KB), nv = I.nvalid;
+  const int K = p.K, nkb = ceil_div(K, KB);
   const uint64_t lim = p.wait_limit;
   for (int kb = 0; kb < nkb; ++kb) {
     const int ng = min(KB, K - kb * KB) / G;
@@ -239,7 +264,7 @@ __device__ __forceinline__ bool promote_item(const Params& p, const Item& I, int
         swg[gg] = bf16_at(sgv, g0 + gg);
         swu[gg] = bf16_at(suv, g0 + gg);
       }
-      promote_slot<NA, NP>(lane_base + (uint32_t)(ds * C::D_SLOT), nv, meta, g0, swg, swu, P);
+      promote_slot<NA, NP>(lane_base + (uint32_t)(ds * C::D_SLOT), meta, g0, swg, swu, P);
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&d_empty[ds]);
@@ -291,7 +316,7 @@ __device__ __forceinline__ bool epi_item(const Params& p, const Item& I, int ew,
     for (int c = 0; c < NP; ++c) {
       if (c < nv) {
         const float a = fmaxf(fmaxf(red[c], red[NT + c]), fmaxf(red[2 * NT + c], red[3 * NT + c]));
-        const float sc = fmaxf(a, 1e-30f) * (1.0f / 32639.0f);
+        const float sc = fmaxf(a, 1e-30f) * (1.0f / kFixMax);
         const int X = __float2int_rn(__fdiv_rn(P.ag[c], sc));
         const int h8 = (X + 128) >> 8;
         const size_t o = (size_t)(2 * (I.r0 + c)) * p.out_ld + pos;
@@ -302,7 +327,7 @@ __device__ __forceinline__ bool epi_item(const Params& p, const Item& I, int ew,
         for (int off = 16; off; off >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, off);
         // h's meta: stage I.m / 2, group (I.m & 1) * 4 + ew, block scale 8 + (I.m & 1)
         int32_t* m = p.out_meta + (size_t)(I.r0 + c) * mw_h + (I.m >> 1) * kMetaWords;
-        if (lane == 0) m[(I.m & 1) * 4 + ew] = sum;
+        if (lane == 0) m[(I.m & 1) * 4 + ew] = kFixBias - 8 * sum;
         if (mrow == 0) m[8 + (I.m & 1)] = __float_as_int(sc);
       }
     }
@@ -353,7 +378,9 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (threadIdx.x == 0) {
     for (int i = 0; i < ST; ++i) {
       mbar_init(&full[i], p.scales_tma ? 1 : 1 + 32);
-      mbar_init(&empty[i], kNumUnpack + 1 + 4);  // unpack warps (words), MMA commit (planes), epilogue (meta)
+      // unpack warps (words) and epilogue warps (meta, scales; they finish a stage only after
+      // its last MMA completed, so the planes are free too)
+      mbar_init(&empty[i], kNumUnpack + 4);
     }
     for (int i = 0; i < ASL; ++i) {
       mbar_init(&a_full[i], kNumUnpack);
@@ -438,24 +465,23 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     if (lane == 0)
       for (int i = max(0, issued - ST); i < issued; ++i) mbar_wait_plain(&full[i % ST], (i / ST) & 1, lim);
-  } else if (warp == 1) {
+  } else if (warp == kMmaWarp) {
     // ---------------------------------------------------------------- MMA issuer
-    if (lane == 0) {
-      // u8 A x s8 B -> s32, M = 128, N = DC (NT tokens x (hi, lo))
-      const uint32_t idesc = (2u << 4) | (0u << 7) | (1u << 10) | ((uint32_t)(DC >> 3) << 17) |
-                             ((uint32_t)(BM >> 4) << 24);
-      int s = 0, as = 0, ds = 0;
-      uint32_t ph = 0, ph_a = 0, ph_d = 0;
-      bool ok = true;
-      for (int it = blockIdx.x; it < total && ok; it += gridDim.x) {
-        for (int kb = 0; kb < nkb && ok; ++kb) {
-          const int ng = min(KB, K - kb * KB) / G;
-          if (!(ok = mbar_wait(&full[s], ph, abort_flag, lim))) break;
-          if (!(ok = mbar_wait(&a_full[as], ph_a, abort_flag, lim))) break;
-          const uint8_t* st = smem + s * C::STAGE;
-          const uint32_t a_slot = tmem_base + (uint32_t)(C::A_COL0 + as * C::A_SLOT);
-          for (int g0 = 0; g0 < ng; g0 += SG) {
-            if (!(ok = mbar_wait(&d_empty[ds], ph_d ^ 1u, abort_flag, lim))) break;
+    // Released slot by slot by the scheduler warp; identical loop bounds on both sides, so
+    // both take the same number of named-barrier steps.
+    // u8 A x s8 B -> s32, M = 128, N = DC (NT tokens x (hi, lo))
+    const uint32_t idesc = (2u << 4) | (0u << 7) | (1u << 10) | ((uint32_t)(DC >> 3) << 17) |
+                           ((uint32_t)(BM >> 4) << 24);
+    int s = 0, as = 0, ds = 0;
+    bool ok = true;
+    for (int it = blockIdx.x; it < total && ok; it += gridDim.x) {
+      for (int kb = 0; kb < nkb && ok; ++kb) {
+        const int ng = min(KB, K - kb * KB) / G;
+        const uint8_t* st = smem + s * C::STAGE;
+        const uint32_t a_slot = tmem_base + (uint32_t)(C::A_COL0 + as * C::A_SLOT);
+        for (int g0 = 0; g0 < ng; g0 += SG) {
+          if (!(ok = bar_red_and(kMmaBarrier, 64, true))) break;
+          if (lane == 0) {
             tc_fence_after();
 #pragma unroll
             for (int gg = 0; gg < SG; ++gg) {
@@ -468,26 +494,51 @@ __global__ void __launch_bounds__(kThreads, 1)
               }
             }
             umma_commit(&d_full[ds]);
-            if (++ds == DSL) {
-              ds = 0;
-              ph_d ^= 1u;
-            }
           }
-          if (!ok) break;
-          umma_commit(&a_empty[as]);
-          umma_commit(&empty[s]);
-          if (++as == ASL) {
-            as = 0;
-            ph_a ^= 1u;
-          }
-          if (++s == ST) {
-            s = 0;
-            ph ^= 1u;
-          }
+          __syncwarp();
+          if (++ds == DSL) ds = 0;
         }
+        if (!ok) break;
+        if (lane == 0) umma_commit(&a_empty[as]);
+        __syncwarp();
+        if (++as == ASL) as = 0;
+        if (++s == ST) s = 0;
       }
+    }
+    if (lane == 0) {
       umma_commit(drain);
       mbar_wait_plain(drain, 0, lim);
+    }
+  } else if (warp == kSchedWarp) {
+    // ---------------------------------------------------------------- MMA scheduler
+    // For each D slot: the stage's copies landed, its A slot is unpacked and the D slot is
+    // free; then one named-barrier step releases the MMA warp (false on timeout or abort).
+    int s = 0, as = 0, ds = 0;
+    uint32_t ph = 0, ph_a = 0, ph_d = 0;
+    bool ok = true;
+    for (int it = blockIdx.x; it < total && ok; it += gridDim.x) {
+      for (int kb = 0; kb < nkb && ok; ++kb) {
+        const int ng = min(KB, K - kb * KB) / G;
+        bool ready = __all_sync(0xffffffffu, mbar_wait(&full[s], ph, abort_flag, lim)) &&
+                     __all_sync(0xffffffffu, mbar_wait(&a_full[as], ph_a, abort_flag, lim));
+        for (int g0 = 0; g0 < ng; g0 += SG) {
+          ready = ready && __all_sync(0xffffffffu, mbar_wait(&d_empty[ds], ph_d ^ 1u, abort_flag, lim));
+          if (!(ok = bar_red_and(kMmaBarrier, 64, ready))) break;
+          if (++ds == DSL) {
+            ds = 0;
+            ph_d ^= 1u;
+          }
+        }
+        if (!ok) break;
+        if (++as == ASL) {
+          as = 0;
+          ph_a ^= 1u;
+        }
+        if (++s == ST) {
+          s = 0;
+          ph ^= 1u;
+        }
+      }
     }
   } else if (warp >= kEpiWarp0 && warp < kEpiWarp0 + 4) {
     // ---------------------------------------------------------------- promotion + epilogue

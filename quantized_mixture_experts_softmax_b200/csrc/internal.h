@@ -63,9 +63,14 @@ cudaError_t launch_w4a16_gemm(const W4GemmProblem& p, cudaStream_t s);
 // W4A16 grouped GEMM for decode-sized experts on the int8 tensor cores (gemm_w4i8.cu).
 // Activations as 16-bit fixed-point planes: per (row, 128-K block) scale s, X = rint(x/s)
 // = 256*hi + lo.  Plane matrix int8 [2*rows, K]: row 2r holds hi of row r, row 2r+1 its lo,
-// with K in the order (0,2,4,6,1,3,5,7) inside every 8-group.  Meta int32 [rows, ceil(K/256),
-// 12]: per 256-K stage the sums of X over its eight 32-K groups, then the scales of its two
-// 128-K blocks (fp32 bits), then two unused words.
+// with K in the order (0,2,4,6,1,3,5,7) inside every 8-group; |X| <= kFixMax.  Meta int32
+// [rows, ceil(K/256), 12]: per 256-K stage, for each of its eight 32-K groups kFixBias - 8 *
+// (sum of X over the group), then the scales of its two 128-K blocks (fp32 bits), then two
+// unused words.  kFixBias is the fp32 bit pattern of 1.5 * 2^23: adding an integer v with
+// |v| < 2^22 to it gives the bits of the float 1.5 * 2^23 + v, an exact int-to-float step.
+constexpr int kFixMax = 16383;
+constexpr int32_t kFixBias = 0x4B400000;
+constexpr float kFixBiasF = 12582912.0f;
 constexpr int kMetaWords = 12;
 __host__ __device__ inline int meta_words_per_row(int K) { return (K + 255) / 256 * kMetaWords; }
 struct W4I8Problem {

@@ -84,8 +84,8 @@ cudaError_t launch_permute_fp8(const uint8_t* x, const float* xs, const int32_t*
 }
 
 // 16-bit fixed-point planes of activation rows.  16 threads per (row, 128-K block), 8 K
-// elements each: s = max(amax, 1e-30) / 32639, X = rint(x / s) = 256*hi + lo with hi =
-// floor((X + 128) / 256) in [-127, 127] and lo in [-128, 127]; hi goes to plane row 2r, lo to
+// elements each: s = max(amax, 1e-30) / kFixMax, X = rint(x / s) = 256*hi + lo with hi =
+// floor((X + 128) / 256) in [-64, 64] and lo in [-128, 127]; hi goes to plane row 2r, lo to
 // 2r+1, bytes in the order (0,2,4,6,1,3,5,7) of each 8-group (the order in which a packed INT4
 // word unpacks); the sum of X over every 32-K group (for the MMA's offset correction) and the
 // block scales go to the row's meta words.
@@ -124,7 +124,7 @@ __global__ void __launch_bounds__(256) planes_kernel(const uint4* __restrict__ a
   }
 #pragma unroll
   for (int off = 8; off; off >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, off));  // 16 lanes
-  const float sc = fmaxf(amax, 1e-30f) * (1.0f / 32639.0f);
+  const float sc = fmaxf(amax, 1e-30f) * (1.0f / kFixMax);
   int X[8], sum = 0;
 #pragma unroll
   for (int j = 0; j < 8; ++j) {
@@ -148,7 +148,7 @@ __global__ void __launch_bounds__(256) planes_kernel(const uint4* __restrict__ a
   planes[o] = make_uint2(hb[0], hb[1]);
   planes[o + K / 8] = make_uint2(lb[0], lb[1]);
   int32_t* m = meta + (size_t)r * meta_words_per_row(K) + (blk >> 1) * kMetaWords;
-  if ((i & 3) == 0) m[(blk & 1) * 4 + (i >> 2)] = sum;
+  if ((i & 3) == 0) m[(blk & 1) * 4 + (i >> 2)] = kFixBias - 8 * sum;
   if (i == 0) m[8 + (blk & 1)] = __float_as_int(sc);
 }
 
