@@ -43,7 +43,6 @@ constexpr int G = 32;            // K per scale group = K per MMA
 constexpr int NG = KB / G;       // groups per stage
 constexpr int NT = kI8TileRows;  // token rows per tile (each gives a hi and a lo plane row)
 constexpr int DC = 2 * NT;       // D columns of one MMA (N)
-constexpr int SG = 4;            // groups per D slot
 constexpr int kThreads = 512;
 constexpr int kMmaWarp = 1;
 constexpr int kSchedWarp = 2;
@@ -56,6 +55,7 @@ static_assert(NT == 8, "the promotion code handles up to 8 tokens per tile");
 template <bool GATED>
 struct Cfg {
   static constexpr int NA = GATED ? 2 : 1;
+  static constexpr int SG = GATED ? 4 : 8;  // groups per D slot (SG * NA MMAs per handoff)
   static constexpr int W_TILE = BM * KB / 2;   // INT4 bytes
   static constexpr int B_ATOM = 2 * NT * 128;  // one 128-K atom of the 2*NT plane rows
   static constexpr int STAGE_B = NA * W_TILE;
@@ -193,11 +193,12 @@ struct Promo {
   float ag[NP], au[NP];
 };
 
-// Tokens [0, NP) of one D slot (groups g0 .. g0+SG-1 x NA matrices): loads their 2*NP columns
-// of every (group, matrix) in batches of at most 32 registers, one wait per batch.  swg/swu:
-// weight scales of this thread's rows per group; meta: the stage's meta words per token.
-template <int NA, int NP>
-__device__ __forceinline__ void promote_slot(uint32_t slot_addr, const int* meta, int g0,
+// Tokens [0, NP) of one D slot (groups g0 .. g0+SG-1 x NA matrices, the first `ngs` of them
+// present): loads their 2*NP columns of every (group, matrix) in batches of at most 32
+// registers, one wait per batch.  swg/swu: weight scales of this thread's rows per group;
+// meta: the stage's meta words per token.
+template <int NA, int SG, int NP>
+__device__ __forceinline__ void promote_slot(uint32_t slot_addr, const int* meta, int g0, int ngs,
                                              const float (&swg)[SG], const float (&swu)[SG], Promo<NP>& P) {
   constexpr int NC = 2 * NP, U = SG * NA;
   constexpr int PER = (32 / NC) < U ? (32 / NC) : U;
@@ -210,6 +211,7 @@ __device__ __forceinline__ void promote_slot(uint32_t slot_addr, const int* meta
 #pragma unroll
     for (int u = 0; u < PER; ++u) {
       const int unit = b0 + u, gg = unit / NA, mat = unit % NA;
+      if (SG > 4 && gg >= ngs) continue;  // group beyond K (a half stage; 4 divides every stage)
       const float sw = mat ? swu[gg] : swg[gg];
       // all NP columns are promoted: those of tokens >= nv hold finite values of other rows and
       // are never stored
@@ -241,7 +243,7 @@ __device__ __forceinline__ bool promote_item(const Params& p, const Item& I, int
                                              uint64_t* empty, int& ds, uint32_t& ph_d, uint64_t* d_full,
                                              uint64_t* d_empty, volatile int* abort_flag, Promo<NP>& P) {
   using C = Cfg<GATED>;
-  constexpr int NA = C::NA, DSL = C::DSLOTS, ST = C::ST;
+  constexpr int NA = C::NA, DSL = C::DSLOTS, ST = C::ST, SG = C::SG;
   const int K = p.K, nkb = ceil_div(K, KB);
   const uint64_t lim = p.wait_limit;
   for (int kb = 0; kb < nkb; ++kb) {
@@ -264,7 +266,7 @@ __device__ __forceinline__ bool promote_item(const Params& p, const Item& I, int
         swg[gg] = bf16_at(sgv, g0 + gg);
         swu[gg] = bf16_at(suv, g0 + gg);
       }
-      promote_slot<NA, NP>(lane_base + (uint32_t)(ds * C::D_SLOT), meta, g0, swg, swu, P);
+      promote_slot<NA, SG, NP>(lane_base + (uint32_t)(ds * C::D_SLOT), meta, g0, min(SG, ng - g0), swg, swu, P);
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&d_empty[ds]);
@@ -355,7 +357,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                      const __grid_constant__ CUtensorMap tm_m, const __grid_constant__ CUtensorMap tm_s,
                      const Params p) {
   using C = Cfg<GATED>;
-  constexpr int NA = C::NA, ST = C::ST, ASL = C::ASLOTS, DSL = C::DSLOTS;
+  constexpr int NA = C::NA, ST = C::ST, ASL = C::ASLOTS, DSL = C::DSLOTS, SG = C::SG;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + C::OFF_BAR);
@@ -486,6 +488,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
             for (int gg = 0; gg < SG; ++gg) {
               const int g = g0 + gg;
+              if (SG > 4 && g >= ng) break;  // a half stage (4 divides every stage)
               const uint64_t b = sw128_kmajor_desc(smem_u32(st + C::STAGE_B + (g >> 2) * C::B_ATOM)) + 2 * (g & 3);
 #pragma unroll
               for (int mat = 0; mat < NA; ++mat) {
