@@ -52,6 +52,32 @@ def load_peaks():
     return dict(hbm=6650.0, bf16=1590.0, bf16_sus=1400.0, src="fallback")
 
 
+# source file of each grouped GEMM: a measured traffic figure stands only while it is unchanged
+KERNEL_SOURCES = {"w4i8": "gemm_w4i8.cu", "w4a16": "gemm_w4a16.cu", "fp8": "gemm_fp8.cu"}
+
+
+def source_sha256(family: str) -> str:
+    import hashlib
+    path = os.path.join(ROOT, "quantized_mixture_experts_softmax_b200", "csrc", KERNEL_SOURCES[family])
+    return hashlib.sha256(open(path, "rb").read()).hexdigest()
+
+
+def load_traffic(workload: str, kernel: str, family: str):
+    """DRAM bytes per launch of `kernel` on `workload` from an ncu summary under profiles/ (a line
+    `traffic: workload=W kernel=K family=F bytes_per_launch=N source_sha256=H`), or None when there
+    is none or the kernel's source changed since the counters were taken."""
+    import glob
+    import re
+    sha = source_sha256(family)
+    for path in sorted(glob.glob(os.path.join(ROOT, "profiles", "*.md"))):
+        for line in open(path):
+            m = re.match(r"\s*traffic: workload=(\S+) kernel=(\S+) family=(\S+) bytes_per_launch=(\d+) "
+                         r"source_sha256=([0-9a-f]+)", line)
+            if m and m.group(1) == workload and m.group(2) == kernel and m.group(3) == family and m.group(5) == sha:
+                return int(m.group(4))
+    return None
+
+
 class ClockSampler:
     """nvidia-smi clock / throttle-reason samples while the timed region runs."""
 
@@ -323,6 +349,8 @@ def run_ours(args, world, rank):
     t_peak = peaks["bf16"] * (2.0 if kind == "fp8" else 1.0)
     t_peak_src = peaks["src"] + (" bf16 GEMM x 2 (nominal fp8:bf16)" if kind == "fp8" else " bf16 GEMM, burst")
     top = max(kern.items(), key=lambda kv: kv[1][0]) if kern else None
+    # which grouped GEMM runs: the int8-MMA kernel when no expert can get more than 64 rows
+    family = "fp8" if kind == "fp8" else ("w4i8" if T <= 64 else "w4a16")
     roof = None
     if top is not None:
         name, (ms_k, n_k) = top
@@ -336,22 +364,25 @@ def run_ours(args, world, rank):
         else:
             alg_bytes, alg_flops = None, None
         hbm_bound = alg_bytes is not None and (alg_flops / alg_bytes) < (t_peak * 1e3 / peaks["hbm"])
+        traffic = None if (args.tokens or args.experts) else load_traffic(args.workload, name, family)
         if alg_bytes and hbm_bound:
             ach = alg_bytes / per_launch_s / 1e9
             roof = dict(kernel=name, bound="hbm", achieved=round(ach, 1), peak=peaks["hbm"], unit="GB/s",
-                        frac=round(ach / peaks["hbm"], 4), traffic=None, peak_source=peaks["src"] + " (copy, burst)",
+                        frac=round(ach / peaks["hbm"], 4), traffic=traffic,
+                        peak_source=peaks["src"] + " (copy, burst)",
                         algorithmic_bytes_per_launch=int(alg_bytes), launch_ms=round(per_launch_s * 1e3, 4))
         elif alg_flops:
             ach = alg_flops / per_launch_s / 1e12
             roof = dict(kernel=name, bound="tensor", achieved=round(ach, 1), peak=t_peak, unit="TFLOP/s",
-                        frac=round(ach / t_peak, 4), traffic=None, peak_source=t_peak_src,
+                        frac=round(ach / t_peak, 4), traffic=traffic, peak_source=t_peak_src,
                         algorithmic_flops_per_launch=alg_flops, launch_ms=round(per_launch_s * 1e3, 4))
     launches = sum(n for (_, n) in kern.values())
     res = {
         "metric": METRIC, "value": round(ms_step * 1e3 / world, 2), "unit": "µs/layer",
         "n_gpus": world, "steps": steps, "warmup": warmup, "ms_per_step": round(ms_step, 4),
         "higher_is_better": False, "scaling": "weak", "vs_baseline": None,
-        "dtype": "e4m3 (fp32 acc)" if kind == "fp8" else "w4a16 (fp16 MMA, fp32 acc)",
+        "dtype": {"fp8": "e4m3 (fp32 acc)", "w4a16": "w4a16 (fp16 MMA, fp32 acc)",
+                  "w4i8": "w4a16 as int8 MMA (u8 weights x 16-bit fixed-point activations, s32) + fp32 promotion"}[family],
         "data": "synthetic (seeded counter-based generator; random-init quantized weights)",
         "config": {"workload": f"{args.workload} {'block-FP8' if kind == 'fp8' else 'W4A16'} MoE layer T={T} "
                                f"H={H} I={I} E={E} top-{k}",

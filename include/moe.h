@@ -113,10 +113,17 @@ moe_status_t moe_align_noalloc(const int32_t* topk_ids, int T, int k, int E, int
  *   w13_s  bf16  [E, 2I, H/32] one scale per 32 K elements per output row
  *   w2_q   int32 [E, H, I/8],  w2_s bf16 [E, H, I/32]   (down projection, same packing)
  *   out    bf16  [T, H] (RNE of the fp32 result), or fp32 [T, H] when out_fp32 != 0
- * Numerics: activations and dequantized weights are fed to the tensor cores in fp16, which
- * is exact for bf16 x inside the fp16 normal range and for |q*s| inside it (scales in
- * [2^-14/8... , 65504/8]); accumulation is fp32; h is rounded to fp16; the combine sums the
- * k slots in fp32 in slot order, so the result is deterministic run to run.
+ * Numerics, two paths chosen from T:
+ *   T <= 64: the INT4 values meet 16-bit fixed-point activations on the int8 tensor cores:
+ *     per (row, 128-K block) s = max(|x|max, 1e-30) / 16383 and X = rint(x / s); each 32-K
+ *     group's sum of q*X is exact in int32 and is scaled by (weight scale * s) and
+ *     accumulated in fp32; h is stored the same way (one scale per token per 128 rows of I).
+ *     The only rounding besides fp32 accumulation is X (at most s / 2 per element).
+ *   T > 64: activations and dequantized weights are fed to the tensor cores in fp16, which is
+ *     exact for bf16 x inside the fp16 normal range and for |q*s| inside it (scales in
+ *     [2^-14/8... , 65504/8]); accumulation is fp32; h is rounded to fp16.
+ * The combine sums the k slots in fp32 in slot order, so the result is deterministic run to
+ * run.
  * ws: moe_w4a16_workspace_size(T, H, I, E, k) bytes. */
 typedef struct {
   const void* x;
@@ -168,7 +175,9 @@ moe_status_t moe_blockfp8_forward(const moe_blockfp8_args* args, void* ws, size_
  *   expert_offsets int32 [E+1] (device), non-decreasing, offsets[0] >= 0, offsets[E] <= M;
  *                  rows outside every range are not written
  *   out            bf16 or fp32 (out_fp32 != 0) [M, N]
- * K and N multiples of 128.  ws: moe_w4a16_gemm_workspace_size(M, K, N, E) bytes. */
+ * K and N multiples of 128.  M <= 64 runs the int8 tensor-core path and M > 64 the fp16 path,
+ * with the numerics described at moe_w4a16_forward.
+ * ws: moe_w4a16_gemm_workspace_size(M, K, N, E) bytes. */
 size_t moe_w4a16_gemm_workspace_size(int M, int K, int N, int E);
 moe_status_t moe_w4a16_gemm(const void* a, int a_is_bf16, const int32_t* w_q, const void* w_s,
                             const int32_t* expert_offsets, int M, int K, int N, int E, void* out, int out_fp32,
