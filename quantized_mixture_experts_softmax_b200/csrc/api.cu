@@ -196,7 +196,6 @@ GemmWs carve_gemm(void* ws, int M, int K, int E) {
   w.bytes = c.off + 256;
   return w;
 }
-// token-tile height cap: thin variant (w4::kThinN rows) when no expert can exceed 64 rows
 struct F8Ws {
   int32_t *counts, *offsets, *sorted, *inv, *blockcnt, *tile_prefix, *chunk;
   uint8_t *x_perm, *h;
@@ -222,6 +221,7 @@ F8Ws carve_fp8_forward(void* ws, int T, int H, int I, int E, int k) {
   w.bytes = c.off + 256;
   return w;
 }
+// token-tile height cap of the W4A16 GEMM that runs
 int pick_nmax(int max_rows_per_expert) { return use_i8(max_rows_per_expert) ? kI8TileRows : 256; }
 
 bool shape_ok(int T, int H, int I, int E, int k) {

@@ -147,6 +147,24 @@ __device__ __forceinline__ void tmem_relinquish() {
 __device__ __forceinline__ void tmem_dealloc(uint32_t taddr, uint32_t ncols) {
   asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols) : "memory");
 }
+// Named barrier `id` over `n` threads that also returns the AND of every thread's `in`.
+// A thread that has tcgen05 MMAs in flight stalls on its next mbarrier wait (or shared-memory
+// access) until they drain, idling the tensor core; the GEMMs therefore keep such waits in a
+// scheduler warp that releases the MMA warp through this barrier (no timeout of its own: both
+// sides take the same number of steps, and a failed wait travels as `in` = false).
+__device__ __forceinline__ bool bar_red_and(int id, int n, bool in) {
+  uint32_t r;
+  asm volatile(
+      "{\n\t.reg .pred pi, po;\n\t"
+      "setp.ne.u32 pi, %1, 0;\n\t"
+      "bar.red.and.pred po, %2, %3, pi;\n\t"
+      "selp.u32 %0, 1, 0, po;\n\t}\n"
+      : "=r"(r)
+      : "r"((uint32_t)in), "r"(id), "r"(n)
+      : "memory");
+  return r != 0;
+}
+
 __device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
 __device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
 

@@ -123,20 +123,6 @@ __device__ __forceinline__ Item decode_item(int it, const int* __restrict__ spre
   return I;
 }
 
-// Named barrier `id` over `n` threads that also returns the AND of every thread's `in`.
-__device__ __forceinline__ bool bar_red_and(int id, int n, bool in) {
-  uint32_t r;
-  asm volatile(
-      "{\n\t.reg .pred pi, po;\n\t"
-      "setp.ne.u32 pi, %1, 0;\n\t"
-      "bar.red.and.pred po, %2, %3, pi;\n\t"
-      "selp.u32 %0, 1, 0, po;\n\t}\n"
-      : "=r"(r)
-      : "r"((uint32_t)in), "r"(id), "r"(n)
-      : "memory");
-  return r != 0;
-}
-
 // D[tmem] = A[tmem] * B[smem]^T, u8 x s8 -> s32, D overwritten (no accumulation)
 __device__ __forceinline__ void umma_i8_ts(uint32_t d, uint32_t a, uint64_t b, uint32_t idesc) {
   asm volatile(
