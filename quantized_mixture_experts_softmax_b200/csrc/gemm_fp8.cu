@@ -13,7 +13,9 @@
 //               tiles for the gate/up GEMM) and the token tile's activations, one stage per
 //               128-K block;
 //   warp 1      TMEM allocator and single-thread MMA issuer: four K=32 MMAs per matrix per block
-//               into a double-buffered partial-product tile;
+//               into a double-buffered partial-product tile; it never waits on an mbarrier
+//               (see bar_red_and) and is released block by block by
+//   warp 2      the MMA scheduler, which waits for the stage's copies and a free partial tile;
 //   warps 4-7   promotion and epilogue: each thread owns one weight row and keeps its tokens'
 //               fp32 accumulators in registers.  The gate/up GEMM ends with h = SiLU(gate) * up,
 //               requantized per (token, 128-column group) - the tile's 128 rows are exactly one
@@ -30,6 +32,9 @@ constexpr int BM = 128;   // weight rows per tile (MMA M)
 constexpr int KB = 128;   // K per stage = one scale block
 constexpr int NMAX = 32;  // token rows per tile
 constexpr int kThreads = 256;
+constexpr int kMmaWarp = 1;
+constexpr int kSchedWarp = 2;
+constexpr int kMmaBarrier = 1;  // named barrier of the MMA and scheduler warps (0 is __syncthreads)
 constexpr int kEpiWarp0 = 4;
 
 template <bool GATED>
@@ -141,7 +146,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     prefetch_tmap(&tm_w);
     prefetch_tmap(&tm_b);
   }
-  if (warp == 1) {
+  if (warp == kMmaWarp) {
     tmem_alloc(tmem_slot, C::TMEM_COLS);
     tmem_relinquish();
   }
@@ -181,18 +186,17 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       for (int i = max(0, issued - ST); i < issued; ++i) mbar_wait_plain(&full[i % ST], (i / ST) & 1, lim);
     }
-  } else if (warp == 1) {
+  } else if (warp == kMmaWarp) {
     // ---------------------------------------------------------------- MMA issuer
-    if (lane == 0) {
-      int s = 0, pb = 0;
-      uint32_t ph = 0, ph_p = 0;
-      bool ok = true;
-      for (int it = blockIdx.x; it < total && ok; it += gridDim.x) {
-        const Item I = decode_item(it, sprefix, p);
-        const uint32_t idesc = make_idesc(BM, I.nmma, 0, 0);  // e4m3 x e4m3 -> fp32
-        for (int kb = 0; kb < nkb; ++kb) {
-          if (!(ok = mbar_wait(&full[s], ph, abort_flag, lim))) break;
-          if (!(ok = mbar_wait(&p_empty[pb], ph_p ^ 1u, abort_flag, lim))) break;
+    // Released block by block by the scheduler warp; identical loop bounds on both sides.
+    int s = 0, pb = 0;
+    bool ok = true;
+    for (int it = blockIdx.x; it < total && ok; it += gridDim.x) {
+      const Item I = decode_item(it, sprefix, p);
+      const uint32_t idesc = make_idesc(BM, I.nmma, 0, 0);  // e4m3 x e4m3 -> fp32
+      for (int kb = 0; kb < nkb; ++kb) {
+        if (!(ok = bar_red_and(kMmaBarrier, 64, true))) break;
+        if (lane == 0) {
           tc_fence_after();
           const uint8_t* st = smem + s * C::STAGE;
           const uint64_t a0 = sw128_kmajor_desc(smem_u32(st));
@@ -206,18 +210,35 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
           umma_commit(&p_full[pb]);
           umma_commit(&empty[s]);
-          if (++s == ST) {
-            s = 0;
-            ph ^= 1u;
-          }
-          if (++pb == 2) {
-            pb = 0;
-            ph_p ^= 1u;
-          }
         }
+        __syncwarp();
+        if (++s == ST) s = 0;
+        if (++pb == 2) pb = 0;
       }
+    }
+    if (lane == 0) {
       umma_commit(drain);
       mbar_wait_plain(drain, 0, lim);
+    }
+  } else if (warp == kSchedWarp) {
+    // ---------------------------------------------------------------- MMA scheduler
+    int s = 0, pb = 0;
+    uint32_t ph = 0, ph_p = 0;
+    bool ok = true;
+    for (int it = blockIdx.x; it < total && ok; it += gridDim.x) {
+      for (int kb = 0; kb < nkb; ++kb) {
+        const bool ready = __all_sync(0xffffffffu, mbar_wait(&full[s], ph, abort_flag, lim)) &&
+                           __all_sync(0xffffffffu, mbar_wait(&p_empty[pb], ph_p ^ 1u, abort_flag, lim));
+        if (!(ok = bar_red_and(kMmaBarrier, 64, ready))) break;
+        if (++s == ST) {
+          s = 0;
+          ph ^= 1u;
+        }
+        if (++pb == 2) {
+          pb = 0;
+          ph_p ^= 1u;
+        }
+      }
     }
   } else if (warp >= kEpiWarp0) {
     // ---------------------------------------------------------------- promotion + epilogue
@@ -234,10 +255,19 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int c = 0; c < NMAX; ++c) ag[c] = au[c] = 0.f;
       const float* wsg = p.w_scale + ((size_t)I.e * (p.rows_per_expert / BM) + I.m) * GK;
       const float* wsu = GATED ? wsg + (size_t)(p.I / BM) * GK : wsg;
+      // per-token activation scales (lane c holds token c's) and weight-block scales, one block
+      // ahead so that their load latency hides behind the current block
+      auto xs_at = [&](int kb) {
+        return (lane < I.nvalid && kb < nkb) ? __ldg(p.x_scale + (size_t)kb * p.act_rows + I.r0 + lane) : 0.f;
+      };
+      float xs_n = xs_at(0), sg_n = __ldg(wsg), su_n = GATED ? __ldg(wsu) : 0.f;
       for (int kb = 0; kb < nkb; ++kb) {
-        // this block's per-token activation scales: lane c holds token c's
-        const float xs_l = (lane < I.nvalid) ? __ldg(p.x_scale + (size_t)kb * p.act_rows + I.r0 + lane) : 0.f;
-        const float sg = __ldg(wsg + kb), su = GATED ? __ldg(wsu + kb) : 0.f;
+        const float xs_l = xs_n, sg = sg_n, su = su_n;
+        xs_n = xs_at(kb + 1);
+        if (kb + 1 < nkb) {
+          sg_n = __ldg(wsg + kb + 1);
+          if (GATED) su_n = __ldg(wsu + kb + 1);
+        }
         ok = __all_sync(0xffffffffu, mbar_wait(&p_full[pb], ph_p, abort_flag, lim));
         if (!ok) break;
         tc_fence_after();
@@ -307,7 +337,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   tc_fence_before();
   __syncthreads();
-  if (warp == 1) {
+  if (warp == kMmaWarp) {
     tc_fence_after();
     tmem_dealloc(tmem_base, C::TMEM_COLS);
   }
