@@ -53,8 +53,8 @@ template <bool GATED>
 struct Cfg {
   static constexpr int NA = GATED ? 2 : 1;
   // ring depths: activation tiles, dequantized A tiles
-  static constexpr int BST = GATED ? 4 : 5;
-  static constexpr int ABUF = 2;
+  static constexpr int BST = GATED ? 3 : 5;
+  static constexpr int ABUF = GATED ? 3 : 2;
   static constexpr int NSUB = KB / KS;               // 64-K steps per weight stage
   static constexpr int A_TILE = BM * KS * 2;         // dequantized fp16 operand
   static constexpr int B_ATOM = NMAX * KS * 2;       // activation tile of one 64-K step

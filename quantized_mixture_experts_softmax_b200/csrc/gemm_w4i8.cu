@@ -465,22 +465,27 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (int it = blockIdx.x; it < total && ok; it += gridDim.x) {
       for (int kb = 0; kb < nkb && ok; ++kb) {
         const int ng = min(KB, K - kb * KB) / G;
-        const uint8_t* st = smem + s * C::STAGE;
+        // descriptors and addresses from per-stage bases plus constants, so that the issue loop
+        // between MMAs is a few instructions
+        const uint64_t b_base = sw128_kmajor_desc(smem_u32(smem + s * C::STAGE + C::STAGE_B));
         const uint32_t a_slot = tmem_base + (uint32_t)(C::A_COL0 + as * C::A_SLOT);
-        for (int g0 = 0; g0 < ng; g0 += SG) {
+#pragma unroll
+        for (int g0 = 0; g0 < NG; g0 += SG) {
+          if (g0 >= ng) break;
           if (!(ok = bar_red_and(kMmaBarrier, 64, true))) break;
           if (lane == 0) {
             tc_fence_after();
+            const uint32_t d_slot = tmem_base + (uint32_t)(ds * C::D_SLOT);
 #pragma unroll
             for (int gg = 0; gg < SG; ++gg) {
               const int g = g0 + gg;
               if (SG > 4 && g >= ng) break;  // a half stage (4 divides every stage)
-              const uint64_t b = sw128_kmajor_desc(smem_u32(st + C::STAGE_B + (g >> 2) * C::B_ATOM)) + 2 * (g & 3);
+              // B atom g/4 (B_ATOM bytes = B_ATOM/16 descriptor units), 32-byte K step within it
+              const uint64_t b = b_base + (uint64_t)((g >> 2) * (C::B_ATOM >> 4) + 2 * (g & 3));
 #pragma unroll
-              for (int mat = 0; mat < NA; ++mat) {
-                const uint32_t d = tmem_base + (uint32_t)(ds * C::D_SLOT + (gg * NA + mat) * DC);
-                umma_i8_ts(d, a_slot + (uint32_t)(mat * NG * 8 + g * 8), b, idesc);
-              }
+              for (int mat = 0; mat < NA; ++mat)
+                umma_i8_ts(d_slot + (uint32_t)((gg * NA + mat) * DC), a_slot + (uint32_t)(mat * NG * 8 + g * 8), b,
+                           idesc);
             }
             umma_commit(&d_full[ds]);
           }
