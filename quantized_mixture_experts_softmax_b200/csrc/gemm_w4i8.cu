@@ -23,14 +23,17 @@
 //
 // The MMA-issuing thread never waits on an mbarrier: a wait (or any shared-memory access) by
 // the thread that has MMAs in flight stalls until they drain, idling the tensor core for
-// hundreds of cycles per wait.  A scheduler warp does the waits and releases the MMA warp
-// through a named barrier with an AND reduction (which also carries a timeout or abort).
+// hundreds of cycles per wait.  A scheduler warp does the waits and releases an MMA warp
+// through a named barrier with an AND reduction (which also carries a timeout or abort).  Even
+// that hand-off waits for the releasing warp's own MMAs to drain, so two MMA warps take the D
+// slots in turn: while one is held at its barrier, the other's MMAs keep the tensor core busy.
 //
 // Work list, swap (weights in the MMA's M slot) and persistence as in the fp16 GEMM.  Warps
 // (512 threads): 0 producer (TMA of the INT4 words, weight scales, activation planes and meta
 // words of the token tile per 256-K stage; cp.async for scale rows not 16-byte aligned),
-// 1 TMEM allocator + MMA issuer, 2 MMA scheduler, 4-7 promotion and epilogue, 8-15 unpacking
-// INT4 words into u8 rows of tensor memory (the MMA's A operand).
+// 1 TMEM allocator + MMA issuer of even D slots, 3 MMA issuer of odd D slots, 2 MMA scheduler,
+// 4-7 promotion and epilogue, 8-15 unpacking INT4 words into u8 rows of tensor memory (the
+// MMA's A operand).
 #include "common.cuh"
 #include "internal.h"
 
@@ -44,9 +47,11 @@ constexpr int NG = KB / G;       // groups per stage
 constexpr int NT = kI8TileRows;  // token rows per tile (each gives a hi and a lo plane row)
 constexpr int DC = 2 * NT;       // D columns of one MMA (N)
 constexpr int kThreads = 512;
-constexpr int kMmaWarp = 1;
+constexpr int kMmaWarp = 1;     // even D slots (and the TMEM allocator)
+constexpr int kMmaWarpOdd = 3;  // odd D slots
 constexpr int kSchedWarp = 2;
-constexpr int kMmaBarrier = 1;  // named barrier of the MMA and scheduler warps (0 is __syncthreads)
+constexpr int kMmaBarrier = 1;  // named barriers 1 (even slots) and 2 (odd slots) of an MMA warp
+                                // and the scheduler warp (0 is __syncthreads)
 constexpr int kEpiWarp0 = 4;
 constexpr int kUnpackWarp0 = 8;
 constexpr int kNumUnpack = 8;
@@ -372,13 +377,13 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     for (int i = 0; i < ASL; ++i) {
       mbar_init(&a_full[i], kNumUnpack);
-      mbar_init(&a_empty[i], 1);
+      mbar_init(&a_empty[i], 2);  // a commit from each MMA warp
     }
     for (int i = 0; i < DSL; ++i) {
       mbar_init(&d_full[i], 1);
       mbar_init(&d_empty[i], 4);
     }
-    mbar_init(drain, 1);
+    mbar_init(drain, 2);
     mbar_init(epi_bar, 4);
     *abort_flag = 0;
     fence_mbar_init();
@@ -453,14 +458,16 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     if (lane == 0)
       for (int i = max(0, issued - ST); i < issued; ++i) mbar_wait_plain(&full[i % ST], (i / ST) & 1, lim);
-  } else if (warp == kMmaWarp) {
-    // ---------------------------------------------------------------- MMA issuer
-    // Released slot by slot by the scheduler warp; identical loop bounds on both sides, so
-    // both take the same number of named-barrier steps.
+  } else if (warp == kMmaWarp || warp == kMmaWarpOdd) {
+    // ---------------------------------------------------------------- MMA issuers
+    // Warp 1 takes the even D slots, warp 3 the odd ones (a running slot count q), each released
+    // by the scheduler warp on its own named barrier; every loop bound is the scheduler's, so
+    // both sides take the same barrier steps.
     // u8 A x s8 B -> s32, M = 128, N = DC (NT tokens x (hi, lo))
     const uint32_t idesc = (2u << 4) | (0u << 7) | (1u << 10) | ((uint32_t)(DC >> 3) << 17) |
                            ((uint32_t)(BM >> 4) << 24);
-    int s = 0, as = 0, ds = 0;
+    const int mine = warp == kMmaWarpOdd ? 1 : 0;
+    int s = 0, as = 0, ds = 0, q = 0;
     bool ok = true;
     for (int it = blockIdx.x; it < total && ok; it += gridDim.x) {
       for (int kb = 0; kb < nkb && ok; ++kb) {
@@ -472,27 +479,31 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
         for (int g0 = 0; g0 < NG; g0 += SG) {
           if (g0 >= ng) break;
-          if (!(ok = bar_red_and(kMmaBarrier, 64, true))) break;
-          if (lane == 0) {
-            tc_fence_after();
-            const uint32_t d_slot = tmem_base + (uint32_t)(ds * C::D_SLOT);
+          if ((q & 1) == mine) {
+            if (!(ok = bar_red_and(kMmaBarrier + mine, 64, true))) break;
+            if (lane == 0) {
+              tc_fence_after();
+              const uint32_t d_slot = tmem_base + (uint32_t)(ds * C::D_SLOT);
 #pragma unroll
-            for (int gg = 0; gg < SG; ++gg) {
-              const int g = g0 + gg;
-              if (SG > 4 && g >= ng) break;  // a half stage (4 divides every stage)
-              // B atom g/4 (B_ATOM bytes = B_ATOM/16 descriptor units), 32-byte K step within it
-              const uint64_t b = b_base + (uint64_t)((g >> 2) * (C::B_ATOM >> 4) + 2 * (g & 3));
+              for (int gg = 0; gg < SG; ++gg) {
+                const int g = g0 + gg;
+                if (SG > 4 && g >= ng) break;  // a half stage (4 divides every stage)
+                // B atom g/4 (B_ATOM bytes = B_ATOM/16 descriptor units), 32-byte K step within it
+                const uint64_t b = b_base + (uint64_t)((g >> 2) * (C::B_ATOM >> 4) + 2 * (g & 3));
 #pragma unroll
-              for (int mat = 0; mat < NA; ++mat)
-                umma_i8_ts(d_slot + (uint32_t)((gg * NA + mat) * DC), a_slot + (uint32_t)(mat * NG * 8 + g * 8), b,
-                           idesc);
+                for (int mat = 0; mat < NA; ++mat)
+                  umma_i8_ts(d_slot + (uint32_t)((gg * NA + mat) * DC), a_slot + (uint32_t)(mat * NG * 8 + g * 8),
+                             b, idesc);
+              }
+              umma_commit(&d_full[ds]);
             }
-            umma_commit(&d_full[ds]);
+            __syncwarp();
           }
-          __syncwarp();
+          ++q;
           if (++ds == DSL) ds = 0;
         }
         if (!ok) break;
+        // each MMA warp's commit: the A slot is free once both warps' MMAs of the stage are done
         if (lane == 0) umma_commit(&a_empty[as]);
         __syncwarp();
         if (++as == ASL) as = 0;
@@ -506,10 +517,15 @@ __global__ void __launch_bounds__(kThreads, 1)
   } else if (warp == kSchedWarp) {
     // ---------------------------------------------------------------- MMA scheduler
     // For each D slot: the stage's copies landed, its A slot is unpacked and the D slot is
-    // free; then one named-barrier step releases the MMA warp (false on timeout or abort).
-    int s = 0, as = 0, ds = 0;
+    // free; then one named-barrier step releases the slot's MMA warp (false on timeout or
+    // abort, after which the other MMA warp, held for the next slot, is released with false).
+    int s = 0, as = 0, ds = 0, q = 0;
     uint32_t ph = 0, ph_a = 0, ph_d = 0;
     bool ok = true;
+    int slots_per_item = 0;
+    for (int kb = 0; kb < nkb; ++kb) slots_per_item += ceil_div(min(KB, K - kb * KB) / G, SG);
+    const int my_items = blockIdx.x < total ? (total - blockIdx.x + gridDim.x - 1) / gridDim.x : 0;
+    const int nq = my_items * slots_per_item;
     for (int it = blockIdx.x; it < total && ok; it += gridDim.x) {
       for (int kb = 0; kb < nkb && ok; ++kb) {
         const int ng = min(KB, K - kb * KB) / G;
@@ -517,7 +533,11 @@ __global__ void __launch_bounds__(kThreads, 1)
                      __all_sync(0xffffffffu, mbar_wait(&a_full[as], ph_a, abort_flag, lim));
         for (int g0 = 0; g0 < ng; g0 += SG) {
           ready = ready && __all_sync(0xffffffffu, mbar_wait(&d_empty[ds], ph_d ^ 1u, abort_flag, lim));
-          if (!(ok = bar_red_and(kMmaBarrier, 64, ready))) break;
+          if (!(ok = bar_red_and(kMmaBarrier + (q & 1), 64, ready))) {
+            if (q + 1 < nq) bar_red_and(kMmaBarrier + ((q + 1) & 1), 64, false);
+            break;
+          }
+          ++q;
           if (++ds == DSL) {
             ds = 0;
             ph_d ^= 1u;
