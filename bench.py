@@ -145,11 +145,13 @@ def dist_init():
 
 
 def max_over_ranks(v: float, world: int) -> float:
+    """The slowest rank's time (every rank gets it); NCCL reduces a device tensor, gloo a host one."""
     if world == 1:
         return v
     import torch
     import torch.distributed as dist
-    t = torch.tensor([v], dtype=torch.float64, device="cuda")
+    dev = "cuda" if dist.get_backend() == "nccl" else "cpu"
+    t = torch.tensor([v], dtype=torch.float64, device=dev)
     dist.all_reduce(t, op=dist.ReduceOp.MAX)
     return float(t.item())
 
