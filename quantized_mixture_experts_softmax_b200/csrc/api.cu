@@ -355,17 +355,19 @@ moe_status_t moe_blockfp8_forward(const moe_blockfp8_args* a, void* ws, size_t w
   if (moe_status_t st = check_device()) return st;
   const F8Ws w = carve_fp8_forward(ws, T, H, I, E, k);
   const int P = T * k;
-  const int nmax = 32;  // the FP8 GEMM's token tile
+  // token tile of the FP8 GEMM: 64 rows once experts can get that many tokens (halves the
+  // weight re-reads and doubles the tokens per MMA), else 32 (a deeper copy pipeline)
+  const int nmax = T > 512 ? 64 : 32;
   cudaError_t e = launch_align(a->topk_ids, T, k, E, 1, w.counts, w.offsets, w.sorted, w.inv, w.blockcnt, nmax,
                                w.tile_prefix, w.chunk, stream);
   if (e == cudaSuccess) e = launch_permute_fp8(a->x, a->xs, w.inv, T, k, H, w.x_perm, w.xs_t, P, stream);
   const TileSched sched{w.offsets, w.counts, w.tile_prefix, w.chunk};
   if (e == cudaSuccess) {
-    F8GemmProblem g{a->w13, a->w13_s, w.x_perm, w.xs_t, P, H, E, 2 * I, true, I, sched, w.h, I, w.hs_t};
+    F8GemmProblem g{a->w13, a->w13_s, w.x_perm, w.xs_t, P, H, E, 2 * I, true, I, sched, w.h, I, w.hs_t, nmax};
     e = launch_fp8_gemm(g, stream);
   }
   if (e == cudaSuccess) {
-    F8GemmProblem g{a->w2, a->w2_s, w.h, w.hs_t, P, I, E, H, false, 0, sched, w.y, H, nullptr};
+    F8GemmProblem g{a->w2, a->w2_s, w.h, w.hs_t, P, I, E, H, false, 0, sched, w.y, H, nullptr, nmax};
     e = launch_fp8_gemm(g, stream);
   }
   if (e == cudaSuccess) e = launch_combine(w.y, w.inv, a->topk_w, T, k, H, a->out, a->out_fp32, stream);

@@ -8,7 +8,7 @@
 //     acc[row][tok] += P_kb[row][tok] * (w_scale[tile][kb] * x_scale[tok][kb]).
 //
 // One persistent CTA per SM over the same (expert, 128-row weight tile, token tile) work list as
-// the W4A16 GEMM, weights swapped into the MMA's M slot.  Warp roles (256 threads):
+// the W4A16 GEMM, weights swapped into the MMA's M slot.  Warp roles (352 threads):
 //   warp 0      TMA producer: e4m3 weight tiles (128 rows x 128 K, 128-byte swizzle; gate and up
 //               tiles for the gate/up GEMM) and the token tile's activations, one stage per
 //               128-K block;
@@ -16,8 +16,9 @@
 //               into a double-buffered partial-product tile; it never waits on an mbarrier
 //               (see bar_red_and) and is released block by block by
 //   warp 2      the MMA scheduler, which waits for the stage's copies and a free partial tile;
-//   warps 4-7   promotion and epilogue: each thread owns one weight row and keeps its tokens'
-//               fp32 accumulators in registers.  The gate/up GEMM ends with h = SiLU(gate) * up,
+//   warps 3-10  promotion and epilogue, two per TMEM lane quarter: each thread owns one weight
+//               row and keeps the fp32 accumulators of one half of the tile's tokens (32 of up
+//               to 64) in registers.  The gate/up GEMM ends with h = SiLU(gate) * up,
 //               requantized per (token, 128-column group) - the tile's 128 rows are exactly one
 //               group - to e4m3 with s = max(amax, 1e-10) / 448; the down GEMM stores fp32.
 #include <cuda_fp8.h>
@@ -30,26 +31,30 @@ namespace f8 {
 
 constexpr int BM = 128;   // weight rows per tile (MMA M)
 constexpr int KB = 128;   // K per stage = one scale block
-constexpr int NMAX = 32;  // token rows per tile
-constexpr int kThreads = 256;
+constexpr int NH = 32;          // tokens per promotion thread (one 32-token part of the tile)
 constexpr int kMmaWarp = 1;
 constexpr int kSchedWarp = 2;
 constexpr int kMmaBarrier = 1;  // named barrier of the MMA and scheduler warps (0 is __syncthreads)
-constexpr int kEpiWarp0 = 4;
+constexpr int kEpiWarp0 = 3;    // warps 3..: promotion; lane quarter warp % 4, token part (warp - 3) / 4
 
-template <bool GATED>
+// NMAX = token rows per tile (32 or 64): 4 promotion warps per 32 tokens
+template <bool GATED, int NMAX>
 struct Cfg {
+  static_assert(NMAX % NH == 0 && NMAX <= 64, "32 or 64 token rows per tile");
+  static constexpr int kNumEpi = 4 * (NMAX / NH);
+  static constexpr int kThreads = (kEpiWarp0 + kNumEpi) * 32;
   static constexpr int NA = GATED ? 2 : 1;
   static constexpr int W_TILE = BM * KB;    // e4m3 bytes
   static constexpr int B_TILE = NMAX * KB;  // activation bytes
   static constexpr int STAGE = NA * W_TILE + B_TILE;
-  static constexpr int ST = GATED ? 6 : 10;
+  static constexpr int ST = NMAX == 32 ? (GATED ? 6 : 10) : (GATED ? 5 : 9);
   static constexpr int P_COLS = NA * NMAX;  // one partial-product tile: [matrix][NMAX] columns
-  static constexpr int TMEM_COLS = 2 * P_COLS <= 32 ? 32 : (2 * P_COLS <= 64 ? 64 : 128);
+  static constexpr int TMEM_COLS = 2 * P_COLS <= 32 ? 32 : (2 * P_COLS <= 64 ? 64 : (2 * P_COLS <= 128 ? 128 : 256));
+  static_assert(2 * P_COLS <= TMEM_COLS, "two partial-product tiles fit the allocation");
   static constexpr int OFF_BAR = ST * STAGE;
   static constexpr int NUM_BARS = 2 * ST + 4 + 2;
   static constexpr int OFF_MISC = OFF_BAR + NUM_BARS * 8;
-  static constexpr int OFF_RED = OFF_MISC + 16;              // [4 warps][NMAX] amax partials
+  static constexpr int OFF_RED = OFF_MISC + 16;              // [4 lane quarters][NMAX] amax partials
   static constexpr int OFF_PREFIX = OFF_RED + 4 * NMAX * 4;
   static_assert(STAGE % 1024 == 0, "swizzled tiles need 1024-byte alignment");
   static constexpr size_t smem_bytes(int E) { return (size_t)OFF_PREFIX + 4 * (size_t)(E + 1) + 1024; }
@@ -96,7 +101,7 @@ __device__ __forceinline__ Item decode_item(int it, const int* __restrict__ spre
   return I;
 }
 
-// Bounded barrier among the 4 epilogue warps (an mbarrier of count 4, alternating phases).
+// Bounded barrier among the 8 epilogue warps (an mbarrier of count 8, alternating phases).
 __device__ __forceinline__ bool epi_sync(uint64_t* bar, uint32_t& phase, volatile int* abort, uint64_t lim) {
   __syncwarp();
   if ((threadIdx.x & 31) == 0) mbar_arrive(bar);
@@ -105,12 +110,12 @@ __device__ __forceinline__ bool epi_sync(uint64_t* bar, uint32_t& phase, volatil
   return ok;
 }
 
-template <bool GATED>
-__global__ void __launch_bounds__(kThreads, 1)
+template <bool GATED, int NMAX>
+__global__ void __launch_bounds__(Cfg<GATED, NMAX>::kThreads, 1)
     fp8_gemm_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CUtensorMap tm_b,
                     const Params p) {
-  using C = Cfg<GATED>;
-  constexpr int NA = C::NA, ST = C::ST;
+  using C = Cfg<GATED, NMAX>;
+  constexpr int NA = C::NA, ST = C::ST, kNumEpi = C::kNumEpi;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + C::OFF_BAR);
@@ -135,10 +140,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     for (int i = 0; i < 2; ++i) {
       mbar_init(&p_full[i], 1);
-      mbar_init(&p_empty[i], 4);
+      mbar_init(&p_empty[i], kNumEpi);
     }
     mbar_init(drain, 1);
-    mbar_init(epi_bar, 4);
+    mbar_init(epi_bar, kNumEpi);
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -242,7 +247,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   } else if (warp >= kEpiWarp0) {
     // ---------------------------------------------------------------- promotion + epilogue
-    const int ew = warp - kEpiWarp0;  // == warp % 4: TMEM lanes 32*ew..32*ew+31
+    const int ew = warp & 3;                    // TMEM lanes 32*ew..32*ew+31 (the warp's quarter)
+    const int tok0 = ((warp - kEpiWarp0) >> 2) * NH;  // this warp's half of the tile's tokens
     const int mrow = ew * 32 + lane;
     const int GK = p.K / KB;
     int pb = 0;
@@ -250,15 +256,16 @@ __global__ void __launch_bounds__(kThreads, 1)
     bool ok = true;
     for (int it = blockIdx.x; it < total && ok; it += gridDim.x) {
       const Item I = decode_item(it, sprefix, p);
-      float ag[NMAX], au[NMAX];
+      const int nv = I.nvalid - tok0;  // tokens of this half (may be <= 0)
+      float ag[NH], au[NH];
 #pragma unroll
-      for (int c = 0; c < NMAX; ++c) ag[c] = au[c] = 0.f;
+      for (int c = 0; c < NH; ++c) ag[c] = au[c] = 0.f;
       const float* wsg = p.w_scale + ((size_t)I.e * (p.rows_per_expert / BM) + I.m) * GK;
       const float* wsu = GATED ? wsg + (size_t)(p.I / BM) * GK : wsg;
-      // per-token activation scales (lane c holds token c's) and weight-block scales, one block
-      // ahead so that their load latency hides behind the current block
+      // per-token activation scales (lane c holds token tok0+c's) and weight-block scales, one
+      // block ahead so that their load latency hides behind the current block
       auto xs_at = [&](int kb) {
-        return (lane < I.nvalid && kb < nkb) ? __ldg(p.x_scale + (size_t)kb * p.act_rows + I.r0 + lane) : 0.f;
+        return (lane < nv && kb < nkb) ? __ldg(p.x_scale + (size_t)kb * p.act_rows + I.r0 + tok0 + lane) : 0.f;
       };
       float xs_n = xs_at(0), sg_n = __ldg(wsg), su_n = GATED ? __ldg(wsu) : 0.f;
       for (int kb = 0; kb < nkb; ++kb) {
@@ -271,11 +278,11 @@ __global__ void __launch_bounds__(kThreads, 1)
         ok = __all_sync(0xffffffffu, mbar_wait(&p_full[pb], ph_p, abort_flag, lim));
         if (!ok) break;
         tc_fence_after();
-        const uint32_t tb = tmem_base + ((uint32_t)(ew * 32) << 16) + (uint32_t)(pb * C::P_COLS);
+        const uint32_t tb = tmem_base + ((uint32_t)(ew * 32) << 16) + (uint32_t)(pb * C::P_COLS + tok0);
         uint32_t pg[16], pu[16];
 #pragma unroll
-        for (int c0 = 0; c0 < NMAX; c0 += 16) {
-          if (c0 < I.nmma) {
+        for (int c0 = 0; c0 < NH; c0 += 16) {
+          if (tok0 + c0 < I.nmma) {
             tmem_ld16(tb + c0, pg);
             if (GATED) tmem_ld16(tb + NMAX + c0, pu);
             tmem_ld_wait();
@@ -297,31 +304,29 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       if (!ok) break;
       if constexpr (GATED) {
-        // h = SiLU(gate) * up; requantize each token's 128 values of this tile (one 1x128 group)
-        float amax[NMAX];
+        // h = SiLU(gate) * up; requantize each token's 128 values of this tile (one 1x128 group):
+        // the token's amax over the tile's rows comes from the four warps of its half
 #pragma unroll
-        for (int c = 0; c < NMAX; ++c) {
+        for (int c = 0; c < NH; ++c) {
           const float h = ag[c] / (1.0f + __expf(-ag[c])) * au[c];
           ag[c] = h;
           float m = fabsf(h);
 #pragma unroll
           for (int off = 16; off; off >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, off));
-          amax[c] = m;
+          if (lane == 0) red[ew * NMAX + tok0 + c] = m;
         }
-        if (lane == 0)
-#pragma unroll
-          for (int c = 0; c < NMAX; ++c) red[ew * NMAX + c] = amax[c];
         if (!(ok = epi_sync(epi_bar, ph_e, abort_flag, lim))) break;
         uint8_t* hq = reinterpret_cast<uint8_t*>(p.out);
         const int j = I.m * BM + mrow;
 #pragma unroll
-        for (int c = 0; c < NMAX; ++c) {
-          if (c < I.nvalid) {
-            const float a = fmaxf(fmaxf(red[c], red[NMAX + c]), fmaxf(red[2 * NMAX + c], red[3 * NMAX + c]));
+        for (int c = 0; c < NH; ++c) {
+          if (c < nv) {
+            const int t = tok0 + c;
+            const float a = fmaxf(fmaxf(red[t], red[NMAX + t]), fmaxf(red[2 * NMAX + t], red[3 * NMAX + t]));
             const float sc = __fdiv_rn(fmaxf(a, 1e-10f), 448.0f);
             const __nv_fp8_e4m3 q(__fdiv_rn(ag[c], sc));  // round to nearest even, saturating
-            hq[(size_t)(I.r0 + c) * p.out_ld + j] = *reinterpret_cast<const uint8_t*>(&q);
-            if (mrow == 0) p.h_scale[(size_t)I.m * p.act_rows + I.r0 + c] = sc;
+            hq[(size_t)(I.r0 + t) * p.out_ld + j] = *reinterpret_cast<const uint8_t*>(&q);
+            if (mrow == 0) p.h_scale[(size_t)I.m * p.act_rows + I.r0 + t] = sc;
           }
         }
         if (!(ok = epi_sync(epi_bar, ph_e, abort_flag, lim))) break;  // red[] is reused by the next item
@@ -329,8 +334,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         float* y = reinterpret_cast<float*>(p.out);
         const int n = I.m * BM + mrow;
 #pragma unroll
-        for (int c = 0; c < NMAX; ++c)
-          if (c < I.nvalid) y[(size_t)(I.r0 + c) * p.out_ld + n] = ag[c];
+        for (int c = 0; c < NH; ++c)
+          if (c < nv) y[(size_t)(I.r0 + tok0 + c) * p.out_ld + n] = ag[c];
       }
     }
   }
@@ -343,9 +348,9 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
 }
 
-template <bool GATED>
+template <bool GATED, int NMAX>
 cudaError_t launch_t(const F8GemmProblem& pr, cudaStream_t s) {
-  using C = Cfg<GATED>;
+  using C = Cfg<GATED, NMAX>;
   CUtensorMap tm_w, tm_b;
   const uint64_t wrows = (uint64_t)pr.E * pr.rows_per_expert;
   if (encode_tmap_2d(&tm_w, pr.w, CU_TENSOR_MAP_DATA_TYPE_UINT8, pr.K, wrows, (uint64_t)pr.K, KB, BM,
@@ -369,12 +374,12 @@ cudaError_t launch_t(const F8GemmProblem& pr, cudaStream_t s) {
   p.h_scale = pr.h_scale;
   p.wait_limit = wait_limit_ns();
   const size_t smem = C::smem_bytes(pr.E);
-  auto kern = fp8_gemm_kernel<GATED>;
+  auto kern = fp8_gemm_kernel<GATED, NMAX>;
   cudaError_t err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (err != cudaSuccess) return err;
   const char* name = GATED ? "fp8_gemm_gate_up" : "fp8_gemm_down";
   timing_before(name, s);
-  kern<<<sm_count(), kThreads, smem, s>>>(tm_w, tm_b, p);
+  kern<<<sm_count(), C::kThreads, smem, s>>>(tm_w, tm_b, p);
   timing_after(name, s);
   return cudaGetLastError();
 }
@@ -382,7 +387,9 @@ cudaError_t launch_t(const F8GemmProblem& pr, cudaStream_t s) {
 }  // namespace f8
 
 cudaError_t launch_fp8_gemm(const F8GemmProblem& p, cudaStream_t s) {
-  return p.gated ? f8::launch_t<true>(p, s) : f8::launch_t<false>(p, s);
+  if (p.nmax == 32) return p.gated ? f8::launch_t<true, 32>(p, s) : f8::launch_t<false, 32>(p, s);
+  if (p.nmax == 64) return p.gated ? f8::launch_t<true, 64>(p, s) : f8::launch_t<false, 64>(p, s);
+  return cudaErrorInvalidValue;
 }
 
 }  // namespace moe

@@ -109,6 +109,7 @@ struct F8GemmProblem {
   void* out;
   int out_ld;
   float* h_scale;          // gated: [I/128, act_rows]
+  int nmax;                // token rows per tile: 32 or 64 (the cap the schedule was built with)
 };
 cudaError_t launch_fp8_gemm(const F8GemmProblem& p, cudaStream_t s);
 cudaError_t launch_permute_fp8(const uint8_t* x, const float* xs, const int32_t* inv_pos, int T, int k, int H,
