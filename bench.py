@@ -40,6 +40,11 @@ WORKLOADS = {
 for _t in (1, 16, 64, 512, 4096):  # block-FP8 layer, 256 experts
     WORKLOADS[f"fp8_t{_t}"] = dict(kind="fp8", T=_t, zipf=0.0, steps=200 if _t <= 512 else 60, warmup=10)
 FP8_MODEL = dict(H=7168, I=2048, E=256, k=8)
+# the single-expert grouped-GEMM sweep: [M,7168]x[7168,512] and [M,256]x[256,7168]
+for (_k, _n) in ((7168, 512), (256, 7168)):
+    for _m in (1, 64, 512, 4096, 32768):
+        WORKLOADS[f"gemm_m{_m}_k{_k}_n{_n}"] = dict(kind="gemm", M=_m, K=_k, N=_n, steps=50, warmup=5)
+GEMM_METRIC = "grouped W4A16 GEMM µs (one expert, no activation) and % roofline"
 W13_BYTES_PER_EXPERT = 2 * 2048 * 7168 // 2 + 2 * 2048 * (7168 // 32) * 2   # INT4 words + bf16 scales
 W2_BYTES_PER_EXPERT = 7168 * 2048 // 2 + 7168 * (2048 // 32) * 2
 
@@ -224,6 +229,78 @@ def make_inputs(seed: int, T: int, zipf: float, kind: str = "w4a16"):
     x = synth.x_bf16(seed, T, MODEL["H"])
     lg = synth.logits(seed, T, MODEL["E"], zipf_s=zipf)
     return x, lg
+
+
+def run_gemm(args, world, rank):
+    """The single-expert W4A16 GEMM sweep through moe_w4a16_gemm.  Small operands fit in L2, so
+    a 512 MB buffer is read between steps (a read leaves no dirty lines to write back during the
+    next step) and the step time is the sum of the library's own kernels (CUDA events around
+    each launch), the flush excluded."""
+    import torch
+    import quantized_mixture_experts_softmax_b200 as moe
+    import synth
+
+    wl = WORKLOADS[args.workload]
+    M, K, N = wl["M"], wl["K"], wl["N"]
+    steps = args.steps if args.steps is not None else wl["steps"]
+    warmup = max(3, args.warmup if args.warmup is not None else wl["warmup"])
+    a, w_q, w_s = synth.gemm_operands(0, M, K, N)
+    d_a = torch.from_numpy(a).cuda().view(torch.bfloat16)
+    d_q = torch.from_numpy(w_q).cuda()
+    d_s = torch.from_numpy(w_s).cuda().view(torch.bfloat16)
+    off = torch.tensor([0, M], dtype=torch.int32, device="cuda")
+    out = torch.empty(M, N, dtype=torch.bfloat16, device="cuda")
+    ws = torch.empty(max(moe.moe_w4a16_gemm_workspace_size(M, K, N, 1), 1), dtype=torch.uint8, device="cuda")
+    flush = torch.ones(128 << 20, dtype=torch.float32, device="cuda")  # 512 MB
+
+    def step():
+        moe.moe_w4a16_gemm(d_a, d_q, d_s, off, out=out, workspace=ws)
+
+    for _ in range(warmup):
+        flush.sum()
+        step()
+    torch.cuda.synchronize()
+    assert moe.moe_get_device_status() == 0
+    with ClockSampler(torch.cuda.current_device()) as clk:
+        moe.moe_timing_enable(True)
+        moe.moe_timing_read()
+        barrier(world)
+        for _ in range(steps):
+            flush.sum()
+            step()
+        torch.cuda.synchronize()
+        barrier(world)
+        moe.moe_timing_enable(False)
+    kern = moe.moe_timing_read()
+    assert moe.moe_get_device_status() == 0
+    ms_step = max_over_ranks(sum(v[0] for v in kern.values()) / steps, world)
+    launches = sum(n for (_, n) in kern.values())
+    peaks = load_peaks()
+    bytes_ = K * N // 2 + (K // 32) * N * 2 + M * K * 2 + M * N * 2
+    flops = 2.0 * M * N * K
+    s_ = ms_step / 1e3
+    hbm_bound = flops / bytes_ < peaks["bf16"] * 1e3 / peaks["hbm"]
+    if hbm_bound:
+        ach = bytes_ / s_ / 1e9
+        roof = dict(kernel="all", bound="hbm", achieved=round(ach, 1), peak=peaks["hbm"], unit="GB/s",
+                    frac=round(ach / peaks["hbm"], 4), traffic=None, peak_source=peaks["src"] + " (copy, burst)",
+                    algorithmic_bytes_per_launch=int(bytes_))
+    else:
+        ach = flops / s_ / 1e12
+        roof = dict(kernel="all", bound="tensor", achieved=round(ach, 1), peak=peaks["bf16"], unit="TFLOP/s",
+                    frac=round(ach / peaks["bf16"], 4), traffic=None, peak_source=peaks["src"] + " bf16 GEMM, burst",
+                    algorithmic_flops_per_launch=flops)
+    return {
+        "metric": GEMM_METRIC, "value": round(ms_step * 1e3, 2), "unit": "µs/GEMM", "n_gpus": world,
+        "steps": steps, "warmup": warmup, "ms_per_step": round(ms_step, 4), "higher_is_better": False,
+        "scaling": "weak", "vs_baseline": None,
+        "dtype": "w4a16 as int8 MMA + fp32 promotion" if M <= 64 else "w4a16 (fp16 MMA, fp32 acc)",
+        "data": "synthetic (seeded counter-based generator)",
+        "config": {"workload": f"single-expert W4A16 GEMM [{M},{K}]x[{K},{N}]", "M": M, "K": K, "N": N,
+                   "l2": "512 MB buffer read between steps; time = the library's kernels only"},
+        "kernels_ms_per_step": {k_: round(v[0] / steps, 4) for k_, v in kern.items()},
+        "gpu_launches": launches, "roofline": roof, "clocks": clk.summary(),
+    }
 
 
 def run_ours(args, world, rank):
@@ -468,8 +545,46 @@ def oracle_sample_time(x_h, lg_h, T, kind="w4a16", budget_s=15.0):
     return us_layer, f"{n} of {T} tokens (all {k} experts each), extrapolated linearly to {T}", cores, 0.0
 
 
+def gemm_oracle_time(M, K, N, budget_s=8.0):
+    """CPU oracle of the single-expert GEMM on a bounded row sample -> (us per GEMM, sample, cores)."""
+    import oracle
+    import synth
+    a, w_q, w_s = synth.gemm_operands(0, M, K, N)
+    cores = oracle.nthreads()
+
+    def run(n):
+        t0 = time.time()
+        oracle.w4a16_gemm(a[:n], True, w_q, w_s, np.array([0, n], np.int32))
+        return time.time() - t0
+
+    n_probe = max(1, min(M, cores))
+    per_row = run(n_probe) / n_probe
+    n = int(min(M, max(n_probe, budget_s / max(per_row, 1e-9))))
+    el = run(n)
+    return el / n * M * 1e6, f"{n} of {M} rows, extrapolated linearly to {M}", cores
+
+
 def run_reference(args, world, rank):
     wl = WORKLOADS[args.workload]
+    if wl["kind"] == "gemm":
+        M, K, N = wl["M"], wl["K"], wl["N"]
+        steps = args.steps if args.steps is not None else 3
+        warmup = args.warmup if args.warmup is not None else 1
+        vals, sample, cores = [], None, None
+        for i in range(warmup + steps):
+            us, sample, cores = gemm_oracle_time(M, K, N)
+            if i >= warmup:
+                vals.append(us)
+        v = statistics.median(vals)
+        return {
+            "metric": GEMM_METRIC, "value": round(v, 1), "unit": "µs/GEMM", "n_gpus": world, "steps": steps,
+            "warmup": warmup, "ms_per_step": round(v / 1e3, 3), "higher_is_better": False, "scaling": "weak",
+            "vs_baseline": None, "dtype": "f64 (oracle)", "data": "synthetic",
+            "config": {"workload": f"single-expert W4A16 GEMM [{M},{K}]x[{K},{N}]"}, "impl": "reference",
+            "cpu_baseline": {"value": round(v, 1), "unit": "µs/GEMM", "cores": cores, "kind": "oracle",
+                             "sample": sample},
+            "e2e": {"value": round(v, 1), "unit": "µs/GEMM", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+        }
     T = wl["T"]
     steps = args.steps if args.steps is not None else 3
     warmup = args.warmup if args.warmup is not None else 1
@@ -521,6 +636,11 @@ def main():
         return
 
     world, rank, _ = dist_init()
+    if WORKLOADS[args.workload]["kind"] == "gemm":
+        res = run_gemm(args, world, rank)
+        if rank == 0:
+            print(json.dumps(res), flush=True)
+        return
     res, (x_h, lg_h, T, kind) = run_ours(args, world, rank)
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         us, sample, cores, _ = oracle_sample_time(x_h, lg_h, T, kind)

@@ -177,22 +177,40 @@ FwdWs carve_w4_forward(void* ws, int T, int H, int I, int E, int k) {
   w.bytes = c.off + 256;
   return w;
 }
+// K splits of the single grouped GEMM on the int8 path: when even the fewest work items the
+// shape can have (all M rows in one expert) leave most of the 148 SMs of a B200 idle, each item's
+// K range is split so that items x splits ~ 148 (at most one 256-K stage per split, at most 32);
+// a shape-only rule, so the workspace size needs no device.
+int gemm_splits(int M, int K, int N) {
+  if (!use_i8(M)) return 1;
+  const int nkb = (K + 255) / 256;
+  const int items = (N / 128) * ((M + kI8TileRows - 1) / kI8TileRows);
+  int s = 148 / (items > 0 ? items : 1);
+  if (s > nkb) s = nkb;
+  if (s > 32) s = 32;
+  return s < 1 ? 1 : s;
+}
+
 struct GemmWs {
   int32_t *row_count, *tile_prefix, *chunk;
-  __half* a;  // fp16 path
-  Planes aq;  // int8 path
+  __half* a;    // fp16 path
+  Planes aq;    // int8 path
+  float* part;  // int8 path with K splits: [splits, M, N] fp32 partial sums
   size_t bytes;
 };
-GemmWs carve_gemm(void* ws, int M, int K, int E) {
+GemmWs carve_gemm(void* ws, int M, int K, int N, int E) {
   Carver c(ws);
   GemmWs w{};
   w.row_count = c.take<int32_t>(E);
   w.tile_prefix = c.take<int32_t>(E + 1);
   w.chunk = c.take<int32_t>(E);
-  if (use_i8(M))
+  if (use_i8(M)) {
     w.aq = take_planes(c, M, K);
-  else
+    const int sp = gemm_splits(M, K, N);
+    if (sp > 1) w.part = c.take<float>((size_t)sp * M * N);
+  } else {
     w.a = c.take<__half>((size_t)M * K);
+  }
   w.bytes = c.off + 256;
   return w;
 }
@@ -376,7 +394,7 @@ moe_status_t moe_blockfp8_forward(const moe_blockfp8_args* a, void* ws, size_t w
 
 size_t moe_w4a16_gemm_workspace_size(int M, int K, int N, int E) {
   if (M < 1 || K < 128 || N < 128 || K % 128 || N % 128 || E < 1 || E > 1024) return 0;
-  return carve_gemm(nullptr, M, K, E).bytes;
+  return carve_gemm(nullptr, M, K, N, E).bytes;
 }
 
 moe_status_t moe_w4a16_gemm(const void* a, int a_is_bf16, const int32_t* w_q, const void* w_s,
@@ -389,18 +407,20 @@ moe_status_t moe_w4a16_gemm(const void* a, int a_is_bf16, const int32_t* w_q, co
     return MOE_ERR_INVALID_ARG;
   if (ws_bytes < moe_w4a16_gemm_workspace_size(M, K, N, E)) return MOE_ERR_WORKSPACE;
   if (moe_status_t st = check_device()) return st;
-  const GemmWs w = carve_gemm(ws, M, K, E);
+  const GemmWs w = carve_gemm(ws, M, K, N, E);
   const int nmax = pick_nmax(M);
   cudaError_t e = launch_sched_from_offsets(expert_offsets, E, M, nmax, w.row_count, w.tile_prefix, w.chunk, stream);
   const TileSched sched{expert_offsets, w.row_count, w.tile_prefix, w.chunk};
   if (use_i8(M)) {
     if (e == cudaSuccess)
       e = launch_planes(static_cast<const uint16_t*>(a), a_is_bf16, nullptr, M, 1, K, w.aq.x, w.aq.meta, stream);
+    const int sp = gemm_splits(M, K, N);
     if (e == cudaSuccess) {
       W4I8Problem g{w_q, static_cast<const uint16_t*>(w_s), w.aq.x, w.aq.meta, M, K, E, N, false, 0, sched,
-                    out_fp32 ? OUT_F32 : OUT_BF16, out, nullptr, N};
+                    out_fp32 ? OUT_F32 : OUT_BF16, out, nullptr, N, sp, w.part};
       e = launch_w4i8_gemm(g, stream);
     }
+    if (e == cudaSuccess && sp > 1) e = launch_reduce_splits(w.part, sp, M, N, expert_offsets, E, out, out_fp32, stream);
     return e == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
   }
   if (e == cudaSuccess) e = launch_convert_rows(static_cast<const uint16_t*>(a), a_is_bf16, M, K, w.a, stream);

@@ -98,6 +98,9 @@ struct Params {
   void* out;             // planes int8 [2*rows, out_ld]; else fp32/bf16 [rows, out_ld]
   int32_t* out_meta;     // planes: meta words of h
   int out_ld;
+  int splits;            // K splits per (expert, weight tile, token tile); > 1 only for plain outputs
+  float* part;           // splits > 1: fp32 partial sums [splits, act_rows, out_ld]
+  int act_rows;
   uint64_t wait_limit;
 };
 
@@ -105,8 +108,21 @@ struct Item {
   int e, m, r0, nvalid;
 };
 
-__device__ __forceinline__ Item decode_item(int it, const int* __restrict__ sprefix, const Params& p) {
+// K stages [kb0, kb1) of work item `it` (its K split: it % splits of the nkb stages, balanced)
+__device__ __forceinline__ void kb_range(int it, int nkb, int splits, int& kb0, int& kb1) {
+  if (splits == 1) {
+    kb0 = 0;
+    kb1 = nkb;
+    return;
+  }
+  const int sp = it % splits;
+  kb0 = sp * nkb / splits;
+  kb1 = (sp + 1) * nkb / splits;
+}
+
+__device__ __forceinline__ Item decode_item(int it_, const int* __restrict__ sprefix, const Params& p) {
   Item I;
+  const int it = p.splits == 1 ? it_ : it_ / p.splits;  // the (expert, weight tile, token tile)
   const int tile = it / p.m_tiles;
   int lo = 0, hi = p.E;  // sprefix[lo] <= tile < sprefix[hi]
   while (hi - lo > 1) {
@@ -232,12 +248,13 @@ template <bool GATED, int NP>
 __device__ __forceinline__ bool promote_item(const Params& p, const Item& I, int mrow, int lane, uint32_t lane_base,
                                              const uint8_t* smem, int& s, uint32_t& ph, uint64_t* full,
                                              uint64_t* empty, int& ds, uint32_t& ph_d, uint64_t* d_full,
-                                             uint64_t* d_empty, volatile int* abort_flag, Promo<NP>& P) {
+                                             uint64_t* d_empty, volatile int* abort_flag, int kb0, int kb1,
+                                             Promo<NP>& P) {
   using C = Cfg<GATED>;
   constexpr int NA = C::NA, DSL = C::DSLOTS, ST = C::ST, SG = C::SG;
-  const int K = p.K, nkb = ceil_div(K, KB);
+  const int K = p.K;
   const uint64_t lim = p.wait_limit;
-  for (int kb = 0; kb < nkb; ++kb) {
+  for (int kb = kb0; kb < kb1; ++kb) {
     const int ng = min(KB, K - kb * KB) / G;
     // the stage's meta words and weight scales (their copies completed long before; this wait
     // also orders the reads after them)
@@ -279,7 +296,7 @@ __device__ __forceinline__ bool promote_item(const Params& p, const Item& I, int
 // One work item of the promotion warps: the K loop, then the epilogue (GATED: h = SiLU(gate)
 // * up as fixed-point planes with one scale per (token, tile); else fp32 or bf16 rows).
 template <bool GATED, int NP>
-__device__ __forceinline__ bool epi_item(const Params& p, const Item& I, int ew, int lane, uint32_t lane_base,
+__device__ __forceinline__ bool epi_item(const Params& p, const Item& I, int it, int ew, int lane, uint32_t lane_base,
                                          const uint8_t* smem, int& s, uint32_t& ph, uint64_t* full, uint64_t* empty,
                                          int& ds, uint32_t& ph_d, uint64_t* d_full, uint64_t* d_empty,
                                          float* red, uint64_t* epi_bar, uint32_t& ph_e, volatile int* abort_flag) {
@@ -287,8 +304,10 @@ __device__ __forceinline__ bool epi_item(const Params& p, const Item& I, int ew,
   Promo<NP> P;
 #pragma unroll
   for (int c = 0; c < NP; ++c) P.ag[c] = P.au[c] = 0.f;
+  int kb0, kb1;
+  kb_range(it, ceil_div(p.K, KB), p.splits, kb0, kb1);
   if (!promote_item<GATED, NP>(p, I, mrow, lane, lane_base, smem, s, ph, full, empty, ds, ph_d, d_full, d_empty,
-                               abort_flag, P))
+                               abort_flag, kb0, kb1, P))
     return false;
   if constexpr (GATED) {
 #pragma unroll
@@ -327,7 +346,12 @@ __device__ __forceinline__ bool epi_item(const Params& p, const Item& I, int ew,
     return epi_sync(epi_bar, ph_e, abort_flag, p.wait_limit);  // red[] is reused by the next item
   } else {
     const int n = I.m * BM + mrow;
-    if (p.out_kind == OUT_F32) {
+    if (p.splits > 1) {  // this split's partial sum, reduced in split order by another kernel
+      float* y = p.part + (size_t)(it % p.splits) * p.act_rows * p.out_ld;
+#pragma unroll
+      for (int c = 0; c < NP; ++c)
+        if (c < nv) y[(size_t)(I.r0 + c) * p.out_ld + n] = P.ag[c];
+    } else if (p.out_kind == OUT_F32) {
       float* y = reinterpret_cast<float*>(p.out);
 #pragma unroll
       for (int c = 0; c < NP; ++c)
@@ -402,7 +426,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
-  const int total = p.m_tiles * sprefix[p.E];
+  const int total = p.m_tiles * sprefix[p.E] * p.splits;
   const int K = p.K;
   const int nkb = ceil_div(K, KB);
 
@@ -418,7 +442,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       const Item I = decode_item(it, sprefix, p);
       const int row_g = I.e * p.rows_per_expert + I.m * BM;
       const int row_u = row_g + p.I;
-      for (int kb = 0; kb < nkb; ++kb) {
+      int kb0, kb1;
+      kb_range(it, nkb, p.splits, kb0, kb1);
+      for (int kb = kb0; kb < kb1; ++kb) {
         if (!(ok = __all_sync(0xffffffffu, mbar_wait(&empty[s], ph ^ 1u, abort_flag, lim)))) break;
         uint8_t* st = smem + s * C::STAGE;
         const int natom = min(KB, K - kb * KB) / 128;  // 2, or 1 for a half stage
@@ -470,7 +496,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     int s = 0, as = 0, ds = 0, q = 0;
     bool ok = true;
     for (int it = blockIdx.x; it < total && ok; it += gridDim.x) {
-      for (int kb = 0; kb < nkb && ok; ++kb) {
+      int kb0, kb1;
+      kb_range(it, nkb, p.splits, kb0, kb1);
+      for (int kb = kb0; kb < kb1 && ok; ++kb) {
         const int ng = min(KB, K - kb * KB) / G;
         // descriptors and addresses from per-stage bases plus constants, so that the issue loop
         // between MMAs is a few instructions
@@ -522,19 +550,20 @@ __global__ void __launch_bounds__(kThreads, 1)
     int s = 0, as = 0, ds = 0, q = 0;
     uint32_t ph = 0, ph_a = 0, ph_d = 0;
     bool ok = true;
-    int slots_per_item = 0;
-    for (int kb = 0; kb < nkb; ++kb) slots_per_item += ceil_div(min(KB, K - kb * KB) / G, SG);
-    const int my_items = blockIdx.x < total ? (total - blockIdx.x + gridDim.x - 1) / gridDim.x : 0;
-    const int nq = my_items * slots_per_item;
+
     for (int it = blockIdx.x; it < total && ok; it += gridDim.x) {
-      for (int kb = 0; kb < nkb && ok; ++kb) {
+      int kb0, kb1;
+      kb_range(it, nkb, p.splits, kb0, kb1);
+      for (int kb = kb0; kb < kb1 && ok; ++kb) {
         const int ng = min(KB, K - kb * KB) / G;
         bool ready = __all_sync(0xffffffffu, mbar_wait(&full[s], ph, abort_flag, lim)) &&
                      __all_sync(0xffffffffu, mbar_wait(&a_full[as], ph_a, abort_flag, lim));
         for (int g0 = 0; g0 < ng; g0 += SG) {
           ready = ready && __all_sync(0xffffffffu, mbar_wait(&d_empty[ds], ph_d ^ 1u, abort_flag, lim));
           if (!(ok = bar_red_and(kMmaBarrier + (q & 1), 64, ready))) {
-            if (q + 1 < nq) bar_red_and(kMmaBarrier + ((q + 1) & 1), 64, false);
+            // the other MMA warp is held for the next slot, if there is one
+            if (g0 + SG < ng || kb + 1 < kb1 || it + (int)gridDim.x < total)
+              bar_red_and(kMmaBarrier + ((q + 1) & 1), 64, false);
             break;
           }
           ++q;
@@ -565,7 +594,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       const Item I = decode_item(it, sprefix, p);
       const int nv = I.nvalid;
 #define MOE_EPI_ITEM(NP_)                                                                                           \
-  epi_item<GATED, NP_>(p, I, ew, lane, lane_base, smem, s, ph, full, empty, ds, ph_d, d_full, d_empty, red, epi_bar, \
+  epi_item<GATED, NP_>(p, I, it, ew, lane, lane_base, smem, s, ph, full, empty, ds, ph_d, d_full, d_empty, red, epi_bar, \
                        ph_e, abort_flag)
       if (nv <= 1)
         ok = MOE_EPI_ITEM(1);
@@ -592,7 +621,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     uint32_t ph = 0, ph_a = 0;
     bool ok = true;
     for (int it = blockIdx.x; it < total && ok; it += gridDim.x) {
-      for (int kb = 0; kb < nkb && ok; ++kb) {
+      int kb0, kb1;
+      kb_range(it, nkb, p.splits, kb0, kb1);
+      for (int kb = kb0; kb < kb1 && ok; ++kb) {
         const int ng = min(KB, K - kb * KB) / G;
         ok = __all_sync(0xffffffffu, mbar_wait(&full[s], ph, abort_flag, lim));
         if (!ok) break;
@@ -694,6 +725,9 @@ cudaError_t launch_t(const W4I8Problem& pr, cudaStream_t s) {
   p.out = pr.out;
   p.out_meta = pr.out_meta;
   p.out_ld = pr.out_ld;
+  p.splits = pr.splits > 1 && !GATED ? pr.splits : 1;
+  p.part = pr.part;
+  p.act_rows = pr.act_rows;
   p.wait_limit = wait_limit_ns();
   const size_t smem = C::smem_bytes(pr.E);
   auto kern = w4i8_gemm_kernel<GATED>;

@@ -163,6 +163,46 @@ cudaError_t launch_planes(const uint16_t* a, int a_is_bf16, const int32_t* inv_p
   return cudaGetLastError();
 }
 
+// Split-K reduction: out[r][n] = sum_s part[s][r][n] in split order (deterministic), for the
+// rows the expert ranges cover; one thread per 4 outputs.
+__global__ void __launch_bounds__(256) reduce_splits_kernel(const float4* __restrict__ part, int splits, int rows,
+                                                            int N, const int32_t* __restrict__ offsets, int E,
+                                                            void* __restrict__ out, int out_fp32) {
+  const int r0 = __ldg(offsets), r1 = __ldg(offsets + E);
+  const size_t n4 = (size_t)N / 4, plane = (size_t)rows * n4;
+  for (size_t i = (size_t)blockIdx.x * blockDim.x + threadIdx.x; i < plane; i += (size_t)gridDim.x * blockDim.x) {
+    const int r = (int)(i / n4);
+    if (r < r0 || r >= r1) continue;
+    float4 acc = __ldg(part + i);
+    for (int sp = 1; sp < splits; ++sp) {
+      const float4 v = __ldg(part + (size_t)sp * plane + i);
+      acc.x += v.x;
+      acc.y += v.y;
+      acc.z += v.z;
+      acc.w += v.w;
+    }
+    if (out_fp32) {
+      reinterpret_cast<float4*>(out)[i] = acc;
+    } else {
+      __nv_bfloat162* o = reinterpret_cast<__nv_bfloat162*>(out) + 2 * i;
+      o[0] = __floats2bfloat162_rn(acc.x, acc.y);
+      o[1] = __floats2bfloat162_rn(acc.z, acc.w);
+    }
+  }
+}
+
+cudaError_t launch_reduce_splits(const float* part, int splits, int rows, int N, const int32_t* offsets, int E,
+                                 void* out, int out_fp32, cudaStream_t s) {
+  const size_t n = (size_t)rows * (N / 4);
+  const size_t want = (n + 255) / 256;
+  const unsigned blocks = (unsigned)(want < 148 * 8 ? want : 148 * 8);
+  timing_before("reduce_splits", s);
+  reduce_splits_kernel<<<blocks, 256, 0, s>>>(reinterpret_cast<const float4*>(part), splits, rows, N, offsets, E, out,
+                                              out_fp32);
+  timing_after("reduce_splits", s);
+  return cudaGetLastError();
+}
+
 __global__ void __launch_bounds__(256) convert_rows_kernel(const uint4* __restrict__ a, int a_is_bf16, size_t n8,
                                                            uint4* __restrict__ out) {
   for (size_t i = blockIdx.x * (size_t)blockDim.x + threadIdx.x; i < n8; i += (size_t)gridDim.x * blockDim.x) {

@@ -75,3 +75,33 @@ def test_ragged_experts(offsets):
     covered[off[0]:off[-1]] = True
     check_tol(got[covered], ref[covered], what="ragged")
     assert np.all(got[~covered] == 12345.0)
+
+
+@pytest.mark.parametrize("K", [384, 1024])
+@pytest.mark.parametrize("offsets", [[4, 4, 20, 21, 50, 56], [0, 60, 60, 60, 60, 60]])
+def test_ragged_experts_decode_sized_split_k(K, offsets):
+    """M <= 64 runs the int8 path; with few work items its K range is split (fp32 partial sums
+    reduced in split order), here into 2 (K=384, a half 256-K stage last) or 4 (K=1024) parts.
+    Rows outside every expert range keep their previous contents (12288, exact in bf16)."""
+    M, N, E = 60, 256, 5
+    a = synth.x_bf16(5, M, K)
+    W = synth.w4a16_weights(5, K, N // 2, range(E))
+    w_q, w_s = W["w13_q"], W["w13_s"]
+    off = np.array(offsets, np.int32)
+    ref = oracle.w4a16_gemm(a, True, w_q, w_s, off)
+    covered = np.zeros(M, bool)
+    covered[off[0]:off[-1]] = True
+    outs = {}
+    for fp32 in (True, False):
+        init = torch.full((M, N), 12288.0, device="cuda", dtype=torch.float32 if fp32 else torch.bfloat16)
+        outs[fp32] = moe.moe_w4a16_gemm(dev(a, torch.bfloat16), dev(w_q), dev(w_s, torch.bfloat16), dev(off),
+                                        out=init, out_fp32=fp32)
+    torch.cuda.synchronize()
+    assert moe.moe_get_device_status() == 0
+    g32 = outs[True].double().cpu().numpy()
+    g16 = outs[False].float().cpu().numpy()
+    check_tol(g32[covered], ref[covered], what=f"split-K K={K} fp32")
+    check_tol(g16[covered], ref[covered], bf16_out=True, what=f"split-K K={K} bf16")
+    assert np.all(g32[~covered] == 12288.0) and np.all(g16[~covered] == 12288.0)
+    assert torch.equal(outs[True].to(torch.bfloat16)[covered.tolist()].view(torch.int16),
+                       outs[False][covered.tolist()].view(torch.int16))
