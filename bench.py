@@ -1,20 +1,22 @@
 """Benchmark of the routed W4A16 MoE layer (router + align + permute + gate/up GEMM with SiLU*up
 + down GEMM + weighted combine) on B200, through the library's C ABI.
 
-    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload decode|prefill]
-                    [--impl ours|reference]
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl ours|reference]
 
-One JSON line on stdout (rank 0).  Workloads (seeded synthetic inputs, see DESIGN.md):
-  decode   T=64 tokens, hidden 7168, intermediate 2048, 384 experts, top-8, N(0,1) logits
-  prefill  T=8192 tokens, same model, logits skewed by a Zipf(1.1) per-expert bias
-The model's 384 experts (9.5 GB of INT4 weights + bf16 scales) stay resident in HBM; each step
-streams the active experts' weights (about 7 GB for decode), far more than the 126 MB L2, so
-no L2 flush is needed between steps.
+One JSON line on stdout (rank 0).  Workloads (seeded synthetic inputs):
+  decode            T=64 tokens, hidden 7168, intermediate 2048, 384 experts, top-8, N(0,1) logits
+  prefill           T=8192 tokens, same model, logits skewed by a Zipf(1.1) per-expert bias
+  fp8_t{1,16,64,512,4096}   the block-FP8 layer, 256 experts, top-8
+  gemm_m{M}_k{K}_n{N}       the single-expert grouped GEMM sweep (no activation)
+The layer models' experts (9.5 GB of INT4 weights + bf16 scales for W4A16) stay resident in HBM;
+each step streams the active experts' weights (about 7 GB for decode), far more than the
+126 MB L2, so no L2 flush is needed between layer steps (the GEMM sweep reads a 512 MB buffer
+between steps instead).
 
---impl reference times the CPU oracle (the only other implementation of this layer; the pages
-ship no code) on a bounded sample of the same workload on the host cores.
-Multi-GPU (torchrun, N>1): the layer does not shard in this build; every rank runs an
-independent replica and the line reports the max-over-ranks time.
+--impl reference times the CPU oracle (the only other implementation of this layer; the source
+pages ship no code) on a bounded sample of the same workload on the host cores.
+Multi-GPU (torchrun, N>1): the layer does not shard; every rank runs an independent replica and
+the line reports the max-over-ranks time.
 """
 from __future__ import annotations
 
