@@ -176,9 +176,10 @@ moe_status_t moe_blockfp8_forward(const moe_blockfp8_args* args, void* ws, size_
  *                  rows outside every range are not written
  *   out            bf16 or fp32 (out_fp32 != 0) [M, N]
  * K and N multiples of 128.  M <= 64 runs the int8 tensor-core path and M > 64 the fp16 path,
- * with the numerics described at moe_w4a16_forward.  On the int8 path, when the shape has few
- * work items (N/128 x ceil(M/8) well below the SM count) the K range is split and the fp32
- * partial sums are added in a fixed order, so results stay identical run to run.
+ * with the numerics described at moe_w4a16_forward.  When the shape has few work items
+ * (N/128 x ceil(M/tile rows), 8 or 256 rows per tile, well below the SM count) the K range is
+ * split and the fp32 partial sums are added in a fixed order, so results stay identical run
+ * to run.
  * ws: moe_w4a16_gemm_workspace_size(M, K, N, E) bytes (includes the partial sums). */
 size_t moe_w4a16_gemm_workspace_size(int M, int K, int N, int E);
 moe_status_t moe_w4a16_gemm(const void* a, int a_is_bf16, const int32_t* w_q, const void* w_s,

@@ -177,14 +177,14 @@ FwdWs carve_w4_forward(void* ws, int T, int H, int I, int E, int k) {
   w.bytes = c.off + 256;
   return w;
 }
-// K splits of the single grouped GEMM on the int8 path: when even the fewest work items the
-// shape can have (all M rows in one expert) leave most of the 148 SMs of a B200 idle, each item's
-// K range is split so that items x splits ~ 148 (at most one 256-K stage per split, at most 32);
-// a shape-only rule, so the workspace size needs no device.
+// K splits of the single grouped GEMM: when even the fewest work items the shape can have (all
+// M rows in one expert) leave most of the 148 SMs of a B200 idle, each item's K range is split
+// so that items x splits ~ 148 (at least one 256-K stage per split, at most 32 splits); a
+// shape-only rule, so the workspace size needs no device.
 int gemm_splits(int M, int K, int N) {
-  if (!use_i8(M)) return 1;
+  const int tile_rows = use_i8(M) ? kI8TileRows : 256;
   const int nkb = (K + 255) / 256;
-  const int items = (N / 128) * ((M + kI8TileRows - 1) / kI8TileRows);
+  const int items = (N / 128) * ((M + tile_rows - 1) / tile_rows);
   int s = 148 / (items > 0 ? items : 1);
   if (s > nkb) s = nkb;
   if (s > 32) s = 32;
@@ -195,7 +195,7 @@ struct GemmWs {
   int32_t *row_count, *tile_prefix, *chunk;
   __half* a;    // fp16 path
   Planes aq;    // int8 path
-  float* part;  // int8 path with K splits: [splits, M, N] fp32 partial sums
+  float* part;  // with K splits: [splits, M, N] fp32 partial sums
   size_t bytes;
 };
 GemmWs carve_gemm(void* ws, int M, int K, int N, int E) {
@@ -204,13 +204,12 @@ GemmWs carve_gemm(void* ws, int M, int K, int N, int E) {
   w.row_count = c.take<int32_t>(E);
   w.tile_prefix = c.take<int32_t>(E + 1);
   w.chunk = c.take<int32_t>(E);
-  if (use_i8(M)) {
+  if (use_i8(M))
     w.aq = take_planes(c, M, K);
-    const int sp = gemm_splits(M, K, N);
-    if (sp > 1) w.part = c.take<float>((size_t)sp * M * N);
-  } else {
+  else
     w.a = c.take<__half>((size_t)M * K);
-  }
+  const int sp = gemm_splits(M, K, N);
+  if (sp > 1) w.part = c.take<float>((size_t)sp * M * N);
   w.bytes = c.off + 256;
   return w;
 }
@@ -424,11 +423,13 @@ moe_status_t moe_w4a16_gemm(const void* a, int a_is_bf16, const int32_t* w_q, co
     return e == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
   }
   if (e == cudaSuccess) e = launch_convert_rows(static_cast<const uint16_t*>(a), a_is_bf16, M, K, w.a, stream);
+  const int sp = gemm_splits(M, K, N);
   if (e == cudaSuccess) {
     W4GemmProblem g{w_q, static_cast<const uint16_t*>(w_s), w.a, M, K, E, N, false, 0, sched, nmax, out, N,
-                    out_fp32 ? OUT_F32 : OUT_BF16};
+                    out_fp32 ? OUT_F32 : OUT_BF16, sp, w.part};
     e = launch_w4a16_gemm(g, stream);
   }
+  if (e == cudaSuccess && sp > 1) e = launch_reduce_splits(w.part, sp, M, N, expert_offsets, E, out, out_fp32, stream);
   return e == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
 }
 

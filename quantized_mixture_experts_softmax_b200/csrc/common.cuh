@@ -265,4 +265,17 @@ __host__ __device__ constexpr uint32_t make_idesc(int M, int N, uint32_t a_fmt, 
 
 __host__ __device__ constexpr int ceil_div(int a, int b) { return (a + b - 1) / b; }
 
+// K stages [kb0, kb1) of split work item `it`: its split is it % splits, and the nkb stages are
+// shared out in balanced contiguous ranges (each split gets at least one when splits <= nkb)
+__device__ __forceinline__ void split_range(int it, int nkb, int splits, int& kb0, int& kb1) {
+  if (splits == 1) {
+    kb0 = 0;
+    kb1 = nkb;
+    return;
+  }
+  const int sp = it % splits;
+  kb0 = sp * nkb / splits;
+  kb1 = (sp + 1) * nkb / splits;
+}
+
 }  // namespace moe

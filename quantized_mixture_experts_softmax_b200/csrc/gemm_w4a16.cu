@@ -81,6 +81,9 @@ struct Params {
   void* out;
   int out_ld;
   int out_kind;
+  int splits;   // K splits per (expert, weight tile, token tile); > 1 only for plain outputs
+  float* part;  // splits > 1: fp32 partial sums [splits, act_rows, out_ld]
+  int act_rows;
   uint64_t wait_limit;
 };
 
@@ -88,8 +91,9 @@ struct Item {
   int e, m, r0, nvalid, nmma;
 };
 
-__device__ __forceinline__ Item decode_item(int it, const int* __restrict__ sprefix, const Params& p) {
+__device__ __forceinline__ Item decode_item(int it_, const int* __restrict__ sprefix, const Params& p) {
   Item I;
+  const int it = p.splits == 1 ? it_ : it_ / p.splits;  // the (expert, weight tile, token tile)
   const int tile = it / p.m_tiles;
   int lo = 0, hi = p.E;  // sprefix[lo] <= tile < sprefix[hi]
   while (hi - lo > 1) {
@@ -203,7 +207,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
-  const int total = p.m_tiles * sprefix[p.E];
+  const int total = p.m_tiles * sprefix[p.E] * p.splits;
   const int K = p.K;
   const int nkb = ceil_div(K, KB);
 
@@ -219,7 +223,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       const uint32_t idesc = make_idesc(BM, I.nmma, 0, 0);
       const uint32_t d0 = tmem_base + (uint32_t)(acc * C::ACC_COLS);  // [matrix][NMAX] columns
       const uint32_t d1 = d0 + NMAX;
-      for (int kb = 0; kb < nkb && ok; ++kb) {
+      int kb0, kb1;
+      split_range(it, nkb, p.splits, kb0, kb1);
+      for (int kb = kb0; kb < kb1 && ok; ++kb) {
         const int nsub = min(NSUB, (K - kb * KB) / KS);
         for (int j = 0; j < nsub; ++j) {
           if (!(ok = bar_red_and(kMmaBarrier, 64, true))) break;
@@ -230,7 +236,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             const uint64_t a1 = sw128_kmajor_desc(smem_u32(smem + C::OFF_A + (ab * NA + (NA - 1)) * C::A_TILE));
 #pragma unroll
             for (int kk = 0; kk < KS / 16; ++kk) {
-              const uint32_t accum = (kb | j | kk) != 0;
+              const uint32_t accum = (kb != kb0) || j != 0 || kk != 0;  // fresh at the split's first K
               umma_f16(d0, a0 + 2 * kk, b + 2 * kk, idesc, accum);  // +32 bytes along K
               if (GATED) umma_f16(d1, a1 + 2 * kk, b + 2 * kk, idesc, accum);
             }
@@ -260,7 +266,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     bool ok = true;
     for (int it = blockIdx.x; it < total && ok; it += gridDim.x) {
       bool ready = __all_sync(0xffffffffu, mbar_wait(&acc_empty[acc], ph_acc ^ 1u, abort_flag, lim));
-      for (int kb = 0; kb < nkb && ok; ++kb) {
+      int kb0, kb1;
+      split_range(it, nkb, p.splits, kb0, kb1);
+      for (int kb = kb0; kb < kb1 && ok; ++kb) {
         const int nsub = min(NSUB, (K - kb * KB) / KS);
         for (int j = 0; j < nsub; ++j) {
           ready = ready && __all_sync(0xffffffffu, mbar_wait(&a_full[ab], ph_a, abort_flag, lim)) &&
@@ -292,7 +300,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       bool ok = true;
       for (int it = blockIdx.x; it < total && ok; it += gridDim.x) {
         const Item I = decode_item(it, sprefix, p);
-        for (int ks = 0; ks < nks; ++ks) {
+        int kb0, kb1;
+        split_range(it, nkb, p.splits, kb0, kb1);
+        const int ks1 = min(nks, kb1 * (KB / KS));
+        for (int ks = kb0 * (KB / KS); ks < ks1; ++ks) {
           if (!(ok = mbar_wait(&empty_b[bs], ph ^ 1u, abort_flag, lim))) break;
           mbar_arrive_expect_tx(&full_b[bs], (uint32_t)(I.nmma * KS * 2));
           // 128-row boxes, then 16-row boxes for the rest (few large copies per step)
@@ -337,6 +348,11 @@ __global__ void __launch_bounds__(kThreads, 1)
               out[(size_t)i * p.out_ld] = __float2half_rn(gv / (1.0f + __expf(-gv)) * uv);
             }
           }
+        } else if (p.splits > 1) {  // this split's partial sum, reduced in split order by another kernel
+          float* out = p.part + (size_t)(it % p.splits) * p.act_rows * p.out_ld + (size_t)(I.r0 + c0) * p.out_ld + col;
+#pragma unroll
+          for (int i = 0; i < 16; ++i)
+            if (i < nv) out[(size_t)i * p.out_ld] = __uint_as_float(g[i]);
         } else if (p.out_kind == OUT_F32) {
           float* out = reinterpret_cast<float*>(p.out) + (size_t)(I.r0 + c0) * p.out_ld + col;
 #pragma unroll
@@ -397,17 +413,25 @@ __global__ void __launch_bounds__(kThreads, 1)
     bool ok = true;
     uint4 wn[CHK], sn;
     int wr = blockIdx.x < total ? weight_row(blockIdx.x) : 0;
-    if (blockIdx.x < total) load_stage(wr, 0, wn, sn);
+    if (blockIdx.x < total) {
+      int f0, f1;
+      split_range(blockIdx.x, nkb, p.splits, f0, f1);
+      load_stage(wr, f0, wn, sn);
+    }
     for (int it = blockIdx.x; it < total && ok; it += gridDim.x) {
-      const int wr_next = it + (int)gridDim.x < total ? weight_row(it + gridDim.x) : wr;
-      for (int kb = 0; kb < nkb && ok; ++kb) {
+      const bool has_next = it + (int)gridDim.x < total;
+      const int wr_next = has_next ? weight_row(it + gridDim.x) : wr;
+      int kb0, kb1, nkb0, nkb1;
+      split_range(it, nkb, p.splits, kb0, kb1);
+      split_range(it + gridDim.x, nkb, p.splits, nkb0, nkb1);
+      for (int kb = kb0; kb < kb1 && ok; ++kb) {
         uint4 wv[CHK], sc = sn;
 #pragma unroll
         for (int c = 0; c < CHK; ++c) wv[c] = wn[c];
-        if (kb + 1 < nkb)
+        if (kb + 1 < kb1)
           load_stage(wr, kb + 1, wn, sn);
-        else if (it + (int)gridDim.x < total)
-          load_stage(wr_next, 0, wn, sn);
+        else if (has_next)
+          load_stage(wr_next, nkb0, wn, sn);
         const int nsub = min(NSUB, (K - kb * KB) / KS);
 #pragma unroll
         for (int j = 0; j < NSUB; ++j) {
@@ -470,6 +494,9 @@ cudaError_t launch_t(const W4GemmProblem& pr, cudaStream_t s) {
   p.out = pr.out;
   p.out_ld = pr.out_ld;
   p.out_kind = pr.out_kind;
+  p.splits = pr.splits > 1 && !GATED ? pr.splits : 1;
+  p.part = pr.part;
+  p.act_rows = pr.act_rows;
   p.wait_limit = wait_limit_ns();
   const size_t smem = C::smem_bytes(pr.E);
   auto kern = w4a16_gemm_kernel<GATED>;

@@ -108,18 +108,6 @@ struct Item {
   int e, m, r0, nvalid;
 };
 
-// K stages [kb0, kb1) of work item `it` (its K split: it % splits of the nkb stages, balanced)
-__device__ __forceinline__ void kb_range(int it, int nkb, int splits, int& kb0, int& kb1) {
-  if (splits == 1) {
-    kb0 = 0;
-    kb1 = nkb;
-    return;
-  }
-  const int sp = it % splits;
-  kb0 = sp * nkb / splits;
-  kb1 = (sp + 1) * nkb / splits;
-}
-
 __device__ __forceinline__ Item decode_item(int it_, const int* __restrict__ sprefix, const Params& p) {
   Item I;
   const int it = p.splits == 1 ? it_ : it_ / p.splits;  // the (expert, weight tile, token tile)
@@ -305,7 +293,7 @@ __device__ __forceinline__ bool epi_item(const Params& p, const Item& I, int it,
 #pragma unroll
   for (int c = 0; c < NP; ++c) P.ag[c] = P.au[c] = 0.f;
   int kb0, kb1;
-  kb_range(it, ceil_div(p.K, KB), p.splits, kb0, kb1);
+  split_range(it, ceil_div(p.K, KB), p.splits, kb0, kb1);
   if (!promote_item<GATED, NP>(p, I, mrow, lane, lane_base, smem, s, ph, full, empty, ds, ph_d, d_full, d_empty,
                                abort_flag, kb0, kb1, P))
     return false;
@@ -443,7 +431,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int row_g = I.e * p.rows_per_expert + I.m * BM;
       const int row_u = row_g + p.I;
       int kb0, kb1;
-      kb_range(it, nkb, p.splits, kb0, kb1);
+      split_range(it, nkb, p.splits, kb0, kb1);
       for (int kb = kb0; kb < kb1; ++kb) {
         if (!(ok = __all_sync(0xffffffffu, mbar_wait(&empty[s], ph ^ 1u, abort_flag, lim)))) break;
         uint8_t* st = smem + s * C::STAGE;
@@ -497,7 +485,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     bool ok = true;
     for (int it = blockIdx.x; it < total && ok; it += gridDim.x) {
       int kb0, kb1;
-      kb_range(it, nkb, p.splits, kb0, kb1);
+      split_range(it, nkb, p.splits, kb0, kb1);
       for (int kb = kb0; kb < kb1 && ok; ++kb) {
         const int ng = min(KB, K - kb * KB) / G;
         // descriptors and addresses from per-stage bases plus constants, so that the issue loop
@@ -553,7 +541,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 
     for (int it = blockIdx.x; it < total && ok; it += gridDim.x) {
       int kb0, kb1;
-      kb_range(it, nkb, p.splits, kb0, kb1);
+      split_range(it, nkb, p.splits, kb0, kb1);
       for (int kb = kb0; kb < kb1 && ok; ++kb) {
         const int ng = min(KB, K - kb * KB) / G;
         bool ready = __all_sync(0xffffffffu, mbar_wait(&full[s], ph, abort_flag, lim)) &&
@@ -622,7 +610,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     bool ok = true;
     for (int it = blockIdx.x; it < total && ok; it += gridDim.x) {
       int kb0, kb1;
-      kb_range(it, nkb, p.splits, kb0, kb1);
+      split_range(it, nkb, p.splits, kb0, kb1);
       for (int kb = kb0; kb < kb1 && ok; ++kb) {
         const int ng = min(KB, K - kb * KB) / G;
         ok = __all_sync(0xffffffffu, mbar_wait(&full[s], ph, abort_flag, lim));

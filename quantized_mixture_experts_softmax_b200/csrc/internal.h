@@ -57,6 +57,8 @@ struct W4GemmProblem {
   void* out;
   int out_ld;          // elements per output row
   OutKind out_kind;
+  int splits = 1;          // plain outputs: K split this many ways into `part`, then reduce_splits
+  float* part = nullptr;   // [splits, act_rows, out_ld] fp32
 };
 cudaError_t launch_w4a16_gemm(const W4GemmProblem& p, cudaStream_t s);
 
