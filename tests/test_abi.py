@@ -46,6 +46,12 @@ def test_workspace_queries(native):
     assert ws >= 512 * (7168 * 2 + 2048 * 2 + 7168 * 4)
     assert L.moe_w4a16_workspace_size(64, 7000, 2048, 384, 8) == 0  # H not a multiple of 128
     assert L.moe_w4a16_gemm_workspace_size(1, 7168, 512, 1) > 0
+    # few work items: the K range is split (28 splits of one 256-K stage for 4 items), and the
+    # workspace holds their fp32 partial sums
+    assert L.moe_w4a16_gemm_workspace_size(1, 7168, 512, 1) >= 28 * 1 * 512 * 4
+    assert L.moe_w4a16_gemm_workspace_size(512, 7168, 512, 1) >= 18 * 512 * 512 * 4
+    # enough items (32768 rows): no partial sums beyond the fp16 copy of the activations
+    assert L.moe_w4a16_gemm_workspace_size(32768, 7168, 512, 1) < 32768 * 7168 * 2 + 2 * 32768 * 512 * 4
     assert L.moe_w4a16_gemm_workspace_size(1, 7000, 512, 1) == 0
 
 
