@@ -386,15 +386,24 @@ def run_ours(args, world, rank):
             g.replay()
         torch.cuda.synchronize()
         barrier(world)
-        ev0.record(stream)
-        for _ in range(steps):
+        # an event between replays gives each replay's duration as well as the total
+        reps = max(steps, 100)
+        evs = [torch.cuda.Event(enable_timing=True) for _ in range(reps + 1)]
+        evs[0].record(stream)
+        for i in range(reps):
             g.replay()
-        ev1.record(stream)
+            evs[i + 1].record(stream)
         torch.cuda.synchronize()
         barrier(world)
         assert moe.moe_get_device_status() == 0
-        graph = {"value": round(max_over_ranks(ev0.elapsed_time(ev1), world) / steps * 1e3 / world, 2),
-                 "unit": "µs/layer", "note": "the timed step (route + layer) replayed from one CUDA graph"}
+        per_us = np.array([evs[i].elapsed_time(evs[i + 1]) for i in range(reps)]) * 1e3
+        stats = {name: round(max_over_ranks(float(v), world) / world, 2)
+                 for name, v in (("median", np.median(per_us)), ("min", per_us.min()),
+                                 ("p90", np.percentile(per_us, 90)))}
+        graph = {"value": round(max_over_ranks(evs[0].elapsed_time(evs[-1]), world) / reps * 1e3 / world, 2),
+                 "unit": "µs/layer", "replays": reps, **stats,
+                 "note": "the timed step (route + layer) replayed from one CUDA graph; value = mean, "
+                         "median/min/p90 over the replays (max over ranks)"}
         del g
     except Exception as exc:  # capture refused: report why instead of a number
         graph = {"value": None, "unit": "µs/layer", "note": f"capture failed: {type(exc).__name__}: {exc}"[:200]}
