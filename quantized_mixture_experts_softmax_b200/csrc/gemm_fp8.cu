@@ -13,12 +13,15 @@
 //               tiles for the gate/up GEMM) and the token tile's activations, one stage per
 //               128-K block;
 //   warp 1      TMEM allocator and single-thread MMA issuer: four K=32 MMAs per matrix per block
-//               into a double-buffered partial-product tile; it never waits on an mbarrier
-//               (see bar_red_and) and is released block by block by
+//               into one of four partial-product tiles (two where four would pass 512 columns),
+//               so the MMAs run up to three blocks ahead of the promotion; it never waits on an
+//               mbarrier (see bar_red_and) and is released block by block by
 //   warp 2      the MMA scheduler, which waits for the stage's copies and a free partial tile;
 //   warps 3-10  promotion and epilogue, two per TMEM lane quarter: each thread owns one weight
 //               row and keeps the fp32 accumulators of one half of the tile's tokens (32 of up
-//               to 64) in registers.  The gate/up GEMM ends with h = SiLU(gate) * up,
+//               to 64) in registers.  A block's scale w_scale * x_scale is the same for all 128
+//               rows of a token, so each warp forms the 32 products once (a lane per token) and
+//               every lane reads them back as float4 broadcasts from shared memory.  The gate/up GEMM ends with h = SiLU(gate) * up,
 //               requantized per (token, 128-column group) - the tile's 128 rows are exactly one
 //               group - to e4m3 with s = max(amax, 1e-10) / 448; the down GEMM stores fp32.
 #include <cuda_fp8.h>
@@ -49,13 +52,17 @@ struct Cfg {
   static constexpr int STAGE = NA * W_TILE + B_TILE;
   static constexpr int ST = NMAX == 32 ? (GATED ? 6 : 10) : (GATED ? 5 : 9);
   static constexpr int P_COLS = NA * NMAX;  // one partial-product tile: [matrix][NMAX] columns
-  static constexpr int TMEM_COLS = 2 * P_COLS <= 32 ? 32 : (2 * P_COLS <= 64 ? 64 : (2 * P_COLS <= 128 ? 128 : 256));
-  static_assert(2 * P_COLS <= TMEM_COLS, "two partial-product tiles fit the allocation");
+  // partial-product tiles in flight between the MMA and the promotion warps (as many as fit)
+  static constexpr int NPB = 4 * P_COLS <= 512 ? 4 : 2;
+  static constexpr int TMEM_COLS = NPB * P_COLS <= 32 ? 32 : (NPB * P_COLS <= 64 ? 64 : (NPB * P_COLS <= 128 ? 128 : (NPB * P_COLS <= 256 ? 256 : 512)));
+  static_assert(NPB * P_COLS <= TMEM_COLS && TMEM_COLS <= 512, "the partial-product tiles fit the allocation");
   static constexpr int OFF_BAR = ST * STAGE;
-  static constexpr int NUM_BARS = 2 * ST + 4 + 2;
+  static constexpr int NUM_BARS = 2 * ST + 2 * NPB + 2;
   static constexpr int OFF_MISC = OFF_BAR + NUM_BARS * 8;
   static constexpr int OFF_RED = OFF_MISC + 16;              // [4 lane quarters][NMAX] amax partials
-  static constexpr int OFF_PREFIX = OFF_RED + 4 * NMAX * 4;
+  static constexpr int OFF_CS = OFF_RED + 4 * NMAX * 4;      // [promotion warp][matrix][NH] block scales
+  static constexpr int OFF_PREFIX = OFF_CS + kNumEpi * NA * NH * 4;
+  static_assert(OFF_CS % 16 == 0, "float4 reads of the block scales");
   static_assert(STAGE % 1024 == 0, "swizzled tiles need 1024-byte alignment");
   static constexpr size_t smem_bytes(int E) { return (size_t)OFF_PREFIX + 4 * (size_t)(E + 1) + 1024; }
   static_assert(smem_bytes(1024) <= 232448, "shared memory budget");
@@ -121,12 +128,13 @@ __global__ void __launch_bounds__(Cfg<GATED, NMAX>::kThreads, 1)
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + C::OFF_BAR);
   uint64_t* empty = full + ST;
   uint64_t* p_full = empty + ST;
-  uint64_t* p_empty = p_full + 2;
-  uint64_t* drain = p_empty + 2;
+  uint64_t* p_empty = p_full + C::NPB;
+  uint64_t* drain = p_empty + C::NPB;
   uint64_t* epi_bar = drain + 1;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::OFF_MISC);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::OFF_MISC + 4);
   float* red = reinterpret_cast<float*>(smem + C::OFF_RED);
+  float* cscale = reinterpret_cast<float*>(smem + C::OFF_CS);
   int* sprefix = reinterpret_cast<int*>(smem + C::OFF_PREFIX);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -138,7 +146,7 @@ __global__ void __launch_bounds__(Cfg<GATED, NMAX>::kThreads, 1)
       mbar_init(&full[i], 1);
       mbar_init(&empty[i], 1);
     }
-    for (int i = 0; i < 2; ++i) {
+    for (int i = 0; i < C::NPB; ++i) {
       mbar_init(&p_full[i], 1);
       mbar_init(&p_empty[i], kNumEpi);
     }
@@ -218,7 +226,7 @@ __global__ void __launch_bounds__(Cfg<GATED, NMAX>::kThreads, 1)
         }
         __syncwarp();
         if (++s == ST) s = 0;
-        if (++pb == 2) pb = 0;
+        if (++pb == C::NPB) pb = 0;
       }
     }
     if (lane == 0) {
@@ -239,7 +247,7 @@ __global__ void __launch_bounds__(Cfg<GATED, NMAX>::kThreads, 1)
           s = 0;
           ph ^= 1u;
         }
-        if (++pb == 2) {
+        if (++pb == C::NPB) {
           pb = 0;
           ph_p ^= 1u;
         }
@@ -251,6 +259,8 @@ __global__ void __launch_bounds__(Cfg<GATED, NMAX>::kThreads, 1)
     const int tok0 = ((warp - kEpiWarp0) >> 2) * NH;  // this warp's half of the tile's tokens
     const int mrow = ew * 32 + lane;
     const int GK = p.K / KB;
+    // this warp's combined scales of the current block, w_scale * x_scale per token
+    float* cs = cscale + (warp - kEpiWarp0) * NA * NH;
     int pb = 0;
     uint32_t ph_p = 0, ph_e = 0;
     bool ok = true;
@@ -278,6 +288,11 @@ __global__ void __launch_bounds__(Cfg<GATED, NMAX>::kThreads, 1)
         ok = __all_sync(0xffffffffu, mbar_wait(&p_full[pb], ph_p, abort_flag, lim));
         if (!ok) break;
         tc_fence_after();
+        // the scale of (row block, token) is uniform over the warp's rows: one product per token,
+        // read back by every lane as float4 broadcasts
+        cs[lane] = sg * xs_l;
+        if (GATED) cs[NH + lane] = su * xs_l;
+        __syncwarp();
         const uint32_t tb = tmem_base + ((uint32_t)(ew * 32) << 16) + (uint32_t)(pb * C::P_COLS + tok0);
         uint32_t pg[16], pu[16];
 #pragma unroll
@@ -287,17 +302,26 @@ __global__ void __launch_bounds__(Cfg<GATED, NMAX>::kThreads, 1)
             if (GATED) tmem_ld16(tb + NMAX + c0, pu);
             tmem_ld_wait();
 #pragma unroll
-            for (int i = 0; i < 16; ++i) {
-              const float xs = __shfl_sync(0xffffffffu, xs_l, c0 + i);
-              ag[c0 + i] = fmaf(__uint_as_float(pg[i]), sg * xs, ag[c0 + i]);
-              if (GATED) au[c0 + i] = fmaf(__uint_as_float(pu[i]), su * xs, au[c0 + i]);
+            for (int i = 0; i < 16; i += 4) {
+              const float4 g4 = *reinterpret_cast<const float4*>(cs + c0 + i);
+              ag[c0 + i + 0] = fmaf(__uint_as_float(pg[i + 0]), g4.x, ag[c0 + i + 0]);
+              ag[c0 + i + 1] = fmaf(__uint_as_float(pg[i + 1]), g4.y, ag[c0 + i + 1]);
+              ag[c0 + i + 2] = fmaf(__uint_as_float(pg[i + 2]), g4.z, ag[c0 + i + 2]);
+              ag[c0 + i + 3] = fmaf(__uint_as_float(pg[i + 3]), g4.w, ag[c0 + i + 3]);
+              if (GATED) {
+                const float4 u4 = *reinterpret_cast<const float4*>(cs + NH + c0 + i);
+                au[c0 + i + 0] = fmaf(__uint_as_float(pu[i + 0]), u4.x, au[c0 + i + 0]);
+                au[c0 + i + 1] = fmaf(__uint_as_float(pu[i + 1]), u4.y, au[c0 + i + 1]);
+                au[c0 + i + 2] = fmaf(__uint_as_float(pu[i + 2]), u4.z, au[c0 + i + 2]);
+                au[c0 + i + 3] = fmaf(__uint_as_float(pu[i + 3]), u4.w, au[c0 + i + 3]);
+              }
             }
           }
         }
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(&p_empty[pb]);
-        if (++pb == 2) {
+        if (++pb == C::NPB) {
           pb = 0;
           ph_p ^= 1u;
         }
