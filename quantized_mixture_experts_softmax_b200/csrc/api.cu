@@ -2,6 +2,7 @@
 // launch sequencing, the device status word and the benchmark timing hooks.
 #include <cuda.h>
 #include <cudaTypedefs.h>
+#include <nvtx3/nvToolsExt.h>
 
 #include <algorithm>
 #include <cstring>
@@ -119,13 +120,19 @@ cudaEvent_t get_event() {
 }
 }  // namespace
 
+// Every kernel launch sits between these two calls.  They open and close an NVTX range named
+// after the kernel (a timeline tool attached to the process shows which launch each range
+// enqueued; without one the calls do nothing) and, while moe_timing_enable(1) is in effect,
+// bracket the launch with CUDA events for moe_timing_read.
 void timing_before(const char* name, cudaStream_t s) {
+  nvtxRangePushA(name);
   if (!g_timing_on) return;
   Rec r{name, get_event(), get_event()};
   cudaEventRecord(r.a, s);
   g_recs.push_back(r);
 }
 void timing_after(const char*, cudaStream_t s) {
+  nvtxRangePop();
   if (!g_timing_on || g_recs.empty()) return;
   cudaEventRecord(g_recs.back().b, s);
 }
