@@ -71,3 +71,147 @@ def test_argument_errors_return_codes(native):
     assert L.moe_align(ctypes.c_void_p(fake), 4, 2, 8, 0, *([ctypes.c_void_p(fake)] * 5), 1 << 20,
                        None) == native.MOE_ERR_UNSUPPORTED  # align 0
     assert L.moe_debug_wait_timeout(0, None) == native.MOE_ERR_INVALID_ARG
+
+
+def test_binding_structs_match_the_header(native, tmp_path):
+    """The Python argument structs have the header's field offsets and sizes (a C program built
+    against include/moe.h prints them)."""
+    import shutil
+    import subprocess
+
+    gcc = shutil.which("gcc")
+    if gcc is None:
+        pytest.skip("no C compiler")
+    fields = {"moe_w4a16_args": [f for f, _ in native.W4A16Args._fields_],
+              "moe_blockfp8_args": [f for f, _ in native.BlockFP8Args._fields_]}
+    lines = ["#include <stdio.h>", "#include <stddef.h>", '#include "moe.h"', "int main(void) {"]
+    for st, names in fields.items():
+        lines.append(f'  printf("{st} size %zu\\n", sizeof({st}));')
+        for n in names:
+            lines.append(f'  printf("{st} {n} %zu\\n", offsetof({st}, {n}));')
+    lines += ["  return 0;", "}"]
+    src = tmp_path / "layout.c"
+    src.write_text("\n".join(lines) + "\n")
+    exe = tmp_path / "layout"
+    cuda_inc = os.path.join(os.environ.get("CUDA_HOME", "/usr/local/cuda"), "include")
+    subprocess.check_call([gcc, "-I", os.path.join(ROOT, "include"), "-I", cuda_inc, "-o", str(exe), str(src)])
+    got = {}
+    for line in subprocess.check_output([str(exe)]).decode().splitlines():
+        st, n, v = line.split()
+        got[(st, n)] = int(v)
+    for st, cls in (("moe_w4a16_args", native.W4A16Args), ("moe_blockfp8_args", native.BlockFP8Args)):
+        assert got[(st, "size")] == ctypes.sizeof(cls), st
+        for n in fields[st]:
+            assert got[(st, n)] == getattr(cls, n).offset, (st, n)
+
+
+def _w4(native, **kw):
+    fake = 1 << 20
+    d = dict(x=fake, topk_ids=fake, topk_w=fake, w13_q=fake, w13_s=fake, w2_q=fake, w2_s=fake,
+             T=64, H=7168, I=2048, E=384, k=8, out=fake, out_fp32=0)
+    d.update(kw)
+    return native.W4A16Args(*[d[f] for f, _ in native.W4A16Args._fields_])
+
+
+def _f8(native, **kw):
+    fake = 1 << 20
+    d = dict(x=fake, xs=fake, topk_ids=fake, topk_w=fake, w13=fake, w13_s=fake, w2=fake, w2_s=fake,
+             T=64, H=7168, I=2048, E=256, k=8, out=fake, out_fp32=0)
+    d.update(kw)
+    return native.BlockFP8Args(*[d[f] for f, _ in native.BlockFP8Args._fields_])
+
+
+# shapes outside the documented limits: T >= 1, 1 <= k <= E <= 1024, H and I multiples of 128
+BAD_SHAPES = [dict(T=0), dict(k=0), dict(E=0), dict(E=1025, k=8), dict(k=9, E=8), dict(H=7100), dict(I=2000),
+              dict(H=0), dict(I=64)]
+# pointers the calls need aligned (16 bytes for tensors read as vectors, 4 for scalars)
+BAD_PTRS_W4 = ["x", "w13_q", "w13_s", "w2_q", "w2_s", "out"]
+BAD_PTRS_F8 = ["x", "w13", "w2", "out"]
+
+
+@pytest.mark.parametrize("kw", BAD_SHAPES, ids=lambda d: ",".join(f"{a}={b}" for a, b in d.items()))
+def test_forward_shape_limits(native, kw):
+    L = native.lib
+    fake = ctypes.c_void_p(1 << 20)
+    a = _w4(native, **kw)
+    assert L.moe_w4a16_forward(ctypes.byref(a), fake, 1 << 40, None) == native.MOE_ERR_UNSUPPORTED
+    assert L.moe_w4a16_workspace_size(a.T, a.H, a.I, a.E, a.k) == 0
+    f = _f8(native, **kw)
+    assert L.moe_blockfp8_forward(ctypes.byref(f), fake, 1 << 40, None) == native.MOE_ERR_UNSUPPORTED
+    assert L.moe_blockfp8_workspace_size(f.T, f.H, f.I, f.E, f.k) == 0
+
+
+@pytest.mark.parametrize("field", BAD_PTRS_W4)
+def test_w4a16_forward_rejects_misaligned_or_null(native, field):
+    L = native.lib
+    fake = ctypes.c_void_p(1 << 20)
+    for bad in (0, (1 << 20) + 8):
+        a = _w4(native, **{field: bad})
+        assert L.moe_w4a16_forward(ctypes.byref(a), fake, 1 << 40, None) == native.MOE_ERR_INVALID_ARG, (field, bad)
+    a = _w4(native, topk_ids=(1 << 20) + 2)
+    assert L.moe_w4a16_forward(ctypes.byref(a), fake, 1 << 40, None) == native.MOE_ERR_INVALID_ARG
+    a = _w4(native)
+    assert L.moe_w4a16_forward(ctypes.byref(a), ctypes.c_void_p((1 << 20) + 16), 1 << 40, None) == \
+        native.MOE_ERR_INVALID_ARG  # workspace base must be 256-byte aligned
+
+
+@pytest.mark.parametrize("field", BAD_PTRS_F8)
+def test_blockfp8_forward_rejects_misaligned_or_null(native, field):
+    L = native.lib
+    fake = ctypes.c_void_p(1 << 20)
+    for bad in (0, (1 << 20) + 8):
+        f = _f8(native, **{field: bad})
+        assert L.moe_blockfp8_forward(ctypes.byref(f), fake, 1 << 40, None) == native.MOE_ERR_INVALID_ARG, (field, bad)
+    f = _f8(native, xs=(1 << 20) + 2)
+    assert L.moe_blockfp8_forward(ctypes.byref(f), fake, 1 << 40, None) == native.MOE_ERR_INVALID_ARG
+
+
+def test_forward_workspace_one_byte_short(native):
+    L = native.lib
+    fake = ctypes.c_void_p(1 << 20)
+    a = _w4(native)
+    need = L.moe_w4a16_workspace_size(a.T, a.H, a.I, a.E, a.k)
+    assert L.moe_w4a16_forward(ctypes.byref(a), fake, need - 1, None) == native.MOE_ERR_WORKSPACE
+    f = _f8(native)
+    need = L.moe_blockfp8_workspace_size(f.T, f.H, f.I, f.E, f.k)
+    assert need > 0
+    assert L.moe_blockfp8_forward(ctypes.byref(f), fake, need - 1, None) == native.MOE_ERR_WORKSPACE
+
+
+@pytest.mark.parametrize("M,K,N,E", [(0, 7168, 512, 1), (1, 7100, 512, 1), (1, 7168, 500, 1), (1, 64, 512, 1),
+                                     (1, 7168, 512, 0), (1, 7168, 512, 1025)])
+def test_gemm_shape_limits(native, M, K, N, E):
+    L = native.lib
+    fake = ctypes.c_void_p(1 << 20)
+    assert L.moe_w4a16_gemm_workspace_size(M, K, N, E) == 0
+    assert L.moe_w4a16_gemm(fake, 1, fake, fake, fake, M, K, N, E, fake, 0, fake, 1 << 40, None) == \
+        native.MOE_ERR_UNSUPPORTED
+
+
+def test_gemm_alignment_and_workspace(native):
+    L = native.lib
+    ok, bad = ctypes.c_void_p(1 << 20), ctypes.c_void_p((1 << 20) + 8)
+    M, K, N, E = 64, 7168, 512, 2
+    need = L.moe_w4a16_gemm_workspace_size(M, K, N, E)
+    args = [ok, 1, ok, ok, ok, M, K, N, E, ok, 0, ok, need, None]
+    for i in (0, 2, 3, 9):  # a, w_q, w_s, out
+        a = list(args)
+        a[i] = bad
+        assert L.moe_w4a16_gemm(*a) == native.MOE_ERR_INVALID_ARG, i
+    a = list(args)
+    a[12] = need - 1
+    assert L.moe_w4a16_gemm(*a) == native.MOE_ERR_WORKSPACE
+
+
+def test_route_and_align_limits(native):
+    L = native.lib
+    p = ctypes.c_void_p(1 << 20)
+    for T, E, k in ((0, 8, 2), (4, 8, 0), (4, 1025, 8), (4, 0, 0)):
+        assert L.moe_route(p, T, E, k, 1, p, p, None) == native.MOE_ERR_UNSUPPORTED, (T, E, k)
+    assert L.moe_route(ctypes.c_void_p((1 << 20) + 2), 4, 8, 2, 1, p, p, None) == native.MOE_ERR_INVALID_ARG
+    ws = L.moe_align_workspace_size(4, 2, 8)
+    assert L.moe_align(p, 0, 2, 8, 16, p, p, p, p, p, ws, None) == native.MOE_ERR_UNSUPPORTED
+    assert L.moe_align(p, 4, 2, 1025, 16, p, p, p, p, p, 1 << 30, None) == native.MOE_ERR_UNSUPPORTED
+    assert L.moe_align(ctypes.c_void_p((1 << 20) + 2), 4, 2, 8, 16, p, p, p, p, p, ws, None) == \
+        native.MOE_ERR_INVALID_ARG
+    assert L.moe_align(p, 4, 2, 8, 16, p, p, p, p, p, ws - 1, None) == native.MOE_ERR_WORKSPACE
