@@ -233,6 +233,21 @@ def make_inputs(seed: int, T: int, zipf: float, kind: str = "w4a16"):
     return x, lg
 
 
+def layer_config(workload: str, kind: str, T: int, H: int, I: int, E: int, k: int, active: int, world: int) -> dict:
+    """The `config` object of a layer workload's JSON line (the same for both arms)."""
+    return {"workload": f"{workload} {'block-FP8' if kind == 'fp8' else 'W4A16'} MoE layer T={T} H={H} I={I} E={E} "
+                        f"top-{k}",
+            "T": T, "H": H, "I": I, "E": E, "k": k, "active_experts": active,
+            "parallelism": "replicas" if world > 1 else "single GPU",
+            "l2": "no flush: the active experts' weights streamed per step exceed the 126 MB L2"}
+
+
+def gemm_config(M: int, K: int, N: int) -> dict:
+    """The `config` object of a single-GEMM sweep line (the same for both arms)."""
+    return {"workload": f"single-expert W4A16 GEMM [{M},{K}]x[{K},{N}]", "M": M, "K": K, "N": N,
+            "l2": "512 MB buffer read between steps; time = the library's kernels only"}
+
+
 def run_gemm(args, world, rank):
     """The single-expert W4A16 GEMM sweep through moe_w4a16_gemm.  Small operands fit in L2, so
     a 512 MB buffer is read between steps (a read leaves no dirty lines to write back during the
@@ -298,8 +313,7 @@ def run_gemm(args, world, rank):
         "scaling": "weak", "vs_baseline": None,
         "dtype": "w4a16 as int8 MMA + fp32 promotion" if M <= 64 else "w4a16 (fp16 MMA, fp32 acc)",
         "data": "synthetic (seeded counter-based generator)",
-        "config": {"workload": f"single-expert W4A16 GEMM [{M},{K}]x[{K},{N}]", "M": M, "K": K, "N": N,
-                   "l2": "512 MB buffer read between steps; time = the library's kernels only"},
+        "config": gemm_config(M, K, N),
         "kernels_ms_per_step": {k_: round(v[0] / steps, 4) for k_, v in kern.items()},
         "gpu_launches": launches, "roofline": roof, "clocks": clk.summary(),
     }
@@ -502,11 +516,7 @@ def run_ours(args, world, rank):
         "dtype": {"fp8": "e4m3 (fp32 acc)", "w4a16": "w4a16 (fp16 MMA, fp32 acc)",
                   "w4i8": "w4a16 as int8 MMA (u8 weights x 16-bit fixed-point activations, s32) + fp32 promotion"}[family],
         "data": "synthetic (seeded counter-based generator; random-init quantized weights)",
-        "config": {"workload": f"{args.workload} {'block-FP8' if kind == 'fp8' else 'W4A16'} MoE layer T={T} "
-                               f"H={H} I={I} E={E} top-{k}",
-                   "T": T, "H": H, "I": I, "E": E, "k": k, "active_experts": active,
-                   "parallelism": "replicas" if world > 1 else "single GPU",
-                   "l2": "no flush: the active experts' weights streamed per step exceed the 126 MB L2"},
+        "config": layer_config(args.workload, kind, T, H, I, E, k, active, world),
         "layer": {"us": round(ms_step * 1e3, 2), "tflops": round(flops / (ms_step * 1e-3) / 1e12, 2),
                   "hbm_gbs": round(layer_bytes / (ms_step * 1e-3) / 1e9, 1),
                   "hbm_frac": round(layer_bytes / (ms_step * 1e-3) / 1e9 / peaks["hbm"], 4),
@@ -591,15 +601,18 @@ def run_reference(args, world, rank):
             "metric": GEMM_METRIC, "value": round(v, 1), "unit": "µs/GEMM", "n_gpus": world, "steps": steps,
             "warmup": warmup, "ms_per_step": round(v / 1e3, 3), "higher_is_better": False, "scaling": "weak",
             "vs_baseline": None, "dtype": "f64 (oracle)", "data": "synthetic",
-            "config": {"workload": f"single-expert W4A16 GEMM [{M},{K}]x[{K},{N}]"}, "impl": "reference",
+            "config": gemm_config(M, K, N), "impl": "reference",
             "cpu_baseline": {"value": round(v, 1), "unit": "µs/GEMM", "cores": cores, "kind": "oracle",
                              "sample": sample},
             "e2e": {"value": round(v, 1), "unit": "µs/GEMM", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
         }
+    import oracle
+    M = FP8_MODEL if wl["kind"] == "fp8" else MODEL
     T = wl["T"]
     steps = args.steps if args.steps is not None else 3
     warmup = args.warmup if args.warmup is not None else 1
     x_h, lg_h = make_inputs(0, T, wl["zipf"], wl["kind"])
+    active = int(np.unique(oracle.route(lg_h, M["k"])[0]).size)  # the routing both arms compute
     vals = []
     sample = cores = None
     for i in range(warmup + steps):
@@ -611,8 +624,7 @@ def run_reference(args, world, rank):
         "metric": METRIC, "value": round(v, 1), "unit": "µs/layer", "n_gpus": world, "steps": steps,
         "warmup": warmup, "ms_per_step": round(v / 1e3, 3), "higher_is_better": False, "scaling": "weak",
         "vs_baseline": None, "dtype": "f64 (oracle)", "data": "synthetic",
-        "config": {"workload": f"{args.workload} {'block-FP8' if wl['kind'] == 'fp8' else 'W4A16'} MoE layer "
-                               f"T={T}"},
+        "config": layer_config(args.workload, wl["kind"], T, M["H"], M["I"], M["E"], M["k"], active, world),
         "impl": "reference",
         "cpu_baseline": {"value": round(v, 1), "unit": "µs/layer", "cores": cores, "kind": "oracle",
                          "sample": sample},

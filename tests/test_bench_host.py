@@ -78,3 +78,40 @@ def test_workloads_cover_the_layer_configurations():
     assert sorted(v["T"] for n, v in w.items() if n.startswith("fp8_")) == [1, 16, 64, 512, 4096]
     for v in w.values():
         assert v["warmup"] >= 3  # the timing rule's minimum
+
+
+def _args(workload, steps=1, warmup=0):
+    import argparse
+    return argparse.Namespace(workload=workload, steps=steps, warmup=warmup, gpus=1, impl="reference",
+                              no_cpu_baseline=False, experts=None, tokens=None)
+
+
+def _check_reference_line(line, metric, unit):
+    assert line["impl"] == "reference"
+    assert line["metric"] == metric and line["unit"] == unit and line["higher_is_better"] is False
+    assert line["value"] > 0 and line["steps"] == 1
+    cb = line["cpu_baseline"]
+    assert cb["kind"] == "oracle" and cb["value"] == line["value"] and cb["unit"] == unit and cb["cores"] >= 1
+    assert "of" in cb["sample"]
+    assert line["e2e"] == {"value": line["value"], "unit": unit, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}
+
+
+def test_reference_arm_layer_line(monkeypatch):
+    """The oracle arm prints the contract's line with the config our arm prints for the same
+    workload (checked on a reduced model so that it runs in a moment)."""
+    import oracle
+    for key, v in dict(H=256, I=128, E=8, k=2).items():
+        monkeypatch.setitem(bench.MODEL, key, v)
+    monkeypatch.setitem(bench.WORKLOADS, "decode", dict(bench.WORKLOADS["decode"], T=16))
+    line = bench.run_reference(_args("decode"), 1, 0)
+    _check_reference_line(line, bench.METRIC, "µs/layer")
+    _, lg = bench.make_inputs(0, 16, 0.0)
+    active = int(np.unique(oracle.route(lg, 2)[0]).size)
+    assert line["config"] == bench.layer_config("decode", "w4a16", 16, 256, 128, 8, 2, active, 1)
+    assert line["cpu_baseline"]["sample"].startswith("16 of 16 tokens")
+
+
+def test_reference_arm_gemm_line():
+    line = bench.run_reference(_args("gemm_m1_k7168_n512"), 1, 0)
+    _check_reference_line(line, bench.GEMM_METRIC, "µs/GEMM")
+    assert line["config"] == bench.gemm_config(1, 7168, 512)
