@@ -215,3 +215,19 @@ def test_route_and_align_limits(native):
     assert L.moe_align(ctypes.c_void_p((1 << 20) + 2), 4, 2, 8, 16, p, p, p, p, p, ws, None) == \
         native.MOE_ERR_INVALID_ARG
     assert L.moe_align(p, 4, 2, 8, 16, p, p, p, p, p, ws - 1, None) == native.MOE_ERR_WORKSPACE
+
+
+def test_align_noalloc_limits(native):
+    """The allocation-free alignment call has a fixed 131072-int scratch array: one histogram
+    of E experts per 512-pair chunk, so ceil(T*k/512) * E may not exceed it."""
+    L = native.lib
+    p = ctypes.c_void_p(1 << 20)
+    # at the limit the arguments pass (the call then fails only for want of a GPU here)
+    T, k, E = 65536, 1, 1024  # 128 chunks x 1024 experts = 131072
+    at_limit = L.moe_align_noalloc(p, T, k, E, 16, p, p, p, p, None)
+    assert at_limit not in (native.MOE_ERR_UNSUPPORTED, native.MOE_ERR_INVALID_ARG)
+    assert L.moe_align_noalloc(p, T + 1, k, E, 16, p, p, p, p, None) == native.MOE_ERR_UNSUPPORTED
+    assert L.moe_align_noalloc(p, 0, 2, 8, 16, p, p, p, p, None) == native.MOE_ERR_UNSUPPORTED
+    assert L.moe_align_noalloc(p, 4, 2, 8, 0, p, p, p, p, None) == native.MOE_ERR_UNSUPPORTED
+    assert L.moe_align_noalloc(ctypes.c_void_p((1 << 20) + 2), 4, 2, 8, 16, p, p, p, p, None) == \
+        native.MOE_ERR_INVALID_ARG
