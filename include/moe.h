@@ -93,12 +93,13 @@ moe_status_t moe_align(const int32_t* topk_ids, int T, int k, int E, int align, 
  * describing the method have no counterpart of this call; it exists for those callers.
  * The scratch lives in a fixed 512 KiB array inside the library (131072 int32, kept on every
  * GPU that loads the library until the process exits); a call needs ceil(T*k/512)*E of them and
- * returns MOE_ERR_UNSUPPORTED when that is more.  It allocates nothing.  The first call on a
- * device looks up the array's device address (cudaGetSymbolAddress) and caches it: make that
- * first call before any stream capture.  Every call reuses the same array and overwrites each
- * entry it reads, so earlier contents never leak into a result; calls that overlap on the GPU
- * race on the array and must be serialised by the caller.  Arguments and outputs otherwise as
- * moe_align. */
+ * returns MOE_ERR_UNSUPPORTED when that is more.  It allocates nothing.  Each call outside stream
+ * capture looks up the array's device address on the current device (cudaGetSymbolAddress, no
+ * allocation) and remembers it; a call on a stream that is being captured uses the remembered
+ * address, so make the first call on each device before any stream capture.  Every call
+ * reuses the same array and overwrites each entry it reads, so earlier contents never leak
+ * into a result; calls that overlap on the GPU race on the array and must be serialised by the
+ * caller.  Arguments and outputs otherwise as moe_align. */
 moe_status_t moe_align_noalloc(const int32_t* topk_ids, int T, int k, int E, int align, int32_t* expert_counts,
                                int32_t* expert_offsets, int32_t* sorted_ids, int32_t* inv_pos, cudaStream_t stream);
 

@@ -11,9 +11,13 @@
 // MOE_ERR_UNSUPPORTED.
 //
 // Host code cannot pass the array's name to a kernel: on the host that name is only a
-// stand-in, not a device address.  The first call on each device looks up the array's device
-// address there with cudaGetSymbolAddress and caches it; make that first call before any
-// stream capture.  All calls share the one array.  Each call overwrites every scratch entry it
+// stand-in, not a device address.  Each call looks up the array's device address on the
+// current device with cudaGetSymbolAddress (a lookup, no allocation) and remembers it per
+// device; a call made while its stream is being captured into a CUDA graph uses the remembered
+// address instead, so make the first call on each device before any stream capture.  Looking
+// the address up again on every uncaptured call keeps it right after cudaDeviceReset, which
+// reloads the library's device code, possibly at another address.  All calls share the one
+// array.  Each call overwrites every scratch entry it
 // reads, so leftovers from an earlier call never matter, but calls that overlap on the GPU
 // (different streams, or several host threads) race on the array and must be serialised by
 // the caller.
@@ -29,13 +33,16 @@ constexpr size_t kNoAllocScratchInts = 131072;  // 512 KiB
 static __device__ __align__(256) int32_t g_align_scratch[kNoAllocScratchInts];
 
 std::mutex g_scratch_mu;
-int32_t* g_scratch_addr[64];  // per device, filled by the first call on that device
 
-moe_status_t scratch_for_current_device(int32_t** out) {
+int32_t* g_scratch_addr[64];  // per device: the address the last uncaptured call looked up
+
+moe_status_t scratch_for_current_device(cudaStream_t stream, int32_t** out) {
   int d = 0;
   if (cudaGetDevice(&d) != cudaSuccess || d < 0 || d >= 64) return MOE_ERR_CUDA;
+  cudaStreamCaptureStatus cs = cudaStreamCaptureStatusNone;
+  if (cudaStreamIsCapturing(stream, &cs) != cudaSuccess) return MOE_ERR_CUDA;
   std::lock_guard<std::mutex> lk(g_scratch_mu);
-  if (g_scratch_addr[d] == nullptr) {
+  if (cs == cudaStreamCaptureStatusNone || g_scratch_addr[d] == nullptr) {
     void* p = nullptr;
     if (cudaGetSymbolAddress(&p, g_align_scratch) != cudaSuccess || p == nullptr) return MOE_ERR_CUDA;
     g_scratch_addr[d] = static_cast<int32_t*>(p);
@@ -59,7 +66,7 @@ extern "C" moe_status_t moe_align_noalloc(const int32_t* topk_ids, int T, int k,
     return MOE_ERR_INVALID_ARG;
   if (moe_status_t st = check_device()) return st;
   int32_t* scratch = nullptr;
-  if (moe_status_t st = scratch_for_current_device(&scratch)) return st;
+  if (moe_status_t st = scratch_for_current_device(stream, &scratch)) return st;
   const cudaError_t e = launch_align(topk_ids, T, k, E, align, expert_counts, expert_offsets, sorted_ids, inv_pos,
                                      scratch, 256, nullptr, nullptr, stream);
   return e == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;

@@ -426,7 +426,7 @@ moe_status_t moe_w4a16_gemm(const void* a, int a_is_bf16, const int32_t* w_q, co
                     out_fp32 ? OUT_F32 : OUT_BF16, out, nullptr, N, sp, w.part};
       e = launch_w4i8_gemm(g, stream);
     }
-    if (e == cudaSuccess && sp > 1) e = launch_reduce_splits(w.part, sp, M, N, expert_offsets, E, out, out_fp32, stream);
+    if (e == cudaSuccess && sp > 1) e = launch_reduce_splits(w.part, sp, M, N, expert_offsets, w.row_count, E, out, out_fp32, stream);
     return e == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
   }
   if (e == cudaSuccess) e = launch_convert_rows(static_cast<const uint16_t*>(a), a_is_bf16, M, K, w.a, stream);
@@ -436,7 +436,7 @@ moe_status_t moe_w4a16_gemm(const void* a, int a_is_bf16, const int32_t* w_q, co
                     out_fp32 ? OUT_F32 : OUT_BF16, sp, w.part};
     e = launch_w4a16_gemm(g, stream);
   }
-  if (e == cudaSuccess && sp > 1) e = launch_reduce_splits(w.part, sp, M, N, expert_offsets, E, out, out_fp32, stream);
+  if (e == cudaSuccess && sp > 1) e = launch_reduce_splits(w.part, sp, M, N, expert_offsets, w.row_count, E, out, out_fp32, stream);
   return e == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
 }
 

@@ -94,10 +94,10 @@ struct W4I8Problem {
 };
 constexpr int kI8TileRows = 8;  // token rows per tile of the int8 GEMM
 cudaError_t launch_w4i8_gemm(const W4I8Problem& p, cudaStream_t s);
-// out[r][n] = sum over s = 0..splits-1 (in that order) of part[s][r][n] for rows
-// r in [offsets[0], offsets[E]), stored as fp32 (out_fp32) or bf16 (RNE)
-cudaError_t launch_reduce_splits(const float* part, int splits, int rows, int N, const int32_t* offsets, int E,
-                                 void* out, int out_fp32, cudaStream_t s);
+// out[r][n] = sum over s = 0..splits-1 (in that order) of part[s][r][n] for the rows of every
+// expert e, [row_start[e], row_start[e] + row_count[e]), stored as fp32 (out_fp32) or bf16 (RNE)
+cudaError_t launch_reduce_splits(const float* part, int splits, int rows, int N, const int32_t* row_start,
+                                 const int32_t* row_count, int E, void* out, int out_fp32, cudaStream_t s);
 // Planes of the K-vectors x_src: plane row r takes source row r (inv_pos == null, k == 1),
 // or for every pair p plane row inv_pos[p] takes source row p / k.
 cudaError_t launch_planes(const uint16_t* a, int a_is_bf16, const int32_t* inv_pos, int n_pairs, int k, int K,

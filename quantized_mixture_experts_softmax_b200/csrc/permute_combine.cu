@@ -163,16 +163,21 @@ cudaError_t launch_planes(const uint16_t* a, int a_is_bf16, const int32_t* inv_p
   return cudaGetLastError();
 }
 
-// Split-K reduction: out[r][n] = sum_s part[s][r][n] in split order (deterministic), for the
-// rows the expert ranges cover; one thread per 4 outputs.
+// Split-K reduction: out[r][n] = sum_s part[s][r][n] in split order (deterministic).  Block row
+// blockIdx.y = expert e reduces the rows [row_start[e], row_start[e] + row_count[e]); the
+// scheduler sets row_count to 0 for an expert whose offsets failed its check, and the GEMM then
+// wrote no partial sums for it, so such rows are left untouched (never filled from unwritten
+// workspace).  One thread per 4 outputs, grid-stride over the expert's rows.
 __global__ void __launch_bounds__(256) reduce_splits_kernel(const float4* __restrict__ part, int splits, int rows,
-                                                            int N, const int32_t* __restrict__ offsets, int E,
+                                                            int N, const int32_t* __restrict__ row_start,
+                                                            const int32_t* __restrict__ row_count,
                                                             void* __restrict__ out, int out_fp32) {
-  const int r0 = __ldg(offsets), r1 = __ldg(offsets + E);
+  const int e = blockIdx.y;
+  const int cnt = __ldg(row_count + e);
+  if (cnt <= 0) return;
   const size_t n4 = (size_t)N / 4, plane = (size_t)rows * n4;
-  for (size_t i = (size_t)blockIdx.x * blockDim.x + threadIdx.x; i < plane; i += (size_t)gridDim.x * blockDim.x) {
-    const int r = (int)(i / n4);
-    if (r < r0 || r >= r1) continue;
+  const size_t i0 = (size_t)__ldg(row_start + e) * n4, i1 = i0 + (size_t)cnt * n4;
+  for (size_t i = i0 + (size_t)blockIdx.x * blockDim.x + threadIdx.x; i < i1; i += (size_t)gridDim.x * blockDim.x) {
     float4 acc = __ldg(part + i);
     for (int sp = 1; sp < splits; ++sp) {
       const float4 v = __ldg(part + (size_t)sp * plane + i);
@@ -191,14 +196,15 @@ __global__ void __launch_bounds__(256) reduce_splits_kernel(const float4* __rest
   }
 }
 
-cudaError_t launch_reduce_splits(const float* part, int splits, int rows, int N, const int32_t* offsets, int E,
-                                 void* out, int out_fp32, cudaStream_t s) {
-  const size_t n = (size_t)rows * (N / 4);
-  const size_t want = (n + 255) / 256;
-  const unsigned blocks = (unsigned)(want < 148 * 8 ? want : 148 * 8);
+cudaError_t launch_reduce_splits(const float* part, int splits, int rows, int N, const int32_t* row_start,
+                                 const int32_t* row_count, int E, void* out, int out_fp32, cudaStream_t s) {
+  // about 8 blocks of 256 threads per SM in total, at least one per expert
+  const size_t want = ((size_t)rows * (N / 4) + 255) / 256;
+  const size_t cap = (size_t)sm_count() * 8;
+  const unsigned bx = (unsigned)std::max<size_t>(1, std::min(want, cap) / (size_t)E);
   timing_before("reduce_splits", s);
-  reduce_splits_kernel<<<blocks, 256, 0, s>>>(reinterpret_cast<const float4*>(part), splits, rows, N, offsets, E, out,
-                                              out_fp32);
+  reduce_splits_kernel<<<dim3(bx, (unsigned)E), 256, 0, s>>>(reinterpret_cast<const float4*>(part), splits, rows, N,
+                                                              row_start, row_count, out, out_fp32);
   timing_after("reduce_splits", s);
   return cudaGetLastError();
 }

@@ -4,7 +4,9 @@ import numpy as np
 import pytest
 import torch
 
-from helpers import dev
+import oracle
+import synth
+from helpers import check_tol, dev
 
 pytestmark = pytest.mark.gpu
 moe = pytest.importorskip("quantized_mixture_experts_softmax_b200")
@@ -31,3 +33,23 @@ def test_bad_offsets_in_grouped_gemm_are_flagged_not_used():
     moe.moe_get_device_status()
     moe.moe_w4a16_gemm(a, w_q, w_s, off, out_fp32=True)
     assert moe.moe_get_device_status() == moe.MOE_ERR_DEVICE_CHECK
+
+
+def test_bad_offsets_with_k_splits_leave_the_flagged_rows_untouched():
+    """M=2 rows against [7168 x 512] weights has 4 work items, so the K range is split and the
+    fp32 partial sums are reduced by a second kernel.  Expert 1's range reaches past M: it is
+    flagged and skipped, so its row must keep what the caller put there (the reduction must not
+    fill it from partial sums nobody wrote), while expert 0's row is computed normally."""
+    M, K, N = 2, 7168, 512
+    a, w_q, w_s = synth.gemm_operands(5, M, K, N)
+    w_q2, w_s2 = np.concatenate([w_q, w_q]), np.concatenate([w_s, w_s])
+    off = np.array([0, 1, 5], np.int32)
+    out = torch.full((M, N), 7.0, dtype=torch.float32, device="cuda")
+    moe.moe_get_device_status()
+    moe.moe_w4a16_gemm(dev(a, torch.bfloat16), dev(w_q2), dev(w_s2, torch.bfloat16), dev(off), out=out,
+                       out_fp32=True)
+    assert moe.moe_get_device_status() == moe.MOE_ERR_DEVICE_CHECK
+    got = out.cpu().numpy()
+    assert np.all(got[1] == 7.0)
+    ref = oracle.w4a16_gemm(a[:1], True, w_q, w_s, np.array([0, 1], np.int32))
+    check_tol(got[:1], ref, what="expert 0 row")
