@@ -168,6 +168,19 @@ typedef struct {
 size_t moe_blockfp8_workspace_size(int T, int H, int I, int E, int k);
 moe_status_t moe_blockfp8_forward(const moe_blockfp8_args* args, void* ws, size_t ws_bytes, cudaStream_t stream);
 
+/* Diagnostic view of the block-FP8 layer's requantized intermediate: given the workspace `ws`
+ * of a moe_blockfp8_forward call with the same (T, H, I, E, k), returns device pointers into
+ * it (nothing is enqueued or read):
+ *   inv_pos    int32 [T*k]          row r of pair p = t*k + s (as moe_align's inv_pos)
+ *   h          e4m3  [T*k, I]       row r = the e4m3 codes of the pair's requantized h
+ *   h_scale_t  fp32  [I/128, T*k]   h_scale_t[g][r] = the scale of row r's 128-column group g
+ * so that h of pair p, column j, is e4m3(h[r][j]) * h_scale_t[j/128][r] with r = inv_pos[p].
+ * The contents are valid once that call's work on its stream has completed and until the next
+ * call that uses the workspace.  Shape errors MOE_ERR_UNSUPPORTED, a null or misaligned
+ * argument MOE_ERR_INVALID_ARG. */
+moe_status_t moe_blockfp8_intermediate(const void* ws, int T, int H, int I, int E, int k, const int32_t** inv_pos,
+                                       const uint8_t** h, const float** h_scale_t);
+
 /* ------------------------------------------------------------------ grouped W4A16 GEMM
  * No activation: rows [expert_offsets[e], expert_offsets[e+1]) of a are multiplied by
  * expert e's dequantized weights:  out[m][n] = sum_c a[m][c] * W[e][n][c].

@@ -17,7 +17,7 @@ from ._native import (MOE_ERR_CUDA, MOE_ERR_DEVICE_CHECK, MOE_ERR_INVALID_ARG, M
                       MOE_ERR_UNSUPPORTED, MOE_ERR_WORKSPACE, MOE_OK, BlockFP8Args, MoeError, W4A16Args, check,
                       lib)
 
-__all__ = ["moe_route", "moe_align", "moe_align_capacity", "moe_w4a16_forward", "moe_w4a16_workspace_size",
+__all__ = ["moe_route", "moe_blockfp8_intermediate", "moe_align", "moe_align_capacity", "moe_w4a16_forward", "moe_w4a16_workspace_size",
            "moe_blockfp8_forward", "moe_blockfp8_workspace_size", "moe_w4a16_gemm", "moe_w4a16_gemm_workspace_size",
            "moe_get_device_status", "moe_debug_wait_timeout", "moe_timing_enable", "moe_timing_read", "MoeError",
            "lib"]
@@ -123,6 +123,25 @@ def moe_blockfp8_forward(x, xs, topk_ids, topk_w, w13, w13_s, w2, w2_s, out=None
     check(lib.moe_blockfp8_forward(ctypes.byref(args), _p(ws), ws.numel() * ws.element_size(), _stream(stream)),
           "moe_blockfp8_forward")
     return out
+
+
+def moe_blockfp8_intermediate(workspace: torch.Tensor, T: int, H: int, I: int, E: int, k: int) -> dict:
+    """Views into the workspace of a finished moe_blockfp8_forward(T, H, I, E, k) call:
+    inv_pos int32 [T*k], h e4m3 codes uint8 [T*k, I], h_scale_t fp32 [I/128, T*k]."""
+    _cuda(workspace)
+    ptrs = [ctypes.c_void_p() for _ in range(3)]
+    check(lib.moe_blockfp8_intermediate(_p(workspace), T, H, I, E, k, *[ctypes.byref(q) for q in ptrs]),
+          "moe_blockfp8_intermediate")
+    raw = workspace.view(torch.uint8).reshape(-1)
+    base = raw.data_ptr()
+
+    def view(ptr, n, dtype):
+        off = ptr.value - base
+        return raw[off: off + n * torch.empty((), dtype=dtype).element_size()].view(dtype)
+
+    P = T * k
+    return dict(inv_pos=view(ptrs[0], P, torch.int32), h=view(ptrs[1], P * I, torch.uint8).view(P, I),
+                h_scale_t=view(ptrs[2], (I // 128) * P, torch.float32).view(I // 128, P))
 
 
 def moe_w4a16_gemm_workspace_size(M: int, K: int, N: int, E: int) -> int:

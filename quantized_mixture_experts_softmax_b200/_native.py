@@ -21,7 +21,7 @@ EXPORTS = [
     "moe_status_string", "moe_route", "moe_align_capacity", "moe_align_workspace_size", "moe_align",
     "moe_w4a16_workspace_size", "moe_w4a16_forward", "moe_blockfp8_workspace_size", "moe_blockfp8_forward",
     "moe_w4a16_gemm_workspace_size", "moe_w4a16_gemm", "moe_get_device_status", "moe_debug_wait_timeout",
-    "moe_timing_enable", "moe_timing_read", "moe_align_noalloc",
+    "moe_timing_enable", "moe_timing_read", "moe_align_noalloc", "moe_blockfp8_intermediate",
 ]
 
 
@@ -72,6 +72,9 @@ def _load():
     L.moe_blockfp8_workspace_size.argtypes = [i32, i32, i32, i32, i32]
     L.moe_blockfp8_forward.restype = i32
     L.moe_blockfp8_forward.argtypes = [ctypes.POINTER(BlockFP8Args), vp, sz, vp]
+    L.moe_blockfp8_intermediate.restype = i32
+    L.moe_blockfp8_intermediate.argtypes = [vp, i32, i32, i32, i32, i32, ctypes.POINTER(vp), ctypes.POINTER(vp),
+                                            ctypes.POINTER(vp)]
     L.moe_w4a16_gemm_workspace_size.restype = sz
     L.moe_w4a16_gemm_workspace_size.argtypes = [i32, i32, i32, i32]
     L.moe_w4a16_gemm.restype = i32

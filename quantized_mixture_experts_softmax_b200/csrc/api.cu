@@ -398,6 +398,17 @@ moe_status_t moe_blockfp8_forward(const moe_blockfp8_args* a, void* ws, size_t w
   return e == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
 }
 
+moe_status_t moe_blockfp8_intermediate(const void* ws, int T, int H, int I, int E, int k, const int32_t** inv_pos,
+                                       const uint8_t** h, const float** h_scale_t) {
+  if (!shape_ok(T, H, I, E, k)) return MOE_ERR_UNSUPPORTED;
+  if (!aligned(ws, 256) || !inv_pos || !h || !h_scale_t) return MOE_ERR_INVALID_ARG;
+  const F8Ws w = carve_fp8_forward(const_cast<void*>(ws), T, H, I, E, k);
+  *inv_pos = w.inv;
+  *h = w.h;
+  *h_scale_t = w.hs_t;
+  return MOE_OK;
+}
+
 size_t moe_w4a16_gemm_workspace_size(int M, int K, int N, int E) {
   if (M < 1 || K < 128 || N < 128 || K % 128 || N % 128 || E < 1 || E > 1024) return 0;
   return carve_gemm(nullptr, M, K, N, E).bytes;

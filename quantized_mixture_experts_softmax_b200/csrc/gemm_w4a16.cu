@@ -341,13 +341,17 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int nv = min(16, I.nvalid - c0);
         if (GATED) {
           __half* out = reinterpret_cast<__half*>(p.out) + (size_t)(I.r0 + c0) * p.out_ld + interleave_pos(col);
+          bool big = false;  // an h the fp16 operand of the down projection cannot hold
 #pragma unroll
           for (int i = 0; i < 16; ++i) {
             if (i < nv) {
               const float gv = __uint_as_float(g[i]), uv = __uint_as_float(u[i]);
-              out[(size_t)i * p.out_ld] = __float2half_rn(gv / (1.0f + __expf(-gv)) * uv);
+              const float hv = gv / (1.0f + __expf(-gv)) * uv;
+              big |= !(fabsf(hv) < 65520.0f);
+              out[(size_t)i * p.out_ld] = __float2half_rn(hv);
             }
           }
+          if (big) set_status(MOE_ERR_DEVICE_CHECK);
         } else if (p.splits > 1) {  // this split's partial sum, reduced in split order by another kernel
           float* out = p.part + (size_t)(it % p.splits) * p.act_rows * p.out_ld + (size_t)(I.r0 + c0) * p.out_ld + col;
 #pragma unroll

@@ -33,7 +33,27 @@ __device__ __forceinline__ uint4 f16x8_interleave(uint4 v) {
   return make_uint4(a, b, c, d);
 }
 
-// one warp per (token, slot) pair: x_perm[inv_pos[p]] = interleave(fp16(x[p / k]))
+// True when one of the 8 bf16 values is outside the finite fp16 range: |x| >= 65536 (the
+// smallest bf16 magnitude above 65504 the cast would turn into infinity), infinite or NaN.
+__device__ __forceinline__ bool bf16x8_beyond_f16(const uint4& v) {
+  const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+  bool bad = false;
+#pragma unroll
+  for (int j = 0; j < 4; ++j) bad |= (w[j] & 0x7FFFu) >= 0x4780u || ((w[j] >> 16) & 0x7FFFu) >= 0x4780u;
+  return bad;
+}
+// True when one of the 8 fp16 values is infinite or NaN.
+__device__ __forceinline__ bool f16x8_nonfinite(const uint4& v) {
+  const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+  bool bad = false;
+#pragma unroll
+  for (int j = 0; j < 4; ++j) bad |= (w[j] & 0x7C00u) == 0x7C00u || (w[j] & 0x7C000000u) == 0x7C000000u;
+  return bad;
+}
+
+// one warp per (token, slot) pair: x_perm[inv_pos[p]] = interleave(fp16(x[p / k])).  A row with
+// a value the fp16 operand cannot hold is still converted (to +-inf) and recorded as
+// MOE_ERR_DEVICE_CHECK.
 __global__ void __launch_bounds__(256) permute_w4_kernel(const uint4* __restrict__ x, const int32_t* __restrict__ inv_pos,
                                                          int P, int k, int H8, uint4* __restrict__ x_perm) {
   const int p = (int)((blockIdx.x * blockDim.x + threadIdx.x) >> 5);
@@ -43,7 +63,13 @@ __global__ void __launch_bounds__(256) permute_w4_kernel(const uint4* __restrict
   if (r < 0) return;
   const uint4* src = x + (size_t)(p / k) * H8;
   uint4* dst = x_perm + (size_t)r * H8;
-  for (int c = lane; c < H8; c += 32) dst[c] = bf16x8_to_f16x8_interleaved(__ldg(src + c));
+  bool bad = false;
+  for (int c = lane; c < H8; c += 32) {
+    const uint4 v = __ldg(src + c);
+    bad |= bf16x8_beyond_f16(v);
+    dst[c] = bf16x8_to_f16x8_interleaved(v);
+  }
+  if (__any_sync(0xffffffffu, bad) && lane == 0) set_status(MOE_ERR_DEVICE_CHECK);
 }
 
 cudaError_t launch_permute_w4(const uint16_t* x_bf16, const int32_t* inv_pos, int T, int k, int H, __half* x_perm,
@@ -124,6 +150,7 @@ __global__ void __launch_bounds__(256) planes_kernel(const uint4* __restrict__ a
   }
 #pragma unroll
   for (int off = 8; off; off >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, off));  // 16 lanes
+  if (!(amax <= 3.402823466e38f) && i == 0) set_status(MOE_ERR_DEVICE_CHECK);  // an inf or NaN input
   const float sc = fmaxf(amax, 1e-30f) * (1.0f / kFixMax);
   int X[8], sum = 0;
 #pragma unroll
@@ -209,12 +236,17 @@ cudaError_t launch_reduce_splits(const float* part, int splits, int rows, int N,
   return cudaGetLastError();
 }
 
+// rows of the single grouped GEMM's activations -> interleaved fp16; a value outside the finite
+// fp16 range (or a non-finite fp16 input) is recorded as MOE_ERR_DEVICE_CHECK
 __global__ void __launch_bounds__(256) convert_rows_kernel(const uint4* __restrict__ a, int a_is_bf16, size_t n8,
                                                            uint4* __restrict__ out) {
+  bool bad = false;
   for (size_t i = blockIdx.x * (size_t)blockDim.x + threadIdx.x; i < n8; i += (size_t)gridDim.x * blockDim.x) {
     const uint4 v = __ldg(a + i);
+    bad |= a_is_bf16 ? bf16x8_beyond_f16(v) : f16x8_nonfinite(v);
     out[i] = a_is_bf16 ? bf16x8_to_f16x8_interleaved(v) : f16x8_interleave(v);
   }
+  if (bad) set_status(MOE_ERR_DEVICE_CHECK);
 }
 
 cudaError_t launch_convert_rows(const uint16_t* a, int a_is_bf16, int M, int K, __half* out, cudaStream_t s) {
