@@ -42,6 +42,11 @@ WORKLOADS = {
 for _t in (1, 16, 64, 512, 4096):  # block-FP8 layer, 256 experts
     WORKLOADS[f"fp8_t{_t}"] = dict(kind="fp8", T=_t, zipf=0.0, steps=200 if _t <= 512 else 60, warmup=10)
 FP8_MODEL = dict(H=7168, I=2048, E=256, k=8)
+# block-FP8 benchmark model: expert e holds the generated weights of expert e mod FP8_DISTINCT (each
+# expert in its own memory); generating 11.3 GB of normal e4m3 values on the host takes minutes
+FP8_DISTINCT = 16
+FP8_DATA = (f"synthetic (seeded counter-based generator; expert e holds the generated weights of expert e mod "
+            f"{FP8_DISTINCT}, each expert in its own memory)")
 # the single-expert grouped-GEMM sweep: [M,7168]x[7168,512] and [M,256]x[256,7168]
 for (_k, _n) in ((7168, 512), (256, 7168)):
     for _m in (1, 64, 512, 4096, 32768):
@@ -197,8 +202,12 @@ def make_model(seed: int):
     return out
 
 
-def make_model_fp8(seed: int):
-    """All 256 block-FP8 experts generated on the host by the seeded generator, copied to HBM."""
+def make_model_fp8(seed: int, distinct: int = 0):
+    """All 256 block-FP8 experts, generated on the host by the seeded generator and copied to
+    HBM.  With distinct > 0 only the first `distinct` experts are generated and expert e holds
+    the weights of expert e mod distinct (every expert still has its own memory, so a step reads
+    the same bytes from HBM; used by the default benchmark run, where generating 11.3 GB of
+    normal e4m3 values on the host would take minutes)."""
     import torch
     import synth
     H, I, E = FP8_MODEL["H"], FP8_MODEL["I"], FP8_MODEL["E"]
@@ -206,19 +215,23 @@ def make_model_fp8(seed: int):
     out = {}
     specs = [("w13", (E, 2 * I, H), torch.uint8, "w13_8"), ("w13_s", (E, 2 * I // 128, H // 128), torch.float32, "w13_8s"),
              ("w2", (E, H, I), torch.uint8, "w2_8"), ("w2_s", (E, H // 128, I // 128), torch.float32, "w2_8s")]
+    gen = E if distinct <= 0 else min(distinct, E)
     for name, shape, dt, tid in specs:
         d = torch.empty(shape, dtype=dt, device="cuda")
         per = int(np.prod(shape[1:]))
         chunk = 16
         stage = torch.empty((chunk, *shape[1:]), dtype=dt, pin_memory=True)
-        for e0 in range(0, E, chunk):
-            n = min(chunk, E - e0)
+        for e0 in range(0, gen, chunk):
+            n = min(chunk, gen - e0)
             buf = stage[:n]
             if dt == torch.uint8:
                 synth.fill_normal_e4m3(seed, synth.TID[tid], e0 * per, buf)
             else:
                 synth.fill_uniform_f32(seed, synth.TID[tid], e0 * per, buf, lo, hi)
             d[e0:e0 + n].copy_(buf)
+        for e0 in range(gen, E, gen):
+            n = min(gen, E - e0)
+            d[e0:e0 + n].copy_(d[:n])
         out[name] = d
     return out
 
@@ -319,11 +332,37 @@ def run_gemm(args, world, rank):
     }
 
 
-def run_ours(args, world, rank):
+def _phase_roofline(kern, suffix, alg_bytes, alg_flops, t_peak, t_peak_src, peaks, traffic):
+    """Roofline of one GEMM phase (gate/up or down): the kernels whose names end with `suffix`
+    (one launch each per step: the int8-MMA kernel for experts with few rows, the fp16 one for
+    the rest), algorithmic bytes / flops of the phase over their summed time per step."""
+    ms = sum(v[0] for n, v in kern.items() if n.endswith(suffix))
+    launches = sum(v[1] for n, v in kern.items() if n.endswith(suffix))
+    names = sorted(n for n in kern if n.endswith(suffix))
+    if not names or ms <= 0:
+        return None
+    steps = max(v[1] for n, v in kern.items() if n.endswith(suffix))
+    per_s = ms / steps / 1e3
+    hbm_bound = (alg_flops / alg_bytes) < (t_peak * 1e3 / peaks["hbm"])
+    common = dict(kernel=" + ".join(names), launches_per_step=launches // steps, launch_ms=round(per_s * 1e3, 4),
+                  traffic=traffic, algorithmic_bytes_per_launch=int(alg_bytes), algorithmic_flops_per_launch=alg_flops)
+    if hbm_bound:
+        ach = alg_bytes / per_s / 1e9
+        return dict(bound="hbm", achieved=round(ach, 1), peak=peaks["hbm"], unit="GB/s",
+                    frac=round(ach / peaks["hbm"], 4), peak_source=peaks["src"] + " (copy, burst)", **common)
+    ach = alg_flops / per_s / 1e12
+    return dict(bound="tensor", achieved=round(ach, 1), peak=t_peak, unit="TFLOP/s", frac=round(ach / t_peak, 4),
+                peak_source=t_peak_src, **common)
+
+
+def measure_layer(args, workload, W, world):
+    """One layer workload on resident weights W: device-timed steps (route + layer, inputs in
+    HBM), CUDA-graph replays, the end-to-end variant with host buffers, per-kernel times and the
+    roofline of each GEMM phase.  Returns (result dict, host inputs for the CPU baseline)."""
     import torch
     import quantized_mixture_experts_softmax_b200 as moe
 
-    wl = WORKLOADS[args.workload]
+    wl = WORKLOADS[workload]
     kind = wl["kind"]
     M = FP8_MODEL if kind == "fp8" else MODEL
     T, H, I, E, k = wl["T"], M["H"], M["I"], M["E"], M["k"]
@@ -331,7 +370,6 @@ def run_ours(args, world, rank):
     warmup = args.warmup if args.warmup is not None else wl["warmup"]
     warmup = max(3, warmup)
     seed = 0
-    W = make_model_fp8(seed) if kind == "fp8" else make_model(seed)
     x_h, lg_h = make_inputs(seed, T, wl["zipf"], kind)
     lg = torch.from_numpy(lg_h).cuda()
     ids = torch.empty(T, k, dtype=torch.int32, device="cuda")
@@ -462,61 +500,47 @@ def run_ours(args, world, rank):
     barrier(world)
     ms_e2e = max_over_ranks(ev0.elapsed_time(ev1), world) / e2e_steps
 
-    # ---- roofline of the dominant kernel
+    # ---- rooflines.  Algorithmic work: only what the method must move or compute - the active
+    # experts' weights, the layer input x (gate/up) and the layer output (down); the
+    # expert-sorted activation copies and y round trips are overhead, not credit.
     peaks = load_peaks()
     P = T * k
     flops = 6.0 * P * H * I
     if kind == "fp8":
         w13_b = 2 * I * H + (2 * I // 128) * (H // 128) * 4
         w2_b = H * I + (H // 128) * (I // 128) * 4
-        act_in, act_mid, y_b = P * H, P * I, P * H * 4
         x_in = T * H + T * (H // 128) * 4
     else:
         w13_b, w2_b = W13_BYTES_PER_EXPERT, W2_BYTES_PER_EXPERT
-        act_in, act_mid, y_b = P * H * 2, P * I * 2, P * H * 4
         x_in = T * H * 2
-    layer_bytes = active * (w13_b + w2_b) + x_in + T * H * 2 + T * E * 4
-    # tensor peak for the contraction's own operand type: fp16 runs at the measured bf16 rate,
-    # e4m3 at twice it (the nominal dense fp8 : bf16 ratio)
+    out_b = T * H * 2
+    layer_bytes = active * (w13_b + w2_b) + x_in + out_b + T * E * 4
+    # tensor peak for the contraction's own operand type: fp16 and int8 run at the measured bf16
+    # rate, e4m3 at twice it (the nominal dense fp8 : bf16 ratio)
     t_peak = peaks["bf16"] * (2.0 if kind == "fp8" else 1.0)
     t_peak_src = peaks["src"] + (" bf16 GEMM x 2 (nominal fp8:bf16)" if kind == "fp8" else " bf16 GEMM, burst")
-    top = max(kern.items(), key=lambda kv: kv[1][0]) if kern else None
-    # which grouped GEMM runs: the int8-MMA kernel when no expert can get more than 64 rows
     family = "fp8" if kind == "fp8" else ("w4i8" if T <= 64 else "w4a16")
-    roof = None
-    if top is not None:
-        name, (ms_k, n_k) = top
-        per_launch_s = ms_k / n_k / 1e3
-        if name.endswith("gate_up"):
-            alg_bytes = active * w13_b + act_in + act_mid
-            alg_flops = 2.0 * P * H * 2 * I
-        elif name.endswith("down"):
-            alg_bytes = active * w2_b + act_mid + y_b
-            alg_flops = 2.0 * P * I * H
-        else:
-            alg_bytes, alg_flops = None, None
-        hbm_bound = alg_bytes is not None and (alg_flops / alg_bytes) < (t_peak * 1e3 / peaks["hbm"])
-        traffic = None if (args.tokens or args.experts) else load_traffic(args.workload, name, family)
-        if alg_bytes and hbm_bound:
-            ach = alg_bytes / per_launch_s / 1e9
-            roof = dict(kernel=name, bound="hbm", achieved=round(ach, 1), peak=peaks["hbm"], unit="GB/s",
-                        frac=round(ach / peaks["hbm"], 4), traffic=traffic,
-                        peak_source=peaks["src"] + " (copy, burst)",
-                        algorithmic_bytes_per_launch=int(alg_bytes), launch_ms=round(per_launch_s * 1e3, 4))
-        elif alg_flops:
-            ach = alg_flops / per_launch_s / 1e12
-            roof = dict(kernel=name, bound="tensor", achieved=round(ach, 1), peak=t_peak, unit="TFLOP/s",
-                        frac=round(ach / t_peak, 4), traffic=traffic, peak_source=t_peak_src,
-                        algorithmic_flops_per_launch=alg_flops, launch_ms=round(per_launch_s * 1e3, 4))
+    no_traffic = bool(args.tokens or args.experts)
+    phases = {}
+    for suffix, alg_b, alg_f in (("gate_up", active * w13_b + x_in, 2.0 * P * H * 2 * I),
+                                 ("down", active * w2_b + out_b, 2.0 * P * I * H)):
+        names = [n for n in kern if n.endswith(suffix)]
+        traffic = None
+        if len(names) == 1 and not no_traffic:
+            traffic = load_traffic(workload, names[0], family)
+        phases[suffix] = _phase_roofline(kern, suffix, alg_b, alg_f, t_peak, t_peak_src, peaks, traffic)
+    dom = max((v for v in phases.values() if v), key=lambda r: r["launch_ms"], default=None)
     launches = sum(n for (_, n) in kern.values())
     res = {
         "metric": METRIC, "value": round(ms_step * 1e3 / world, 2), "unit": "µs/layer",
         "n_gpus": world, "steps": steps, "warmup": warmup, "ms_per_step": round(ms_step, 4),
         "higher_is_better": False, "scaling": "weak", "vs_baseline": None,
-        "dtype": {"fp8": "e4m3 (fp32 acc)", "w4a16": "w4a16 (fp16 MMA, fp32 acc)",
+        "dtype": {"fp8": "e4m3 (fp32 acc)",
+                  "w4a16": "w4a16: fp16 MMA (fp32 acc) for experts with many rows, int8 MMA on 16-bit "
+                           "fixed-point activations + fp32 promotion for the rest",
                   "w4i8": "w4a16 as int8 MMA (u8 weights x 16-bit fixed-point activations, s32) + fp32 promotion"}[family],
-        "data": "synthetic (seeded counter-based generator; random-init quantized weights)",
-        "config": layer_config(args.workload, kind, T, H, I, E, k, active, world),
+        "data": FP8_DATA if kind == "fp8" else "synthetic (seeded counter-based generator; random-init quantized weights)",
+        "config": layer_config(workload, kind, T, H, I, E, k, active, world),
         "layer": {"us": round(ms_step * 1e3, 2), "tflops": round(flops / (ms_step * 1e-3) / 1e12, 2),
                   "hbm_gbs": round(layer_bytes / (ms_step * 1e-3) / 1e9, 1),
                   "hbm_frac": round(layer_bytes / (ms_step * 1e-3) / 1e9 / peaks["hbm"], 4),
@@ -527,10 +551,53 @@ def run_ours(args, world, rank):
                 "d2h_bytes_per_step": d2h},
         "gpu_launches": launches,
         "graph": graph,
-        "roofline": roof,
+        "roofline": dom,
+        "phases": phases,
         "clocks": clocks,
     }
     return res, (x_h, lg_h, T, kind)
+
+
+def run_ours(args, world, rank):
+    wl = WORKLOADS[args.workload]
+    W = make_model_fp8(0, distinct=FP8_DISTINCT) if wl["kind"] == "fp8" else make_model(0)
+    return measure_layer(args, args.workload, W, world)
+
+
+# the objects the default run adds to the decode line, measured in the same process
+DEFAULT_EXTRAS = ("prefill", "fp8_t64", "fp8_t4096")
+# keys of a workload's result that stay on the top-level line only
+LINE_ONLY = ("metric", "n_gpus", "higher_is_better", "scaling", "vs_baseline", "data")
+
+
+def run_default(args, world, rank):
+    """The default benchmark: the decode T=64 line (its `value` is the headline), with the
+    prefill T=8192 workload on the same resident 384-expert model and the block-FP8 layer at
+    T=64 and T=4096 as nested objects, each measured like the line itself, with its own
+    CPU-oracle baseline on rank 0."""
+    import torch
+    W = make_model(0)
+    res, inp = measure_layer(args, "decode", W, world)
+    results = [(res, inp)]
+    sub, inp_p = measure_layer(args, "prefill", W, world)
+    res["prefill"] = {k_: v for k_, v in sub.items() if k_ not in LINE_ONLY}
+    results.append((res["prefill"], inp_p))
+    del W
+    torch.cuda.empty_cache()
+    if not args.no_fp8:
+        W8 = make_model_fp8(0, distinct=FP8_DISTINCT)
+        for wl in ("fp8_t64", "fp8_t4096"):
+            sub, inp_f = measure_layer(args, wl, W8, world)
+            res[wl] = {k_: v for k_, v in sub.items() if k_ not in LINE_ONLY}
+            results.append((res[wl], inp_f))
+        del W8
+        torch.cuda.empty_cache()
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        for obj, (x_h, lg_h, T, kind) in results:
+            us, sample, cores, _ = oracle_sample_time(x_h, lg_h, T, kind, budget_s=8.0)
+            obj["cpu_baseline"] = {"value": round(us, 1), "unit": "µs/layer", "cores": cores, "kind": "oracle",
+                                   "sample": sample}
+    return res
 
 
 def oracle_sample_time(x_h, lg_h, T, kind="w4a16", budget_s=15.0):
@@ -542,13 +609,16 @@ def oracle_sample_time(x_h, lg_h, T, kind="w4a16", budget_s=15.0):
     ids, w, _ = oracle.route(lg_h, k)
     cores = oracle.nthreads()
 
+    W8 = synth.fp8_weights(0, M["H"], M["I"], range(FP8_DISTINCT)) if kind == "fp8" else None
+
     def run(n):
         tok = np.arange(n, dtype=np.int32)
         used = np.unique(ids[tok])
         remap = {int(e): i for i, e in enumerate(used)}
         ids_l = np.vectorize(lambda e: remap.get(int(e), 0))(ids[tok]).astype(np.int32)
-        if kind == "fp8":
-            Wt = synth.fp8_weights(0, M["H"], M["I"], used)
+        if kind == "fp8":  # the benchmark's model: expert e has the weights of expert e mod FP8_DISTINCT
+            Wt = W8
+            ids_l = (ids[tok] % FP8_DISTINCT).astype(np.int32)
             t0 = time.time()
             oracle.fp8_tokens(x_h[0][tok], x_h[1][tok], ids_l, w[tok], Wt["w13"], Wt["w13_s"], Wt["w2"], Wt["w2_s"])
         else:
@@ -637,7 +707,9 @@ def main():
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=None)
     ap.add_argument("--warmup", type=int, default=None)
-    ap.add_argument("--workload", choices=sorted(WORKLOADS), default="decode")
+    ap.add_argument("--workload", choices=sorted(WORKLOADS), default=None,
+                    help="one workload's line (default: decode, with prefill and block-FP8 objects)")
+    ap.add_argument("--no-fp8", action="store_true", help="default run: leave out the block-FP8 objects")
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--experts", type=int, default=None,
@@ -649,9 +721,10 @@ def main():
         MODEL["E"] = args.experts
         FP8_MODEL["E"] = args.experts
     if args.tokens:
-        WORKLOADS[args.workload] = dict(WORKLOADS[args.workload], T=args.tokens)
+        WORKLOADS[args.workload or "decode"] = dict(WORKLOADS[args.workload or "decode"], T=args.tokens)
 
     if args.impl == "reference":
+        args.workload = args.workload or "decode"
         rank = int(os.environ.get("RANK", "0"))
         if rank != 0:
             return
@@ -659,6 +732,14 @@ def main():
         return
 
     world, rank, _ = dist_init()
+    if args.workload is None:
+        res = run_default(args, world, rank)
+        if rank == 0:
+            print(json.dumps(res), flush=True)
+        if world > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+        return
     if WORKLOADS[args.workload]["kind"] == "gemm":
         res = run_gemm(args, world, rank)
         if rank == 0:

@@ -114,15 +114,20 @@ moe_status_t moe_align_noalloc(const int32_t* topk_ids, int T, int k, int E, int
  *   w13_s  bf16  [E, 2I, H/32] one scale per 32 K elements per output row
  *   w2_q   int32 [E, H, I/8],  w2_s bf16 [E, H, I/32]   (down projection, same packing)
  *   out    bf16  [T, H] (RNE of the fp32 result), or fp32 [T, H] when out_fp32 != 0
- * Numerics, two paths chosen from T:
- *   T <= 64: the INT4 values meet 16-bit fixed-point activations on the int8 tensor cores:
+ * Numerics: each expert runs on one of two GEMMs, chosen per expert from its token count (every
+ * expert on the first when T <= 64; for larger T an expert with at most 16 rows on the first and
+ * one with more on the second):
+ *   int8 GEMM: the INT4 values meet 16-bit fixed-point activations on the int8 tensor cores:
  *     per (row, 128-K block) s = max(|x|max, 1e-30) / 16383 and X = rint(x / s); each 32-K
  *     group's sum of q*X is exact in int32 and is scaled by (weight scale * s) and
  *     accumulated in fp32; h is stored the same way (one scale per token per 128 rows of I).
- *     The only rounding besides fp32 accumulation is X (at most s / 2 per element).
- *   T > 64: activations and dequantized weights are fed to the tensor cores in fp16, which is
+ *     The only rounding besides fp32 accumulation is X (at most s / 2 per element); any finite
+ *     x is taken.
+ *   fp16 GEMM: activations and dequantized weights are fed to the tensor cores in fp16, which is
  *     exact for bf16 x inside the fp16 normal range and for |q*s| inside it (scales in
- *     [2^-14/8... , 65504/8]); accumulation is fp32; h is rounded to fp16.
+ *     [2^-14/8... , 65504/8]); accumulation is fp32; h is rounded to fp16.  An x or an h
+ *     beyond the fp16 range (|v| >= 65520) becomes +-inf there and records
+ *     MOE_ERR_DEVICE_CHECK.
  * The combine sums the k slots in fp32 in slot order, so the result is deterministic run to
  * run.
  * ws: moe_w4a16_workspace_size(T, H, I, E, k) bytes. */

@@ -68,6 +68,6 @@ extern "C" moe_status_t moe_align_noalloc(const int32_t* topk_ids, int T, int k,
   int32_t* scratch = nullptr;
   if (moe_status_t st = scratch_for_current_device(stream, &scratch)) return st;
   const cudaError_t e = launch_align(topk_ids, T, k, E, align, expert_counts, expert_offsets, sorted_ids, inv_pos,
-                                     scratch, 256, nullptr, nullptr, stream);
+                                     scratch, nullptr, stream);
   return e == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
 }

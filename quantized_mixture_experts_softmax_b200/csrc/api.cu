@@ -139,9 +139,22 @@ void timing_after(const char*, cudaStream_t s) {
 
 // ------------------------------------------------------------------ workspace layouts
 namespace {
-// Decode-sized problems (no expert can get more than 64 rows) run on the int8 tensor-core GEMM
-// with activations as 16-bit fixed-point planes; larger ones on the fp16 GEMM.
+// Decode-sized problems (no expert can get more than 64 rows) run entirely on the int8
+// tensor-core GEMM with activations as 16-bit fixed-point planes.
 bool use_i8(int max_rows_per_expert) { return max_rows_per_expert <= 64; }
+
+// Larger layer calls choose per expert, from its actual token count: an expert with at most
+// kThinRows rows runs on the int8 GEMM (8-row token tiles; its cost is streaming the weights
+// plus a promotion step per live token), one with more on the fp16 GEMM (tiles of up to 256
+// rows, where dequantizing a weight tile once serves many tokens, but a tile of few tokens
+// costs as much dequantization as a full one).  Measured on the 384-expert model with skewed
+// routing at T = 128 ... 8192, switch points of 16, 32, 48 and 64 rows: 16 was fastest at
+// every T (T = 8192: 3% faster than 32, 6% faster than the fp16 GEMM alone).
+#ifndef MOE_THIN_ROWS
+#define MOE_THIN_ROWS 16
+#endif
+constexpr int kThinRows = MOE_THIN_ROWS;
+constexpr int kWideTileRows = 256;
 
 // 16-bit fixed-point planes of an activation matrix [rows, K]
 struct Planes {
@@ -156,9 +169,11 @@ Planes take_planes(Carver& c, size_t rows, int K) {
 }
 
 struct FwdWs {
-  int32_t *counts, *offsets, *sorted, *inv, *blockcnt, *tile_prefix, *chunk;
-  __half *x_perm, *h;  // fp16 path
-  Planes xq, hq;       // int8 path
+  int32_t *counts, *offsets, *sorted, *inv, *blockcnt;
+  int32_t *tile_prefix, *chunk, *row_count;                  // fp16 GEMM schedule (wide experts)
+  int32_t *thin_tile_prefix, *thin_chunk, *thin_row_count;   // int8 GEMM schedule
+  __half *x_perm, *h;  // fp16 path rows
+  Planes xq, hq;       // int8 path rows
   float* y;
   size_t bytes;
 };
@@ -171,12 +186,15 @@ FwdWs carve_w4_forward(void* ws, int T, int H, int I, int E, int k) {
   w.sorted = c.take<int32_t>(P);
   w.inv = c.take<int32_t>(P);
   w.blockcnt = c.take<int32_t>((size_t)align_blocks(T, k) * E);
-  w.tile_prefix = c.take<int32_t>(E + 1);
-  w.chunk = c.take<int32_t>(E);
-  if (use_i8(T)) {
-    w.xq = take_planes(c, P, H);
-    w.hq = take_planes(c, P, I);
-  } else {
+  w.thin_tile_prefix = c.take<int32_t>(E + 1);
+  w.thin_chunk = c.take<int32_t>(E);
+  w.xq = take_planes(c, P, H);
+  w.hq = take_planes(c, P, I);
+  if (!use_i8(T)) {  // some experts may have more than kThinRows rows
+    w.tile_prefix = c.take<int32_t>(E + 1);
+    w.chunk = c.take<int32_t>(E);
+    w.row_count = c.take<int32_t>(E);
+    w.thin_row_count = c.take<int32_t>(E);
     w.x_perm = c.take<__half>(P * H);
     w.h = c.take<__half>(P * I);
   }
@@ -245,8 +263,8 @@ F8Ws carve_fp8_forward(void* ws, int T, int H, int I, int E, int k) {
   w.bytes = c.off + 256;
   return w;
 }
-// token-tile height cap of the W4A16 GEMM that runs
-int pick_nmax(int max_rows_per_expert) { return use_i8(max_rows_per_expert) ? kI8TileRows : 256; }
+// token-tile height cap of the single grouped GEMM's kernel
+int pick_nmax(int max_rows_per_expert) { return use_i8(max_rows_per_expert) ? kI8TileRows : kWideTileRows; }
 
 bool shape_ok(int T, int H, int I, int E, int k) {
   if (T < 1 || k < 1 || E < k || E > 1024) return false;
@@ -306,7 +324,7 @@ moe_status_t moe_align(const int32_t* topk_ids, int T, int k, int E, int align, 
   if (ws_bytes < moe_align_workspace_size(T, k, E)) return MOE_ERR_WORKSPACE;
   if (moe_status_t st = check_device()) return st;
   const cudaError_t e = launch_align(topk_ids, T, k, E, align, expert_counts, expert_offsets, sorted_ids, inv_pos,
-                                     static_cast<int32_t*>(ws), 256, nullptr, nullptr, stream);
+                                     static_cast<int32_t*>(ws), nullptr, stream);
   return e == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
 }
 
@@ -326,36 +344,51 @@ moe_status_t moe_w4a16_forward(const moe_w4a16_args* a, void* ws, size_t ws_byte
   if (ws_bytes < moe_w4a16_workspace_size(T, H, I, E, k)) return MOE_ERR_WORKSPACE;
   if (moe_status_t st = check_device()) return st;
   const FwdWs w = carve_w4_forward(ws, T, H, I, E, k);
-  const int nmax = pick_nmax(T);
   const int P = T * k;
-  cudaError_t e = launch_align(a->topk_ids, T, k, E, 1, w.counts, w.offsets, w.sorted, w.inv, w.blockcnt, nmax,
-                               w.tile_prefix, w.chunk, stream);
-  const TileSched sched{w.offsets, w.counts, w.tile_prefix, w.chunk};
-  if (use_i8(T)) {
-    if (e == cudaSuccess)
-      e = launch_planes(static_cast<const uint16_t*>(a->x), 1, w.inv, P, k, H, w.xq.x, w.xq.meta, stream);
-    if (e == cudaSuccess) {
-      W4I8Problem g{a->w13_q, static_cast<const uint16_t*>(a->w13_s), w.xq.x, w.xq.meta, P, H, E, 2 * I, true, I,
-                    sched, OUT_PLANES, w.hq.x, w.hq.meta, I};
-      e = launch_w4i8_gemm(g, stream);
-    }
-    if (e == cudaSuccess) {
-      W4I8Problem g{a->w2_q, static_cast<const uint16_t*>(a->w2_s), w.hq.x, w.hq.meta, P, I, E, H, false, 0, sched,
-                    OUT_F32, w.y, nullptr, H};
-      e = launch_w4i8_gemm(g, stream);
-    }
-    if (e == cudaSuccess) e = launch_combine(w.y, w.inv, a->topk_w, T, k, H, a->out, a->out_fp32, stream);
-    return e == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
+  const bool mixed = !use_i8(T);  // per-expert choice between the two GEMMs
+  SchedOut so;
+  if (mixed) {
+    so.nmax = kWideTileRows;
+    so.tile_prefix = w.tile_prefix;
+    so.chunk = w.chunk;
+    so.row_count = w.row_count;
+    so.thin_rows = kThinRows;
+    so.thin_nmax = kI8TileRows;
+    so.thin_tile_prefix = w.thin_tile_prefix;
+    so.thin_chunk = w.thin_chunk;
+    so.thin_row_count = w.thin_row_count;
+  } else {  // every expert on the int8 GEMM: its schedule is the main one, row counts = counts
+    so.nmax = kI8TileRows;
+    so.tile_prefix = w.thin_tile_prefix;
+    so.chunk = w.thin_chunk;
   }
-  if (e == cudaSuccess) e = launch_permute_w4(static_cast<const uint16_t*>(a->x), w.inv, T, k, H, w.x_perm, stream);
+  cudaError_t e = launch_align(a->topk_ids, T, k, E, 1, w.counts, w.offsets, w.sorted, w.inv, w.blockcnt, &so, stream);
+  const TileSched thin{w.offsets, mixed ? w.thin_row_count : w.counts, w.thin_tile_prefix, w.thin_chunk};
+  const TileSched wide{w.offsets, w.row_count, w.tile_prefix, w.chunk};
+  const uint16_t* x = static_cast<const uint16_t*>(a->x);
+  const uint16_t* w13_s = static_cast<const uint16_t*>(a->w13_s);
+  const uint16_t* w2_s = static_cast<const uint16_t*>(a->w2_s);
+  // activations of each class of experts in the form its GEMM reads
+  if (e == cudaSuccess)
+    e = launch_planes(x, 1, w.inv, mixed ? a->topk_ids : nullptr, mixed ? w.thin_row_count : nullptr, P, k, H, w.xq.x,
+                      w.xq.meta, stream);
+  if (e == cudaSuccess && mixed) e = launch_permute_w4(x, w.inv, a->topk_ids, w.row_count, T, k, H, w.x_perm, stream);
+  // gate/up with SiLU*up, then down, each on both GEMMs (an empty schedule makes a kernel exit)
   if (e == cudaSuccess) {
-    W4GemmProblem g{a->w13_q, static_cast<const uint16_t*>(a->w13_s), w.x_perm, P, H, E, 2 * I, true, I, sched, nmax,
-                    w.h, I, OUT_H_F16_INTERLEAVED};
+    W4I8Problem g{a->w13_q, w13_s, w.xq.x, w.xq.meta, P, H, E, 2 * I, true, I, thin, OUT_PLANES, w.hq.x, w.hq.meta, I};
+    e = launch_w4i8_gemm(g, stream);
+  }
+  if (e == cudaSuccess && mixed) {
+    W4GemmProblem g{a->w13_q, w13_s, w.x_perm, P, H, E, 2 * I, true, I, wide, kWideTileRows, w.h, I,
+                    OUT_H_F16_INTERLEAVED};
     e = launch_w4a16_gemm(g, stream);
   }
   if (e == cudaSuccess) {
-    W4GemmProblem g{a->w2_q, static_cast<const uint16_t*>(a->w2_s), w.h, P, I, E, H, false, 0, sched, nmax, w.y, H,
-                    OUT_F32};
+    W4I8Problem g{a->w2_q, w2_s, w.hq.x, w.hq.meta, P, I, E, H, false, 0, thin, OUT_F32, w.y, nullptr, H};
+    e = launch_w4i8_gemm(g, stream);
+  }
+  if (e == cudaSuccess && mixed) {
+    W4GemmProblem g{a->w2_q, w2_s, w.h, P, I, E, H, false, 0, wide, kWideTileRows, w.y, H, OUT_F32};
     e = launch_w4a16_gemm(g, stream);
   }
   if (e == cudaSuccess) e = launch_combine(w.y, w.inv, a->topk_w, T, k, H, a->out, a->out_fp32, stream);
@@ -382,8 +415,11 @@ moe_status_t moe_blockfp8_forward(const moe_blockfp8_args* a, void* ws, size_t w
   // token tile of the FP8 GEMM: 64 rows once experts can get that many tokens (halves the
   // weight re-reads and doubles the tokens per MMA), else 32 (a deeper copy pipeline)
   const int nmax = T > 512 ? 64 : 32;
-  cudaError_t e = launch_align(a->topk_ids, T, k, E, 1, w.counts, w.offsets, w.sorted, w.inv, w.blockcnt, nmax,
-                               w.tile_prefix, w.chunk, stream);
+  SchedOut so;
+  so.nmax = nmax;
+  so.tile_prefix = w.tile_prefix;
+  so.chunk = w.chunk;
+  cudaError_t e = launch_align(a->topk_ids, T, k, E, 1, w.counts, w.offsets, w.sorted, w.inv, w.blockcnt, &so, stream);
   if (e == cudaSuccess) e = launch_permute_fp8(a->x, a->xs, w.inv, T, k, H, w.x_perm, w.xs_t, P, stream);
   const TileSched sched{w.offsets, w.counts, w.tile_prefix, w.chunk};
   if (e == cudaSuccess) {
@@ -430,7 +466,8 @@ moe_status_t moe_w4a16_gemm(const void* a, int a_is_bf16, const int32_t* w_q, co
   const TileSched sched{expert_offsets, w.row_count, w.tile_prefix, w.chunk};
   if (use_i8(M)) {
     if (e == cudaSuccess)
-      e = launch_planes(static_cast<const uint16_t*>(a), a_is_bf16, nullptr, M, 1, K, w.aq.x, w.aq.meta, stream);
+      e = launch_planes(static_cast<const uint16_t*>(a), a_is_bf16, nullptr, nullptr, nullptr, M, 1, K, w.aq.x,
+                        w.aq.meta, stream);
     const int sp = gemm_splits(M, K, N);
     if (e == cudaSuccess) {
       W4I8Problem g{w_q, static_cast<const uint16_t*>(w_s), w.aq.x, w.aq.meta, M, K, E, N, false, 0, sched,

@@ -721,7 +721,7 @@ cudaError_t launch_t(const W4I8Problem& pr, cudaStream_t s) {
   auto kern = w4i8_gemm_kernel<GATED>;
   cudaError_t err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (err != cudaSuccess) return err;
-  const char* name = GATED ? "w4a16_gemm_gate_up" : "w4a16_gemm_down";
+  const char* name = GATED ? "w4i8_gemm_gate_up" : "w4i8_gemm_down";
   timing_before(name, s);
   kern<<<sm_count(), kThreads, smem, s>>>(tm_w, tm_x, tm_m, tm_s, p);
   timing_after(name, s);

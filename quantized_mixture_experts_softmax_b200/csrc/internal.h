@@ -27,17 +27,35 @@ struct TileSched {
 cudaError_t launch_route(const float* logits, int T, int E, int k, int renormalize, int32_t* ids, float* w,
                          cudaStream_t s);
 int align_blocks(int T, int k);
-// blockcnt: [align_blocks * E] int32 scratch.  tile_prefix/chunk may be null (no scheduler).
+// Token-tile schedules the alignment builds from each expert's count.  The main schedule cuts
+// an expert's rows into balanced tiles of at most nmax rows.  With thin_tile_prefix given, an
+// expert with at most thin_rows rows goes to the thin schedule instead (tiles of at most
+// thin_nmax rows), and each schedule's row_count holds the expert's rows in that schedule (0 in
+// the other).
+struct SchedOut {
+  int nmax = 0;
+  int32_t* tile_prefix = nullptr;  // [E+1]
+  int32_t* chunk = nullptr;        // [E]
+  int32_t* row_count = nullptr;    // [E], or null: the main schedule takes every expert (= counts)
+  int thin_rows = 0;
+  int thin_nmax = 0;
+  int32_t* thin_tile_prefix = nullptr;
+  int32_t* thin_chunk = nullptr;
+  int32_t* thin_row_count = nullptr;
+};
+// blockcnt: [align_blocks * E] int32 scratch.  sched may be null (no scheduler).
 cudaError_t launch_align(const int32_t* ids, int T, int k, int E, int align, int32_t* counts, int32_t* offsets,
-                         int32_t* sorted_ids, int32_t* inv_pos, int32_t* blockcnt, int nmax, int32_t* tile_prefix,
-                         int32_t* chunk, cudaStream_t s);
+                         int32_t* sorted_ids, int32_t* inv_pos, int32_t* blockcnt, const SchedOut* sched,
+                         cudaStream_t s);
 // Scheduler for the public grouped GEMM: from expert_offsets [E+1] (arbitrary row counts).
 cudaError_t launch_sched_from_offsets(const int32_t* offsets, int E, int M, int nmax, int32_t* row_count,
                                       int32_t* tile_prefix, int32_t* chunk, cudaStream_t s);
 
 // permute / combine (permute_combine.cu)
-cudaError_t launch_permute_w4(const uint16_t* x_bf16, const int32_t* inv_pos, int T, int k, int H, __half* x_perm,
-                              cudaStream_t s);
+// x rows -> expert-sorted interleaved fp16 rows x_perm[inv_pos[p]] for every pair p (or, with
+// ids / cls_rows given, for the pairs whose expert has cls_rows[ids[p]] > 0)
+cudaError_t launch_permute_w4(const uint16_t* x_bf16, const int32_t* inv_pos, const int32_t* ids,
+                              const int32_t* cls_rows, int T, int k, int H, __half* x_perm, cudaStream_t s);
 cudaError_t launch_convert_rows(const uint16_t* a, int a_is_bf16, int M, int K, __half* out, cudaStream_t s);
 cudaError_t launch_combine(const float* y_perm, const int32_t* inv_pos, const float* topk_w, int T, int k, int H,
                            void* out, int out_fp32, cudaStream_t s);
@@ -99,9 +117,11 @@ cudaError_t launch_w4i8_gemm(const W4I8Problem& p, cudaStream_t s);
 cudaError_t launch_reduce_splits(const float* part, int splits, int rows, int N, const int32_t* row_start,
                                  const int32_t* row_count, int E, void* out, int out_fp32, cudaStream_t s);
 // Planes of the K-vectors x_src: plane row r takes source row r (inv_pos == null, k == 1),
-// or for every pair p plane row inv_pos[p] takes source row p / k.
-cudaError_t launch_planes(const uint16_t* a, int a_is_bf16, const int32_t* inv_pos, int n_pairs, int k, int K,
-                          int8_t* planes, int32_t* meta, cudaStream_t s);
+// or for every pair p plane row inv_pos[p] takes source row p / k (with ids / cls_rows given,
+// only the pairs whose expert has cls_rows[ids[p]] > 0).
+cudaError_t launch_planes(const uint16_t* a, int a_is_bf16, const int32_t* inv_pos, const int32_t* ids,
+                          const int32_t* cls_rows, int n_pairs, int k, int K, int8_t* planes, int32_t* meta,
+                          cudaStream_t s);
 
 // block-FP8 grouped GEMM (gemm_fp8.cu)
 struct F8GemmProblem {

@@ -55,12 +55,15 @@ __device__ __forceinline__ bool f16x8_nonfinite(const uint4& v) {
 // a value the fp16 operand cannot hold is still converted (to +-inf) and recorded as
 // MOE_ERR_DEVICE_CHECK.
 __global__ void __launch_bounds__(256) permute_w4_kernel(const uint4* __restrict__ x, const int32_t* __restrict__ inv_pos,
-                                                         int P, int k, int H8, uint4* __restrict__ x_perm) {
+                                                         const int32_t* __restrict__ ids,
+                                                         const int32_t* __restrict__ cls_rows, int P, int k, int H8,
+                                                         uint4* __restrict__ x_perm) {
   const int p = (int)((blockIdx.x * blockDim.x + threadIdx.x) >> 5);
   const int lane = threadIdx.x & 31;
   if (p >= P) return;
   const int r = inv_pos[p];
-  if (r < 0) return;
+  if (r < 0) return;  // an out-of-range id (inv_pos -1): then ids[p] is not read
+  if (cls_rows && __ldg(cls_rows + __ldg(ids + p)) == 0) return;  // the expert runs on the other GEMM
   const uint4* src = x + (size_t)(p / k) * H8;
   uint4* dst = x_perm + (size_t)r * H8;
   bool bad = false;
@@ -72,12 +75,12 @@ __global__ void __launch_bounds__(256) permute_w4_kernel(const uint4* __restrict
   if (__any_sync(0xffffffffu, bad) && lane == 0) set_status(MOE_ERR_DEVICE_CHECK);
 }
 
-cudaError_t launch_permute_w4(const uint16_t* x_bf16, const int32_t* inv_pos, int T, int k, int H, __half* x_perm,
-                              cudaStream_t s) {
+cudaError_t launch_permute_w4(const uint16_t* x_bf16, const int32_t* inv_pos, const int32_t* ids,
+                              const int32_t* cls_rows, int T, int k, int H, __half* x_perm, cudaStream_t s) {
   const int P = T * k;
   timing_before("permute", s);
-  permute_w4_kernel<<<ceil_div(P, 8), 256, 0, s>>>(reinterpret_cast<const uint4*>(x_bf16), inv_pos, P, k, H / 8,
-                                                  reinterpret_cast<uint4*>(x_perm));
+  permute_w4_kernel<<<ceil_div(P, 8), 256, 0, s>>>(reinterpret_cast<const uint4*>(x_bf16), inv_pos, ids, cls_rows, P,
+                                                  k, H / 8, reinterpret_cast<uint4*>(x_perm));
   timing_after("permute", s);
   return cudaGetLastError();
 }
@@ -116,7 +119,9 @@ cudaError_t launch_permute_fp8(const uint8_t* x, const float* xs, const int32_t*
 // word unpacks); the sum of X over every 32-K group (for the MMA's offset correction) and the
 // block scales go to the row's meta words.
 __global__ void __launch_bounds__(256) planes_kernel(const uint4* __restrict__ a, int a_is_bf16,
-                                                     const int32_t* __restrict__ inv_pos, int n_pairs, int k, int K,
+                                                     const int32_t* __restrict__ inv_pos,
+                                                     const int32_t* __restrict__ ids,
+                                                     const int32_t* __restrict__ cls_rows, int n_pairs, int k, int K,
                                                      uint2* __restrict__ planes, int32_t* __restrict__ meta) {
   const int nblk = K / 128;
   const size_t unit = (blockIdx.x * (size_t)blockDim.x + threadIdx.x) >> 4;  // (pair, block)
@@ -124,7 +129,12 @@ __global__ void __launch_bounds__(256) planes_kernel(const uint4* __restrict__ a
   const bool live = unit < (size_t)n_pairs * nblk;
   const int p = live ? (int)(unit / nblk) : 0;
   const int blk = live ? (int)(unit % nblk) : 0;
-  const int r = live ? (inv_pos ? inv_pos[p] : p) : -1;
+  int r = live ? (inv_pos ? inv_pos[p] : p) : -1;
+  // a pair whose expert runs on the other GEMM (ids[p] is read only for a pair inv_pos placed)
+  if (r >= 0 && cls_rows && __ldg(cls_rows + __ldg(ids + p)) == 0) r = -1;
+  // a warp's two units are (pair, block) neighbours, nearly always of one pair: a warp with
+  // nothing to write leaves before any load or arithmetic
+  if (__all_sync(0xffffffffu, r < 0)) return;
   const int src = p / k;
   float x[8];
   float amax = 0.f;
@@ -179,13 +189,14 @@ __global__ void __launch_bounds__(256) planes_kernel(const uint4* __restrict__ a
   if (i == 0) m[8 + (blk & 1)] = __float_as_int(sc);
 }
 
-cudaError_t launch_planes(const uint16_t* a, int a_is_bf16, const int32_t* inv_pos, int n_pairs, int k, int K,
-                          int8_t* planes, int32_t* meta, cudaStream_t s) {
+cudaError_t launch_planes(const uint16_t* a, int a_is_bf16, const int32_t* inv_pos, const int32_t* ids,
+                          const int32_t* cls_rows, int n_pairs, int k, int K, int8_t* planes, int32_t* meta,
+                          cudaStream_t s) {
   const size_t threads = (size_t)n_pairs * (K / 128) * 16;
   timing_before("planes", s);
   planes_kernel<<<(unsigned)((threads + 255) / 256), 256, 0, s>>>(reinterpret_cast<const uint4*>(a), a_is_bf16,
-                                                                  inv_pos, n_pairs, k, K, reinterpret_cast<uint2*>(planes),
-                                                                  meta);
+                                                                  inv_pos, ids, cls_rows, n_pairs, k, K,
+                                                                  reinterpret_cast<uint2*>(planes), meta);
   timing_after("planes", s);
   return cudaGetLastError();
 }

@@ -170,9 +170,7 @@ __global__ void __launch_bounds__(256) align_hist_kernel(const int32_t* __restri
 __global__ void __launch_bounds__(1024) align_scan_kernel(int32_t* __restrict__ blockcnt, int nb, int E, int align,
                                                           int P, int32_t* __restrict__ counts,
                                                           int32_t* __restrict__ offsets,
-                                                          int32_t* __restrict__ sorted_ids, int nmax,
-                                                          int32_t* __restrict__ tile_prefix,
-                                                          int32_t* __restrict__ chunk) {
+                                                          int32_t* __restrict__ sorted_ids, SchedOut sch) {
   __shared__ int warp_tot[32];
   __shared__ int total;
   const int e = threadIdx.x;
@@ -191,15 +189,34 @@ __global__ void __launch_bounds__(1024) align_scan_kernel(int32_t* __restrict__ 
   if (e == 0) offsets[E] = total;
   if (e < E)
     for (int r = off + c; r < off + padded; ++r) sorted_ids[r] = P;
-  if (tile_prefix) {
+  if (sch.tile_prefix) {
+    // per expert, from its actual count: the thin schedule (int8 tensor-core GEMM, small token
+    // tiles) when it has at most thin_rows rows, else the main one (fp16 GEMM, wide tiles)
+    // (with thin_rows = 0 the thin schedule is still written, empty, so no reader sees stale data)
+    const bool two = sch.thin_tile_prefix != nullptr;
+    const bool thin = two && c <= sch.thin_rows;
+    const int c_main = thin ? 0 : c;
     int nt = 0, ch = 16;
-    if (e < E) expert_tiles(c, nmax, &nt, &ch);
+    if (e < E) expert_tiles(c_main, sch.nmax, &nt, &ch);
     const int tp = block_exclusive_scan(nt, warp_tot, &total);
     if (e < E) {
-      tile_prefix[e] = tp;
-      chunk[e] = ch;
+      sch.tile_prefix[e] = tp;
+      sch.chunk[e] = ch;
+      if (sch.row_count) sch.row_count[e] = c_main;
     }
-    if (e == 0) tile_prefix[E] = total;
+    if (e == 0) sch.tile_prefix[E] = total;
+    if (two) {
+      const int c_thin = thin ? c : 0;
+      int nt2 = 0, ch2 = 16;
+      if (e < E) expert_tiles(c_thin, sch.thin_nmax, &nt2, &ch2);
+      const int tp2 = block_exclusive_scan(nt2, warp_tot, &total);
+      if (e < E) {
+        sch.thin_tile_prefix[e] = tp2;
+        sch.thin_chunk[e] = ch2;
+        sch.thin_row_count[e] = c_thin;
+      }
+      if (e == 0) sch.thin_tile_prefix[E] = total;
+    }
   }
 }
 
@@ -234,16 +251,16 @@ __global__ void __launch_bounds__(32) align_scatter_kernel(const int32_t* __rest
 int align_blocks(int T, int k) { return ceil_div(T * k, kAlignChunk); }
 
 cudaError_t launch_align(const int32_t* ids, int T, int k, int E, int align, int32_t* counts, int32_t* offsets,
-                         int32_t* sorted_ids, int32_t* inv_pos, int32_t* blockcnt, int nmax, int32_t* tile_prefix,
-                         int32_t* chunk, cudaStream_t s) {
+                         int32_t* sorted_ids, int32_t* inv_pos, int32_t* blockcnt, const SchedOut* sched,
+                         cudaStream_t s) {
   const int P = T * k;
   const int nb = align_blocks(T, k);
   timing_before("align_hist", s);
   align_hist_kernel<<<nb, 256, 0, s>>>(ids, P, E, blockcnt);
   timing_after("align_hist", s);
   timing_before("align_scan", s);
-  align_scan_kernel<<<1, 1024, 0, s>>>(blockcnt, nb, E, align, P, counts, offsets, sorted_ids, nmax, tile_prefix,
-                                       chunk);
+  SchedOut none{};
+  align_scan_kernel<<<1, 1024, 0, s>>>(blockcnt, nb, E, align, P, counts, offsets, sorted_ids, sched ? *sched : none);
   timing_after("align_scan", s);
   timing_before("align_scatter", s);
   align_scatter_kernel<<<nb, 32, 0, s>>>(ids, P, E, blockcnt, offsets, sorted_ids, inv_pos);

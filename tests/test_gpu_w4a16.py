@@ -72,6 +72,17 @@ def test_expert_counts_at_tile_boundaries_wide():
     run_and_check(W4Layer(8, len(assign), 256, 128, E, 1, logits=lg), what="wide boundaries")
 
 
+def test_expert_counts_straddling_the_kernel_choice():
+    """T > 64: each expert runs on the int8 GEMM when it has few rows and on the fp16 GEMM when
+    it has many, chosen per expert from its count in the same call; counts on both sides of
+    every plausible switch point (8, 16, 32, 48, 64 rows) and of the tile heights."""
+    counts = [1, 7, 8, 9, 15, 16, 17, 31, 32, 33, 47, 48, 49, 63, 64, 65, 100, 129, 0, 2]
+    assign = np.repeat(np.arange(len(counts)), counts)
+    E = 24
+    lg = _onehot_logits(assign, E, 1, 14)
+    run_and_check(W4Layer(14, len(assign), 256, 256, E, 1, logits=lg), what="mixed kernels")
+
+
 def test_all_tokens_one_expert_top2():
     T, E = 300, 8
     lg = synth.logits(9, T, E)
