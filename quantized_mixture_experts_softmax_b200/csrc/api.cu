@@ -173,6 +173,8 @@ struct FwdWs {
   int32_t *tile_prefix, *chunk, *row_count;                  // fp16 GEMM schedule (wide experts)
   int32_t *thin_tile_prefix, *thin_chunk, *thin_row_count;   // int8 GEMM schedule
   __half *x_perm, *h;  // fp16 path rows
+  int32_t *x_exp, *h_exp, *ovf_flag;  // fp16 path: per-row exponents and h overflow flags
+  uint32_t* ovf_mask;                 // fp16 path: [P, I/32] h overflow marks
   Planes xq, hq;       // int8 path rows
   float* y;
   size_t bytes;
@@ -197,6 +199,10 @@ FwdWs carve_w4_forward(void* ws, int T, int H, int I, int E, int k) {
     w.thin_row_count = c.take<int32_t>(E);
     w.x_perm = c.take<__half>(P * H);
     w.h = c.take<__half>(P * I);
+    w.x_exp = c.take<int32_t>(P);
+    w.h_exp = c.take<int32_t>(P);
+    w.ovf_flag = c.take<int32_t>(P);
+    w.ovf_mask = c.take<uint32_t>(P * (I / 32));
   }
   w.y = c.take<float>(P * H);
   w.bytes = c.off + 256;
@@ -218,8 +224,9 @@ int gemm_splits(int M, int K, int N) {
 
 struct GemmWs {
   int32_t *row_count, *tile_prefix, *chunk;
-  __half* a;    // fp16 path
-  Planes aq;    // int8 path
+  __half* a;       // fp16 path
+  int32_t* a_exp;  // fp16 path: per-row exponents
+  Planes aq;       // int8 path
   float* part;  // with K splits: [splits, M, N] fp32 partial sums
   size_t bytes;
 };
@@ -229,10 +236,12 @@ GemmWs carve_gemm(void* ws, int M, int K, int N, int E) {
   w.row_count = c.take<int32_t>(E);
   w.tile_prefix = c.take<int32_t>(E + 1);
   w.chunk = c.take<int32_t>(E);
-  if (use_i8(M))
+  if (use_i8(M)) {
     w.aq = take_planes(c, M, K);
-  else
+  } else {
     w.a = c.take<__half>((size_t)M * K);
+    w.a_exp = c.take<int32_t>(M);
+  }
   const int sp = gemm_splits(M, K, N);
   if (sp > 1) w.part = c.take<float>((size_t)sp * M * N);
   w.bytes = c.off + 256;
@@ -372,7 +381,9 @@ moe_status_t moe_w4a16_forward(const moe_w4a16_args* a, void* ws, size_t ws_byte
   if (e == cudaSuccess)
     e = launch_planes(x, 1, w.inv, mixed ? a->topk_ids : nullptr, mixed ? w.thin_row_count : nullptr, P, k, H, w.xq.x,
                       w.xq.meta, stream);
-  if (e == cudaSuccess && mixed) e = launch_permute_w4(x, w.inv, a->topk_ids, w.row_count, T, k, H, w.x_perm, stream);
+  if (e == cudaSuccess && mixed)
+    e = launch_permute_w4(x, w.inv, a->topk_ids, w.row_count, T, k, H, w.x_perm, w.x_exp, w.ovf_flag, w.ovf_mask, I,
+                          stream);
   // gate/up with SiLU*up, then down, each on both GEMMs (an empty schedule makes a kernel exit)
   if (e == cudaSuccess) {
     W4I8Problem g{a->w13_q, w13_s, w.xq.x, w.xq.meta, P, H, E, 2 * I, true, I, thin, OUT_PLANES, w.hq.x, w.hq.meta, I};
@@ -381,14 +392,20 @@ moe_status_t moe_w4a16_forward(const moe_w4a16_args* a, void* ws, size_t ws_byte
   if (e == cudaSuccess && mixed) {
     W4GemmProblem g{a->w13_q, w13_s, w.x_perm, P, H, E, 2 * I, true, I, wide, kWideTileRows, w.h, I,
                     OUT_H_F16_INTERLEAVED};
+    g.acc_exp = w.x_exp;
+    g.ovf_flag = w.ovf_flag;
+    g.ovf_mask = w.ovf_mask;
     e = launch_w4a16_gemm(g, stream);
   }
+  // rows with an h beyond fp16 (rare) are brought to one power-of-two scale before the down GEMM
+  if (e == cudaSuccess && mixed) e = launch_h_rescale(w.h, P, I, w.ovf_flag, w.ovf_mask, w.h_exp, stream);
   if (e == cudaSuccess) {
     W4I8Problem g{a->w2_q, w2_s, w.hq.x, w.hq.meta, P, I, E, H, false, 0, thin, OUT_F32, w.y, nullptr, H};
     e = launch_w4i8_gemm(g, stream);
   }
   if (e == cudaSuccess && mixed) {
     W4GemmProblem g{a->w2_q, w2_s, w.h, P, I, E, H, false, 0, wide, kWideTileRows, w.y, H, OUT_F32};
+    g.acc_exp = w.h_exp;
     e = launch_w4a16_gemm(g, stream);
   }
   if (e == cudaSuccess) e = launch_combine(w.y, w.inv, a->topk_w, T, k, H, a->out, a->out_fp32, stream);
@@ -477,11 +494,13 @@ moe_status_t moe_w4a16_gemm(const void* a, int a_is_bf16, const int32_t* w_q, co
     if (e == cudaSuccess && sp > 1) e = launch_reduce_splits(w.part, sp, M, N, expert_offsets, w.row_count, E, out, out_fp32, stream);
     return e == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
   }
-  if (e == cudaSuccess) e = launch_convert_rows(static_cast<const uint16_t*>(a), a_is_bf16, M, K, w.a, stream);
+  if (e == cudaSuccess)
+    e = launch_convert_rows(static_cast<const uint16_t*>(a), a_is_bf16, M, K, w.a, w.a_exp, stream);
   const int sp = gemm_splits(M, K, N);
   if (e == cudaSuccess) {
     W4GemmProblem g{w_q, static_cast<const uint16_t*>(w_s), w.a, M, K, E, N, false, 0, sched, nmax, out, N,
                     out_fp32 ? OUT_F32 : OUT_BF16, sp, w.part};
+    g.acc_exp = w.a_exp;
     e = launch_w4a16_gemm(g, stream);
   }
   if (e == cudaSuccess && sp > 1) e = launch_reduce_splits(w.part, sp, M, N, expert_offsets, w.row_count, E, out, out_fp32, stream);

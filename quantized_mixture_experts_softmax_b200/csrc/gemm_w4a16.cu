@@ -84,8 +84,14 @@ struct Params {
   int splits;   // K splits per (expert, weight tile, token tile); > 1 only for plain outputs
   float* part;  // splits > 1: fp32 partial sums [splits, act_rows, out_ld]
   int act_rows;
+  const int32_t* acc_exp;  // null, or per activation row e: its accumulators are multiplied by 2^e
+  int32_t* ovf_flag;       // gated: row r set to 1 when one of its h values was stored prescaled
+  uint32_t* ovf_mask;      // gated: [act_rows, out_ld/32] bit per stored h position prescaled by 2^-16
   uint64_t wait_limit;
 };
+
+// 2^e as a float for an exponent e in [-126, 127]
+__device__ __forceinline__ float exp2_int(int e) { return __int_as_float((127 + e) << 23); }
 
 struct Item {
   int e, m, r0, nvalid, nmma;
@@ -339,19 +345,37 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (GATED) tmem_ld16(tb + NMAX + c0, u);
         tmem_ld_wait();
         const int nv = min(16, I.nvalid - c0);
+        if (p.acc_exp) {  // rows whose fp16 operand was scaled by 2^-e to fit fp16: undo it
+#pragma unroll
+          for (int i = 0; i < 16; ++i) {
+            if (i < nv) {
+              const float sc = exp2_int(__ldg(p.acc_exp + I.r0 + c0 + i));
+              g[i] = __float_as_uint(__uint_as_float(g[i]) * sc);
+              if (GATED) u[i] = __float_as_uint(__uint_as_float(u[i]) * sc);
+            }
+          }
+        }
         if (GATED) {
-          __half* out = reinterpret_cast<__half*>(p.out) + (size_t)(I.r0 + c0) * p.out_ld + interleave_pos(col);
-          bool big = false;  // an h the fp16 operand of the down projection cannot hold
+          const int pos = interleave_pos(col);
+          __half* out = reinterpret_cast<__half*>(p.out) + (size_t)(I.r0 + c0) * p.out_ld + pos;
+          bool huge = false;  // an h beyond even the prescaled fp16 range (2^32)
 #pragma unroll
           for (int i = 0; i < 16; ++i) {
             if (i < nv) {
               const float gv = __uint_as_float(g[i]), uv = __uint_as_float(u[i]);
               const float hv = gv / (1.0f + __expf(-gv)) * uv;
-              big |= !(fabsf(hv) < 65520.0f);
-              out[(size_t)i * p.out_ld] = __float2half_rn(hv);
+              if (fabsf(hv) < 65520.0f) {
+                out[(size_t)i * p.out_ld] = __float2half_rn(hv);
+              } else {  // beyond fp16: stored as h * 2^-16 and marked; h_rescale fixes its row
+                const int r = I.r0 + c0 + i;
+                out[(size_t)i * p.out_ld] = __float2half_rn(hv * (1.0f / 65536.0f));
+                atomicOr(p.ovf_mask + (size_t)r * (p.out_ld / 32) + pos / 32, 1u << (pos & 31));
+                p.ovf_flag[r] = 1;
+                huge |= !(fabsf(hv) < 65520.0f * 65536.0f);
+              }
             }
           }
-          if (big) set_status(MOE_ERR_DEVICE_CHECK);
+          if (huge) set_status(MOE_ERR_DEVICE_CHECK);
         } else if (p.splits > 1) {  // this split's partial sum, reduced in split order by another kernel
           float* out = p.part + (size_t)(it % p.splits) * p.act_rows * p.out_ld + (size_t)(I.r0 + c0) * p.out_ld + col;
 #pragma unroll
@@ -501,6 +525,10 @@ cudaError_t launch_t(const W4GemmProblem& pr, cudaStream_t s) {
   p.splits = pr.splits > 1 && !GATED ? pr.splits : 1;
   p.part = pr.part;
   p.act_rows = pr.act_rows;
+  p.acc_exp = pr.acc_exp;
+  p.ovf_flag = pr.ovf_flag;
+  p.ovf_mask = pr.ovf_mask;
+  if (GATED && (!p.ovf_flag || !p.ovf_mask)) return cudaErrorInvalidValue;
   p.wait_limit = wait_limit_ns();
   const size_t smem = C::smem_bytes(pr.E);
   auto kern = w4a16_gemm_kernel<GATED>;

@@ -52,11 +52,18 @@ cudaError_t launch_sched_from_offsets(const int32_t* offsets, int E, int M, int 
                                       int32_t* tile_prefix, int32_t* chunk, cudaStream_t s);
 
 // permute / combine (permute_combine.cu)
-// x rows -> expert-sorted interleaved fp16 rows x_perm[inv_pos[p]] for every pair p (or, with
-// ids / cls_rows given, for the pairs whose expert has cls_rows[ids[p]] > 0)
+// x rows -> expert-sorted interleaved fp16 rows for every pair p (or, with ids / cls_rows given,
+// for the pairs whose expert has cls_rows[ids[p]] > 0): row r = inv_pos[p] holds
+// fp16(x[p/k] * 2^-x_exp[r]) with x_exp[r] >= 0 the smallest exponent that fits the row into
+// fp16.  For every placed pair ovf_flag[r] is cleared, and for the converted rows the I/32 words
+// of ovf_mask too (the gated GEMM's overflow marks).
 cudaError_t launch_permute_w4(const uint16_t* x_bf16, const int32_t* inv_pos, const int32_t* ids,
-                              const int32_t* cls_rows, int T, int k, int H, __half* x_perm, cudaStream_t s);
-cudaError_t launch_convert_rows(const uint16_t* a, int a_is_bf16, int M, int K, __half* out, cudaStream_t s);
+                              const int32_t* cls_rows, int T, int k, int H, __half* x_perm, int32_t* x_exp,
+                              int32_t* ovf_flag, uint32_t* ovf_mask, int I, cudaStream_t s);
+// rows of a (bf16 or fp16) -> interleaved fp16 rows out[r] = fp16(a[r] * 2^-x_exp[r]), x_exp[r]
+// the smallest exponent >= 0 that fits the row into fp16
+cudaError_t launch_convert_rows(const uint16_t* a, int a_is_bf16, int M, int K, __half* out, int32_t* x_exp,
+                                cudaStream_t s);
 cudaError_t launch_combine(const float* y_perm, const int32_t* inv_pos, const float* topk_w, int T, int k, int H,
                            void* out, int out_fp32, cudaStream_t s);
 
@@ -77,8 +84,19 @@ struct W4GemmProblem {
   OutKind out_kind;
   int splits = 1;          // plain outputs: K split this many ways into `part`, then reduce_splits
   float* part = nullptr;   // [splits, act_rows, out_ld] fp32
+  // Range handling of the fp16 operands (exact power-of-two scalings):
+  const int32_t* acc_exp = nullptr;  // per act row e (or null): accumulators times 2^e before the epilogue
+  int32_t* ovf_flag = nullptr;       // gated (required): [act_rows], set to 1 for a row with an h value
+                                     // beyond fp16, which is then stored as h * 2^-16 ...
+  uint32_t* ovf_mask = nullptr;      // ... and marked in this [act_rows, I/32] bit mask (by stored
+                                     // position); launch_h_rescale rescales such rows
 };
 cudaError_t launch_w4a16_gemm(const W4GemmProblem& p, cudaStream_t s);
+// After a gated fp16 GEMM: every row r with ovf_flag[r] set is rescaled in place to
+// h * 2^-c with the smallest c >= 1 that fits the row into fp16 (h_exp[r] = c), the others get
+// h_exp[r] = 0.  Clears nothing; the rows' flags and masks are cleared by launch_permute_w4.
+cudaError_t launch_h_rescale(__half* h, int rows, int I, const int32_t* ovf_flag, const uint32_t* ovf_mask,
+                             int32_t* h_exp, cudaStream_t s);
 
 // W4A16 grouped GEMM for decode-sized experts on the int8 tensor cores (gemm_w4i8.cu).
 // Activations as 16-bit fixed-point planes: per (row, 128-K block) scale s, X = rint(x/s)

@@ -18,12 +18,6 @@ __device__ __forceinline__ uint32_t pack_h2(float lo, float hi) {
 __device__ __forceinline__ float bf16lo(uint32_t u) { return __uint_as_float(u << 16); }
 __device__ __forceinline__ float bf16hi(uint32_t u) { return __uint_as_float(u & 0xFFFF0000u); }
 
-// 8 bf16 (k0..k7 in order) -> 8 fp16 in the interleaved order (k0,k4,k1,k5,k2,k6,k3,k7)
-__device__ __forceinline__ uint4 bf16x8_to_f16x8_interleaved(uint4 v) {
-  const float f0 = bf16lo(v.x), f1 = bf16hi(v.x), f2 = bf16lo(v.y), f3 = bf16hi(v.y);
-  const float f4 = bf16lo(v.z), f5 = bf16hi(v.z), f6 = bf16lo(v.w), f7 = bf16hi(v.w);
-  return make_uint4(pack_h2(f0, f4), pack_h2(f1, f5), pack_h2(f2, f6), pack_h2(f3, f7));
-}
 __device__ __forceinline__ uint4 f16x8_interleave(uint4 v) {
   // halves: v.x=(k0,k1) v.y=(k2,k3) v.z=(k4,k5) v.w=(k6,k7)
   const uint32_t a = __byte_perm(v.x, v.z, 0x5410);  // (k0,k4)
@@ -33,55 +27,148 @@ __device__ __forceinline__ uint4 f16x8_interleave(uint4 v) {
   return make_uint4(a, b, c, d);
 }
 
-// True when one of the 8 bf16 values is outside the finite fp16 range: |x| >= 65536 (the
-// smallest bf16 magnitude above 65504 the cast would turn into infinity), infinite or NaN.
-__device__ __forceinline__ bool bf16x8_beyond_f16(const uint4& v) {
-  const uint32_t w[4] = {v.x, v.y, v.z, v.w};
-  bool bad = false;
-#pragma unroll
-  for (int j = 0; j < 4; ++j) bad |= (w[j] & 0x7FFFu) >= 0x4780u || ((w[j] >> 16) & 0x7FFFu) >= 0x4780u;
-  return bad;
-}
-// True when one of the 8 fp16 values is infinite or NaN.
-__device__ __forceinline__ bool f16x8_nonfinite(const uint4& v) {
-  const uint32_t w[4] = {v.x, v.y, v.z, v.w};
-  bool bad = false;
-#pragma unroll
-  for (int j = 0; j < 4; ++j) bad |= (w[j] & 0x7C00u) == 0x7C00u || (w[j] & 0x7C000000u) == 0x7C000000u;
-  return bad;
+// 2^e as a float for an exponent e in [-126, 127]
+__device__ __forceinline__ float exp2i(int e) { return __int_as_float((127 + e) << 23); }
+
+// The smallest c >= 0 with amax * 2^-c <= 65504 (the largest finite fp16): scaling a row by
+// 2^-c is exact and fits it into the fp16 operand of the tensor cores.
+__device__ __forceinline__ int fit_exp(float amax) {
+  if (!(amax > 65504.0f) || !(amax <= 3.402823466e38f)) return 0;  // fits, or not finite (flagged)
+  int c = (__float_as_int(amax) >> 23) - 126 - 16;                   // amax < 2^(c + 16)
+  if (c < 0) c = 0;
+  if (amax * exp2i(-c) > 65504.0f) ++c;
+  return c;
 }
 
-// one warp per (token, slot) pair: x_perm[inv_pos[p]] = interleave(fp16(x[p / k])).  A row with
-// a value the fp16 operand cannot hold is still converted (to +-inf) and recorded as
-// MOE_ERR_DEVICE_CHECK.
+// largest magnitude field (bits & 0x7FFF) of 8 packed 16-bit floats: for bf16 and fp16 alike the
+// field orders finite magnitudes, and infinities and NaNs compare above all of them
+__device__ __forceinline__ uint32_t mag16x8_max(const uint4& v) {
+  const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+  uint32_t m = 0;
+#pragma unroll
+  for (int j = 0; j < 4; ++j) m = max(m, max(w[j] & 0x7FFFu, (w[j] >> 16) & 0x7FFFu));
+  return m;
+}
+__device__ __forceinline__ uint32_t warp_max_u32(uint32_t v) {
+#pragma unroll
+  for (int off = 16; off; off >>= 1) v = max(v, __shfl_xor_sync(0xffffffffu, v, off));
+  return v;
+}
+
+// 8 bf16 (k0..k7 in order) times 2^-c -> 8 fp16 in the interleaved order
+__device__ __forceinline__ uint4 bf16x8_scaled_to_f16x8_interleaved(uint4 v, float sc) {
+  const float f0 = bf16lo(v.x) * sc, f1 = bf16hi(v.x) * sc, f2 = bf16lo(v.y) * sc, f3 = bf16hi(v.y) * sc;
+  const float f4 = bf16lo(v.z) * sc, f5 = bf16hi(v.z) * sc, f6 = bf16lo(v.w) * sc, f7 = bf16hi(v.w) * sc;
+  return make_uint4(pack_h2(f0, f4), pack_h2(f1, f5), pack_h2(f2, f6), pack_h2(f3, f7));
+}
+
+// One warp per (token, slot) pair p placed at row r = inv_pos[p]: clears the row's overflow flag
+// (both classes of experts), then, for a pair whose expert runs on the fp16 GEMM, scans the token's
+// bf16 row for its largest magnitude, picks the row exponent c (0 unless a value is beyond fp16)
+// and writes x_perm[r] = interleave(fp16(x * 2^-c)), x_exp[r] = c, and clears the row's overflow
+// mask.  A non-finite input is recorded as MOE_ERR_DEVICE_CHECK.  The second pass over the row
+// reads it again from L1.
 __global__ void __launch_bounds__(256) permute_w4_kernel(const uint4* __restrict__ x, const int32_t* __restrict__ inv_pos,
                                                          const int32_t* __restrict__ ids,
                                                          const int32_t* __restrict__ cls_rows, int P, int k, int H8,
-                                                         uint4* __restrict__ x_perm) {
+                                                         uint4* __restrict__ x_perm, int32_t* __restrict__ x_exp,
+                                                         int32_t* __restrict__ ovf_flag, uint32_t* __restrict__ ovf_mask,
+                                                         int mask_words) {
   const int p = (int)((blockIdx.x * blockDim.x + threadIdx.x) >> 5);
   const int lane = threadIdx.x & 31;
   if (p >= P) return;
   const int r = inv_pos[p];
   if (r < 0) return;  // an out-of-range id (inv_pos -1): then ids[p] is not read
+  if (lane == 0 && ovf_flag) ovf_flag[r] = 0;
   if (cls_rows && __ldg(cls_rows + __ldg(ids + p)) == 0) return;  // the expert runs on the other GEMM
   const uint4* src = x + (size_t)(p / k) * H8;
   uint4* dst = x_perm + (size_t)r * H8;
-  bool bad = false;
-  for (int c = lane; c < H8; c += 32) {
-    const uint4 v = __ldg(src + c);
-    bad |= bf16x8_beyond_f16(v);
-    dst[c] = bf16x8_to_f16x8_interleaved(v);
-  }
-  if (__any_sync(0xffffffffu, bad) && lane == 0) set_status(MOE_ERR_DEVICE_CHECK);
+  uint32_t m = 0;
+  for (int c = lane; c < H8; c += 32) m = max(m, mag16x8_max(__ldg(src + c)));
+  m = warp_max_u32(m);
+  const float amax = __uint_as_float(m << 16);
+  if (lane == 0 && !(amax <= 3.402823466e38f)) set_status(MOE_ERR_DEVICE_CHECK);
+  const int e = fit_exp(amax);
+  const float sc = exp2i(-e);
+  for (int c = lane; c < H8; c += 32) dst[c] = bf16x8_scaled_to_f16x8_interleaved(__ldg(src + c), sc);
+  if (lane == 0) x_exp[r] = e;
+  if (ovf_mask)
+    for (int w = lane; w < mask_words; w += 32) ovf_mask[(size_t)r * mask_words + w] = 0;
 }
 
 cudaError_t launch_permute_w4(const uint16_t* x_bf16, const int32_t* inv_pos, const int32_t* ids,
-                              const int32_t* cls_rows, int T, int k, int H, __half* x_perm, cudaStream_t s) {
+                              const int32_t* cls_rows, int T, int k, int H, __half* x_perm, int32_t* x_exp,
+                              int32_t* ovf_flag, uint32_t* ovf_mask, int I, cudaStream_t s) {
   const int P = T * k;
   timing_before("permute", s);
   permute_w4_kernel<<<ceil_div(P, 8), 256, 0, s>>>(reinterpret_cast<const uint4*>(x_bf16), inv_pos, ids, cls_rows, P,
-                                                  k, H / 8, reinterpret_cast<uint4*>(x_perm));
+                                                  k, H / 8, reinterpret_cast<uint4*>(x_perm), x_exp, ovf_flag, ovf_mask,
+                                                  I / 32);
   timing_after("permute", s);
+  return cudaGetLastError();
+}
+
+// One warp per row r of the gated GEMM's h [rows, I] (fp16, interleaved positions): a row with
+// its overflow flag set holds some values stored as h * 2^-16, marked in its mask by position.
+// The row is brought to one scale: c >= 1 the smallest exponent that fits max|h| into fp16, every
+// value rewritten as fp16(h * 2^-c) (exact power-of-two rescaling of the stored values), and
+// h_exp[r] = c for the down GEMM, which multiplies the row's accumulators by 2^c.  Other rows
+// get h_exp[r] = 0 and are not touched.
+__global__ void __launch_bounds__(256) h_rescale_kernel(uint4* __restrict__ h, int rows, int I8,
+                                                        const int32_t* __restrict__ ovf_flag,
+                                                        const uint32_t* __restrict__ ovf_mask,
+                                                        int32_t* __restrict__ h_exp) {
+  const int lane = threadIdx.x & 31;
+  const int mask_words = I8 / 4;
+  for (int r = (int)((blockIdx.x * blockDim.x + threadIdx.x) >> 5); r < rows;
+       r += (int)((gridDim.x * blockDim.x) >> 5)) {
+    if (__ldg(ovf_flag + r) == 0) {
+      if (lane == 0) h_exp[r] = 0;
+      continue;
+    }
+    uint4* row = h + (size_t)r * I8;
+    const uint32_t* mrow = ovf_mask + (size_t)r * mask_words;
+    float amax = 0.f;
+    for (int c = lane; c < I8; c += 32) {  // chunk c = stored positions 8c .. 8c+7
+      const uint4 v = row[c];
+      const uint32_t bits = (__ldg(mrow + c / 4) >> (8 * (c & 3))) & 0xFFu;
+      const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        const __half2 hh = *reinterpret_cast<const __half2*>(&w[j]);
+        amax = fmaxf(amax, fabsf(__low2float(hh)) * ((bits >> (2 * j)) & 1 ? 65536.0f : 1.0f));
+        amax = fmaxf(amax, fabsf(__high2float(hh)) * ((bits >> (2 * j + 1)) & 1 ? 65536.0f : 1.0f));
+      }
+    }
+#pragma unroll
+    for (int off = 16; off; off >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, off));
+    int e = fit_exp(amax);
+    if (e < 1) e = 1;
+    const float s_plain = exp2i(-e), s_marked = exp2i(16 - e);
+    for (int c = lane; c < I8; c += 32) {
+      const uint4 v = row[c];
+      const uint32_t bits = (__ldg(mrow + c / 4) >> (8 * (c & 3))) & 0xFFu;
+      uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        const __half2 hh = *reinterpret_cast<const __half2*>(&w[j]);
+        const float lo = __low2float(hh) * ((bits >> (2 * j)) & 1 ? s_marked : s_plain);
+        const float hi = __high2float(hh) * ((bits >> (2 * j + 1)) & 1 ? s_marked : s_plain);
+        w[j] = pack_h2(lo, hi);
+      }
+      row[c] = make_uint4(w[0], w[1], w[2], w[3]);
+    }
+    if (lane == 0) h_exp[r] = e;
+  }
+}
+
+cudaError_t launch_h_rescale(__half* h, int rows, int I, const int32_t* ovf_flag, const uint32_t* ovf_mask,
+                             int32_t* h_exp, cudaStream_t s) {
+  const size_t want = ((size_t)rows + 7) / 8;
+  const unsigned blocks = (unsigned)std::min<size_t>(want, (size_t)sm_count() * 16);
+  timing_before("h_rescale", s);
+  h_rescale_kernel<<<blocks, 256, 0, s>>>(reinterpret_cast<uint4*>(h), rows, I / 8, ovf_flag, ovf_mask, h_exp);
+  timing_after("h_rescale", s);
   return cudaGetLastError();
 }
 
@@ -247,25 +334,37 @@ cudaError_t launch_reduce_splits(const float* part, int splits, int rows, int N,
   return cudaGetLastError();
 }
 
-// rows of the single grouped GEMM's activations -> interleaved fp16; a value outside the finite
-// fp16 range (or a non-finite fp16 input) is recorded as MOE_ERR_DEVICE_CHECK
-__global__ void __launch_bounds__(256) convert_rows_kernel(const uint4* __restrict__ a, int a_is_bf16, size_t n8,
-                                                           uint4* __restrict__ out) {
-  bool bad = false;
-  for (size_t i = blockIdx.x * (size_t)blockDim.x + threadIdx.x; i < n8; i += (size_t)gridDim.x * blockDim.x) {
-    const uint4 v = __ldg(a + i);
-    bad |= a_is_bf16 ? bf16x8_beyond_f16(v) : f16x8_nonfinite(v);
-    out[i] = a_is_bf16 ? bf16x8_to_f16x8_interleaved(v) : f16x8_interleave(v);
+// One warp per row of the single grouped GEMM's activations: interleaved fp16 rows
+// out[r] = fp16(a[r] * 2^-x_exp[r]), x_exp[r] the smallest exponent >= 0 that fits the row into
+// fp16 (always 0 for fp16 input); a non-finite input is recorded as MOE_ERR_DEVICE_CHECK.
+__global__ void __launch_bounds__(256) convert_rows_kernel(const uint4* __restrict__ a, int a_is_bf16, int M, int K8,
+                                                           uint4* __restrict__ out, int32_t* __restrict__ x_exp) {
+  const int lane = threadIdx.x & 31;
+  for (int r = (int)((blockIdx.x * (size_t)blockDim.x + threadIdx.x) >> 5); r < M;
+       r += (int)(((size_t)gridDim.x * blockDim.x) >> 5)) {
+    const uint4* src = a + (size_t)r * K8;
+    uint4* dst = out + (size_t)r * K8;
+    uint32_t m = 0;
+    for (int c = lane; c < K8; c += 32) m = max(m, mag16x8_max(__ldg(src + c)));
+    m = warp_max_u32(m);
+    const bool finite = a_is_bf16 ? m < 0x7F80u : m < 0x7C00u;
+    if (lane == 0 && !finite) set_status(MOE_ERR_DEVICE_CHECK);
+    const int e = a_is_bf16 ? fit_exp(__uint_as_float(m << 16)) : 0;
+    const float sc = exp2i(-e);
+    for (int c = lane; c < K8; c += 32) {
+      const uint4 v = __ldg(src + c);
+      dst[c] = a_is_bf16 ? bf16x8_scaled_to_f16x8_interleaved(v, sc) : f16x8_interleave(v);
+    }
+    if (lane == 0) x_exp[r] = e;
   }
-  if (bad) set_status(MOE_ERR_DEVICE_CHECK);
 }
 
-cudaError_t launch_convert_rows(const uint16_t* a, int a_is_bf16, int M, int K, __half* out, cudaStream_t s) {
-  const size_t n8 = (size_t)M * K / 8;
-  const int blocks = (int)std::min<size_t>((n8 + 255) / 256, (size_t)sm_count() * 8);
+cudaError_t launch_convert_rows(const uint16_t* a, int a_is_bf16, int M, int K, __half* out, int32_t* x_exp,
+                                cudaStream_t s) {
+  const int blocks = (int)std::min<size_t>(((size_t)M + 7) / 8, (size_t)sm_count() * 16);
   timing_before("convert", s);
-  convert_rows_kernel<<<blocks, 256, 0, s>>>(reinterpret_cast<const uint4*>(a), a_is_bf16, n8,
-                                             reinterpret_cast<uint4*>(out));
+  convert_rows_kernel<<<blocks, 256, 0, s>>>(reinterpret_cast<const uint4*>(a), a_is_bf16, M, K / 8,
+                                             reinterpret_cast<uint4*>(out), x_exp);
   timing_after("convert", s);
   return cudaGetLastError();
 }

@@ -6,9 +6,9 @@ These tests use what real activations have and N(0,1) has not:
   * blocks with a 100x and a 1000x outlier next to ordinary values, in fixed channels and at
     random positions, on both paths;
   * an intermediate h spanning many decades (gate/up weight scales spread over 2.5 decades);
-  * bf16 values beyond the fp16 range: the int8 path takes them exactly like any other value,
-    the fp16 path cannot hold them and must say so through the device status word (as it must
-    for an h beyond fp16);
+  * bf16 values beyond the fp16 range, and an h beyond it: the int8 path takes them like any
+    other value, the fp16 path scales such rows by exact powers of two (and flags an h beyond
+    even that, |h| >= 2^32);
   * the block-FP8 path's requantized intermediate: its e4m3 codes and 1x128 scales against the
     oracle's, not only the layer output.
 Gates as in the other layer tests: max|err| <= 1e-2*RMS(ref) + 1e-3 (3e-2 for block-FP8).
@@ -128,51 +128,65 @@ def test_int8_path_takes_values_beyond_fp16():
 
 
 def _hot_layer(seed, T=200):
-    """Every token's only expert is expert 0 (T rows: the fp16 path)."""
+    """Every token's only expert is expert 0 (T rows: the fp16 GEMM)."""
     lg = synth.logits(seed, T, 8) * 0.1
     lg[:, 0] += 50.0
     return W4Layer(seed, T, 256, 128, 8, 1, logits=lg)
 
 
-def test_fp16_path_flags_inputs_beyond_its_range():
+def test_fp16_path_takes_inputs_beyond_fp16():
+    """Rows with values beyond the largest fp16 (65504) are scaled by an exact power of two to
+    fit and the accumulators scaled back; h then exceeds fp16 as well and is rescaled per row."""
     L = _hot_layer(52)
     x = bf16_bits_to_f32(L.x).copy()
-    x[5, 17] = 70000.0  # bf16 70144: above the largest finite fp16, 65504
+    x[5, 17] = 70000.0  # bf16 70144
+    x[9, :] *= 3.0e3    # every value of the row scaled; |h| ~ 1e7
+    x[77, 100] = -2.0e5
+    set_x(L, f32_to_bf16_bits(x))
+    run_and_check(L, "fp16 path, |x| up to 2e5")
+
+
+def test_fp16_path_takes_an_intermediate_beyond_fp16():
+    """Large gate/up weight scales: h = SiLU(gate) * up reaches 1e5 .. 1e7 for every token."""
+    L = _hot_layer(53)
+    L.W["w13_s"] = np.full_like(L.W["w13_s"], f32_to_bf16_bits(np.float32(8.0)))
+    L.w.d_w13_s = dev(L.W["w13_s"], torch.bfloat16)
+    ids_ref, w_ref, _ = oracle.route(L.lg, 1)
+    _, h = oracle.w4a16_tokens(L.x, ids_ref, w_ref, L.W["w13_q"], L.W["w13_s"], L.W["w2_q"], L.W["w2_s"],
+                               want_h=True)
+    assert np.abs(h).max() > 1e6
+    run_and_check(L, f"fp16 path, |h| up to {np.abs(h).max():.1e}")
+
+
+def test_fp16_path_flags_an_intermediate_beyond_its_prescaled_range():
+    """|h| >= 65520 * 2^16 (about 4.3e9) is beyond even the prescaled store: flagged."""
+    L = _hot_layer(55)
+    L.W["w13_s"] = np.full_like(L.W["w13_s"], f32_to_bf16_bits(np.float32(8.0)))
+    L.w.d_w13_s = dev(L.W["w13_s"], torch.bfloat16)
+    x = bf16_bits_to_f32(L.x).copy()
+    x[3, :] *= 1.0e4  # |g| ~ 1e7, h ~ 1e14
     set_x(L, f32_to_bf16_bits(x))
     ids, w = moe.moe_route(L.d_lg, 1)
     moe.moe_get_device_status()
     L.forward(moe, ids, w, out_fp32=True)
     assert moe.moe_get_device_status() == moe.MOE_ERR_DEVICE_CHECK
-    # the same layer with that value at 1000 (inside fp16, and h stays inside it too) runs clean
-    # and matches the oracle
-    x[5, 17] = 1000.0
-    set_x(L, f32_to_bf16_bits(x))
-    run_and_check(L, "fp16 path, |x| = 1000")
 
 
-def test_fp16_path_flags_an_intermediate_beyond_its_range():
-    L = _hot_layer(53)
-    big = np.full_like(L.W["w13_s"], f32_to_bf16_bits(np.float32(8.0)))  # |g| ~ 1e3, h ~ 1e5..1e6
-    d_s = L.w.d_w13_s
-    L.w.d_w13_s = dev(big, torch.bfloat16)
-    try:
-        ids, w = moe.moe_route(L.d_lg, 1)
-        moe.moe_get_device_status()
-        L.forward(moe, ids, w, out_fp32=True)
-        assert moe.moe_get_device_status() == moe.MOE_ERR_DEVICE_CHECK
-    finally:
-        L.w.d_w13_s = d_s
-
-
-def test_grouped_gemm_flags_inputs_beyond_fp16():
+def test_grouped_gemm_takes_inputs_beyond_fp16():
     M, K, N = 300, 256, 128  # M > 64: the fp16 path
     a, w_q, w_s = synth.gemm_operands(54, M, K, N)
     a = a.copy()
     a[100, 3] = f32_to_bf16_bits(np.float32(-1.0e5))
+    a[200, :] = f32_to_bf16_bits(bf16_bits_to_f32(a[200, :]) * np.float32(1.0e9))
+    off = np.array([0, M], np.int32)
     moe.moe_get_device_status()
-    moe.moe_w4a16_gemm(dev(a, torch.bfloat16), dev(w_q), dev(w_s, torch.bfloat16),
-                       dev(np.array([0, M], np.int32)), out_fp32=True)
-    assert moe.moe_get_device_status() == moe.MOE_ERR_DEVICE_CHECK
+    out = moe.moe_w4a16_gemm(dev(a, torch.bfloat16), dev(w_q), dev(w_s, torch.bfloat16), dev(off), out_fp32=True)
+    assert moe.moe_get_device_status() == 0
+    ref = oracle.w4a16_gemm(a, True, w_q, w_s, off)
+    got = out.double().cpu().numpy()
+    # rows are independent: check each scale of row against itself
+    for rows in (np.r_[0:100, 101:200, 201:M], [100], [200]):
+        check_tol(got[rows], ref[rows], what=f"grouped GEMM rows {rows[0]}..")
 
 
 # ---------------------------------------------------------------------- block-FP8 intermediate
