@@ -171,7 +171,7 @@ Planes take_planes(Carver& c, size_t rows, int K) {
 struct FwdWs {
   int32_t *counts, *offsets, *sorted, *inv, *blockcnt;
   int32_t *tile_prefix, *chunk, *row_count;                  // fp16 GEMM schedule (wide experts)
-  int32_t *thin_tile_prefix, *thin_chunk, *thin_row_count;   // int8 GEMM schedule
+  int32_t *thin_tile_prefix, *thin_chunk, *thin_row_count, *thin_row_prefix;  // int8 GEMM schedule
   __half *x_perm, *h;  // fp16 path rows
   int32_t *x_exp, *h_exp, *ovf_flag;  // fp16 path: per-row exponents and h overflow flags
   uint32_t* ovf_mask;                 // fp16 path: [P, I/32] h overflow marks
@@ -197,6 +197,7 @@ FwdWs carve_w4_forward(void* ws, int T, int H, int I, int E, int k) {
     w.chunk = c.take<int32_t>(E);
     w.row_count = c.take<int32_t>(E);
     w.thin_row_count = c.take<int32_t>(E);
+    w.thin_row_prefix = c.take<int32_t>(E + 1);
     w.x_perm = c.take<__half>(P * H);
     w.h = c.take<__half>(P * I);
     w.x_exp = c.take<int32_t>(P);
@@ -366,6 +367,7 @@ moe_status_t moe_w4a16_forward(const moe_w4a16_args* a, void* ws, size_t ws_byte
     so.thin_tile_prefix = w.thin_tile_prefix;
     so.thin_chunk = w.thin_chunk;
     so.thin_row_count = w.thin_row_count;
+    so.thin_row_prefix = w.thin_row_prefix;
   } else {  // every expert on the int8 GEMM: its schedule is the main one, row counts = counts
     so.nmax = kI8TileRows;
     so.tile_prefix = w.thin_tile_prefix;
@@ -378,9 +380,13 @@ moe_status_t moe_w4a16_forward(const moe_w4a16_args* a, void* ws, size_t ws_byte
   const uint16_t* w13_s = static_cast<const uint16_t*>(a->w13_s);
   const uint16_t* w2_s = static_cast<const uint16_t*>(a->w2_s);
   // activations of each class of experts in the form its GEMM reads
-  if (e == cudaSuccess)
-    e = launch_planes(x, 1, w.inv, mixed ? a->topk_ids : nullptr, mixed ? w.thin_row_count : nullptr, P, k, H, w.xq.x,
-                      w.xq.meta, stream);
+  if (e == cudaSuccess) {
+    if (mixed)  // the rows of the thin experts only: at most kThinRows per expert
+      e = launch_planes_list(x, w.thin_row_prefix, w.offsets, w.sorted, E, k, std::min(P, kThinRows * E), H, w.xq.x,
+                             w.xq.meta, stream);
+    else
+      e = launch_planes(x, 1, w.inv, P, k, H, w.xq.x, w.xq.meta, stream);
+  }
   if (e == cudaSuccess && mixed)
     e = launch_permute_w4(x, w.inv, a->topk_ids, w.row_count, T, k, H, w.x_perm, w.x_exp, w.ovf_flag, w.ovf_mask, I,
                           stream);
@@ -483,8 +489,7 @@ moe_status_t moe_w4a16_gemm(const void* a, int a_is_bf16, const int32_t* w_q, co
   const TileSched sched{expert_offsets, w.row_count, w.tile_prefix, w.chunk};
   if (use_i8(M)) {
     if (e == cudaSuccess)
-      e = launch_planes(static_cast<const uint16_t*>(a), a_is_bf16, nullptr, nullptr, nullptr, M, 1, K, w.aq.x,
-                        w.aq.meta, stream);
+      e = launch_planes(static_cast<const uint16_t*>(a), a_is_bf16, nullptr, M, 1, K, w.aq.x, w.aq.meta, stream);
     const int sp = gemm_splits(M, K, N);
     if (e == cudaSuccess) {
       W4I8Problem g{w_q, static_cast<const uint16_t*>(w_s), w.aq.x, w.aq.meta, M, K, E, N, false, 0, sched,

@@ -335,6 +335,13 @@ __global__ void __launch_bounds__(kThreads, 1)
     uint32_t ph = 0;
     for (int it = blockIdx.x; it < total; it += gridDim.x) {
       const Item I = decode_item(it, sprefix, p);
+      // the item's row exponents, loaded while the MMAs run: lane l holds rows l + 32j
+      int rexp[NMAX / 32];
+#pragma unroll
+      for (int j = 0; j < NMAX / 32; ++j) {
+        const int rr = lane + 32 * j;
+        rexp[j] = (p.acc_exp && rr < I.nvalid) ? __ldg(p.acc_exp + I.r0 + rr) : 0;
+      }
       if (!__all_sync(0xffffffffu, mbar_wait(&acc_full[acc], ph, abort_flag, lim))) break;
       tc_fence_after();
       const uint32_t tb = tmem_base + ((uint32_t)(ew * 32) << 16) + (uint32_t)(acc * C::ACC_COLS);
@@ -346,13 +353,14 @@ __global__ void __launch_bounds__(kThreads, 1)
         tmem_ld_wait();
         const int nv = min(16, I.nvalid - c0);
         if (p.acc_exp) {  // rows whose fp16 operand was scaled by 2^-e to fit fp16: undo it
+          int ej = rexp[0];  // the exponents of rows c0 .. c0+15 sit in register c0 / 32
+#pragma unroll
+          for (int j = 1; j < NMAX / 32; ++j) ej = (c0 >> 5) == j ? rexp[j] : ej;
 #pragma unroll
           for (int i = 0; i < 16; ++i) {
-            if (i < nv) {
-              const float sc = exp2_int(__ldg(p.acc_exp + I.r0 + c0 + i));
-              g[i] = __float_as_uint(__uint_as_float(g[i]) * sc);
-              if (GATED) u[i] = __float_as_uint(__uint_as_float(u[i]) * sc);
-            }
+            const float sc = exp2_int(__shfl_sync(0xffffffffu, ej, (c0 & 16) + i));
+            g[i] = __float_as_uint(__uint_as_float(g[i]) * sc);
+            if (GATED) u[i] = __float_as_uint(__uint_as_float(u[i]) * sc);
           }
         }
         if (GATED) {

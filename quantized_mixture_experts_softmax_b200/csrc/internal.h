@@ -42,6 +42,7 @@ struct SchedOut {
   int32_t* thin_tile_prefix = nullptr;
   int32_t* thin_chunk = nullptr;
   int32_t* thin_row_count = nullptr;
+  int32_t* thin_row_prefix = nullptr;  // [E+1] exclusive scan of thin_row_count
 };
 // blockcnt: [align_blocks * E] int32 scratch.  sched may be null (no scheduler).
 cudaError_t launch_align(const int32_t* ids, int T, int k, int E, int align, int32_t* counts, int32_t* offsets,
@@ -135,11 +136,15 @@ cudaError_t launch_w4i8_gemm(const W4I8Problem& p, cudaStream_t s);
 cudaError_t launch_reduce_splits(const float* part, int splits, int rows, int N, const int32_t* row_start,
                                  const int32_t* row_count, int E, void* out, int out_fp32, cudaStream_t s);
 // Planes of the K-vectors x_src: plane row r takes source row r (inv_pos == null, k == 1),
-// or for every pair p plane row inv_pos[p] takes source row p / k (with ids / cls_rows given,
-// only the pairs whose expert has cls_rows[ids[p]] > 0).
-cudaError_t launch_planes(const uint16_t* a, int a_is_bf16, const int32_t* inv_pos, const int32_t* ids,
-                          const int32_t* cls_rows, int n_pairs, int k, int K, int8_t* planes, int32_t* meta,
-                          cudaStream_t s);
+// or for every pair p plane row inv_pos[p] takes source row p / k.
+cudaError_t launch_planes(const uint16_t* a, int a_is_bf16, const int32_t* inv_pos, int n_pairs, int k, int K,
+                          int8_t* planes, int32_t* meta, cudaStream_t s);
+// Planes of the rows of the thin schedule's experts: row_prefix [E+1] is the exclusive scan of
+// their row counts, and list row j < row_prefix[E] <= max_rows is row j - row_prefix[e] of expert
+// e; its sorted row offsets[e] + j - row_prefix[e] takes source row sorted_ids[that row] / k.
+cudaError_t launch_planes_list(const uint16_t* x_bf16, const int32_t* row_prefix, const int32_t* offsets,
+                               const int32_t* sorted_ids, int E, int k, int max_rows, int K, int8_t* planes,
+                               int32_t* meta, cudaStream_t s);
 
 // block-FP8 grouped GEMM (gemm_fp8.cu)
 struct F8GemmProblem {

@@ -204,28 +204,13 @@ cudaError_t launch_permute_fp8(const uint8_t* x, const float* xs, const int32_t*
 // floor((X + 128) / 256) in [-64, 64] and lo in [-128, 127]; hi goes to plane row 2r, lo to
 // 2r+1, bytes in the order (0,2,4,6,1,3,5,7) of each 8-group (the order in which a packed INT4
 // word unpacks); the sum of X over every 32-K group (for the MMA's offset correction) and the
-// block scales go to the row's meta words.
-__global__ void __launch_bounds__(256) planes_kernel(const uint4* __restrict__ a, int a_is_bf16,
-                                                     const int32_t* __restrict__ inv_pos,
-                                                     const int32_t* __restrict__ ids,
-                                                     const int32_t* __restrict__ cls_rows, int n_pairs, int k, int K,
-                                                     uint2* __restrict__ planes, int32_t* __restrict__ meta) {
-  const int nblk = K / 128;
-  const size_t unit = (blockIdx.x * (size_t)blockDim.x + threadIdx.x) >> 4;  // (pair, block)
-  const int i = threadIdx.x & 15;                                             // 8-group within the block
-  const bool live = unit < (size_t)n_pairs * nblk;
-  const int p = live ? (int)(unit / nblk) : 0;
-  const int blk = live ? (int)(unit % nblk) : 0;
-  int r = live ? (inv_pos ? inv_pos[p] : p) : -1;
-  // a pair whose expert runs on the other GEMM (ids[p] is read only for a pair inv_pos placed)
-  if (r >= 0 && cls_rows && __ldg(cls_rows + __ldg(ids + p)) == 0) r = -1;
-  // a warp's two units are (pair, block) neighbours, nearly always of one pair: a warp with
-  // nothing to write leaves before any load or arithmetic
-  if (__all_sync(0xffffffffu, r < 0)) return;
-  const int src = p / k;
+// block scales go to the row's meta words.  Called by whole warps (two units of 16 lanes); a
+// lane with r < 0 takes part in the shuffles and writes nothing.
+__device__ __forceinline__ void planes_unit(const uint4* __restrict__ a, int a_is_bf16, int r, int src, int blk,
+                                            int i, int K, uint2* __restrict__ planes, int32_t* __restrict__ meta) {
   float x[8];
   float amax = 0.f;
-  if (live && r >= 0) {
+  if (r >= 0) {
     const uint4 v = __ldg(a + ((size_t)src * K + blk * 128 + 8 * i) / 8);
     const uint32_t w[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
@@ -257,7 +242,7 @@ __global__ void __launch_bounds__(256) planes_kernel(const uint4* __restrict__ a
   }
   sum += __shfl_xor_sync(0xffffffffu, sum, 1);
   sum += __shfl_xor_sync(0xffffffffu, sum, 2);  // 4 threads = one 32-K group
-  if (!live || r < 0) return;
+  if (r < 0) return;
   constexpr int ord[8] = {0, 2, 4, 6, 1, 3, 5, 7};
   uint32_t hb[2] = {0, 0}, lb[2] = {0, 0};
 #pragma unroll
@@ -276,14 +261,70 @@ __global__ void __launch_bounds__(256) planes_kernel(const uint4* __restrict__ a
   if (i == 0) m[8 + (blk & 1)] = __float_as_int(sc);
 }
 
-cudaError_t launch_planes(const uint16_t* a, int a_is_bf16, const int32_t* inv_pos, const int32_t* ids,
-                          const int32_t* cls_rows, int n_pairs, int k, int K, int8_t* planes, int32_t* meta,
-                          cudaStream_t s) {
+// every pair p: plane row inv_pos[p] from source row p / k (or, without inv_pos, row p from row p)
+__global__ void __launch_bounds__(256) planes_kernel(const uint4* __restrict__ a, int a_is_bf16,
+                                                     const int32_t* __restrict__ inv_pos, int n_pairs, int k, int K,
+                                                     uint2* __restrict__ planes, int32_t* __restrict__ meta) {
+  const int nblk = K / 128;
+  const size_t unit = (blockIdx.x * (size_t)blockDim.x + threadIdx.x) >> 4;  // (pair, block)
+  const int i = threadIdx.x & 15;                                             // 8-group within the block
+  const bool live = unit < (size_t)n_pairs * nblk;
+  const int p = live ? (int)(unit / nblk) : 0;
+  const int blk = live ? (int)(unit % nblk) : 0;
+  const int r = live ? (inv_pos ? inv_pos[p] : p) : -1;
+  planes_unit(a, a_is_bf16, r, p / k, blk, i, K, planes, meta);
+}
+
+cudaError_t launch_planes(const uint16_t* a, int a_is_bf16, const int32_t* inv_pos, int n_pairs, int k, int K,
+                          int8_t* planes, int32_t* meta, cudaStream_t s) {
   const size_t threads = (size_t)n_pairs * (K / 128) * 16;
   timing_before("planes", s);
   planes_kernel<<<(unsigned)((threads + 255) / 256), 256, 0, s>>>(reinterpret_cast<const uint4*>(a), a_is_bf16,
-                                                                  inv_pos, ids, cls_rows, n_pairs, k, K,
+                                                                  inv_pos, n_pairs, k, K,
                                                                   reinterpret_cast<uint2*>(planes), meta);
+  timing_after("planes", s);
+  return cudaGetLastError();
+}
+
+// the rows of a list of expert runs: list row j < row_prefix[E] is row j - row_prefix[e] of
+// expert e (row_prefix[e] <= j < row_prefix[e+1]), i.e. sorted row offsets[e] + j - row_prefix[e],
+// whose pair is sorted_ids of that row; the grid covers an upper bound of the list length
+__global__ void __launch_bounds__(256) planes_list_kernel(const uint4* __restrict__ a,
+                                                          const int32_t* __restrict__ row_prefix,
+                                                          const int32_t* __restrict__ offsets,
+                                                          const int32_t* __restrict__ sorted_ids, int E, int k, int K,
+                                                          uint2* __restrict__ planes, int32_t* __restrict__ meta) {
+  const int nblk = K / 128;
+  const size_t unit = (blockIdx.x * (size_t)blockDim.x + threadIdx.x) >> 4;  // (list row, block)
+  const int i = threadIdx.x & 15;
+  const int total = __ldg(row_prefix + E);
+  const int j = (int)(unit / nblk);
+  const int blk = (int)(unit % nblk);
+  if (__all_sync(0xffffffffu, j >= total)) return;
+  int r = -1, src = 0;
+  if (j < total) {
+    int lo = 0, hi = E;  // row_prefix[lo] <= j < row_prefix[hi]
+    while (hi - lo > 1) {
+      const int mid = (lo + hi) >> 1;
+      if (__ldg(row_prefix + mid) <= j)
+        lo = mid;
+      else
+        hi = mid;
+    }
+    r = __ldg(offsets + lo) + j - __ldg(row_prefix + lo);
+    src = __ldg(sorted_ids + r) / k;
+  }
+  planes_unit(a, 1, r, src, blk, i, K, planes, meta);
+}
+
+cudaError_t launch_planes_list(const uint16_t* x_bf16, const int32_t* row_prefix, const int32_t* offsets,
+                               const int32_t* sorted_ids, int E, int k, int max_rows, int K, int8_t* planes,
+                               int32_t* meta, cudaStream_t s) {
+  const size_t threads = (size_t)max_rows * (K / 128) * 16;
+  timing_before("planes", s);
+  planes_list_kernel<<<(unsigned)((threads + 255) / 256), 256, 0, s>>>(
+      reinterpret_cast<const uint4*>(x_bf16), row_prefix, offsets, sorted_ids, E, k, K,
+      reinterpret_cast<uint2*>(planes), meta);
   timing_after("planes", s);
   return cudaGetLastError();
 }

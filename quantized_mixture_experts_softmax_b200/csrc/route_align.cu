@@ -216,6 +216,11 @@ __global__ void __launch_bounds__(1024) align_scan_kernel(int32_t* __restrict__ 
         sch.thin_row_count[e] = c_thin;
       }
       if (e == 0) sch.thin_tile_prefix[E] = total;
+      if (sch.thin_row_prefix) {
+        const int rp = block_exclusive_scan(e < E ? c_thin : 0, warp_tot, &total);
+        if (e < E) sch.thin_row_prefix[e] = rp;
+        if (e == 0) sch.thin_row_prefix[E] = total;
+      }
     }
   }
 }

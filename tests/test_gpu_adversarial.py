@@ -60,7 +60,10 @@ def set_x(L, bits):
     L.d_x = dev(L.x, torch.bfloat16)
 
 
-def run_and_check(L, what, tokens=None, rel=1e-2):
+def run_and_check(L, what, tokens=None, rel=1e-2, own_rows=()):
+    """The layer gate on all tokens; tokens listed in own_rows (rows scaled up on purpose, whose
+    size would otherwise set RMS(ref) for everyone) are checked one by one against their own
+    RMS and left out of the common check.  Tokens are independent, so this is the same gate."""
     ids, w = moe.moe_route(L.d_lg, L.k)
     ids_ref, w_ref, _ = oracle.route(L.lg, L.k)
     assert np.array_equal(ids.cpu().numpy(), ids_ref), f"{what}: routing ids differ"
@@ -72,8 +75,12 @@ def run_and_check(L, what, tokens=None, rel=1e-2):
     g32, g16 = out32.double().cpu().numpy(), out16.float().cpu().numpy()
     if tokens is not None:
         g32, g16 = g32[tokens], g16[tokens]
-    e = check_tol(g32, ref, rel=rel, what=what + " fp32")
-    check_tol(g16, ref, rel=rel, bf16_out=True, what=what + " bf16")
+    rest = np.setdiff1d(np.arange(len(ref)), np.asarray(own_rows, int))
+    groups = [rest] + [[r] for r in own_rows]
+    e = 0.0
+    for rows in groups:
+        e = max(e, check_tol(g32[rows], ref[rows], rel=rel, what=f"{what} fp32 rows {rows[0]}.."))
+        check_tol(g16[rows], ref[rows], rel=rel, bf16_out=True, what=f"{what} bf16 rows {rows[0]}..")
     print(f"{what}: max|err|/rms = {e:.3e}")
     return e
 
@@ -124,7 +131,7 @@ def test_int8_path_takes_values_beyond_fp16():
     x[9, 200] = -3.0e7
     x[12, :128] *= 5.0e4
     set_x(L, f32_to_bf16_bits(x))
-    run_and_check(L, "int8 path, |x| up to 3e7")
+    run_and_check(L, "int8 path, |x| up to 3e7", own_rows=(3, 9, 12))
 
 
 def _hot_layer(seed, T=200):
@@ -143,7 +150,7 @@ def test_fp16_path_takes_inputs_beyond_fp16():
     x[9, :] *= 3.0e3    # every value of the row scaled; |h| ~ 1e7
     x[77, 100] = -2.0e5
     set_x(L, f32_to_bf16_bits(x))
-    run_and_check(L, "fp16 path, |x| up to 2e5")
+    run_and_check(L, "fp16 path, |x| up to 2e5", own_rows=(5, 9, 77))
 
 
 def test_fp16_path_takes_an_intermediate_beyond_fp16():
@@ -176,7 +183,7 @@ def test_grouped_gemm_takes_inputs_beyond_fp16():
     M, K, N = 300, 256, 128  # M > 64: the fp16 path
     a, w_q, w_s = synth.gemm_operands(54, M, K, N)
     a = a.copy()
-    a[100, 3] = f32_to_bf16_bits(np.float32(-1.0e5))
+    a[100, 3] = f32_to_bf16_bits(np.array([-1.0e5], np.float32))[0]
     a[200, :] = f32_to_bf16_bits(bf16_bits_to_f32(a[200, :]) * np.float32(1.0e9))
     off = np.array([0, M], np.int32)
     moe.moe_get_device_status()
