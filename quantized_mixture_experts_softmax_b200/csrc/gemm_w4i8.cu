@@ -57,26 +57,35 @@ constexpr int kUnpackWarp0 = 8;
 constexpr int kNumUnpack = 8;
 static_assert(NT == 8, "the promotion code handles up to 8 tokens per tile");
 
-template <bool GATED>
+// A work item covers NA weight tiles of 128 rows: the gate and up tiles of the same 128
+// columns of h (gate/up GEMM), or two adjacent 128-row tiles of the output (down GEMM, when the
+// output rows come in 256s; one tile otherwise).  A stage (256 K of an item) holds the NA INT4
+// weight tiles, then the token tile's activation atoms, its meta words and the NA tiles' weight
+// scales.  Per stage the pipeline pays a fixed cost (copies, hand-offs, TMEM slot cycles) besides
+// the bytes; two tiles per stage halve that cost per weight byte (measured on the down GEMM of
+// the decode layer: 16 KB stages ran at 0.55 of HBM bandwidth, 32 KB stages of gate/up at 0.88).
+template <bool GATED, int NA_>
 struct Cfg {
-  static constexpr int NA = GATED ? 2 : 1;
-  static constexpr int SG = GATED ? 4 : 8;  // groups per D slot (SG * NA MMAs per handoff)
+  static_assert(NA_ == 1 || NA_ == 2, "one or two weight tiles per item");
+  static_assert(!GATED || NA_ == 2, "gate and up tiles");
+  static constexpr int NA = NA_;
+  static constexpr int SG = NA == 2 ? 4 : 8;  // groups per D slot (SG * NA MMAs per handoff)
   static constexpr int W_TILE = BM * KB / 2;   // INT4 bytes
-  static constexpr int B_ATOM = 2 * NT * 128;  // one 128-K atom of the 2*NT plane rows
   static constexpr int STAGE_B = NA * W_TILE;
+  static constexpr int B_ATOM = 2 * NT * 128;  // one 128-K atom of the 2*NT plane rows
   static constexpr int META = STAGE_B + (KB / 128) * B_ATOM;  // [NT tokens][kMetaWords] int32
   static constexpr int META_BYTES = NT * kMetaWords * 4;
   static constexpr int SCL = META + 1024;            // [NA][BM rows][NG] bf16 weight scales
   static constexpr int S_TILE = BM * NG * 2;
   static constexpr int STAGE = SCL + NA * S_TILE;
   static_assert(META_BYTES <= 1024, "meta box fits its slot");
-  static constexpr int ST = GATED ? 5 : 9;
+  static constexpr int ST = NA == 2 ? 5 : 9;
   // TMEM: D ring of SG-group slots [group][matrix][DC int32 columns], A ring of whole-stage
   // slots [matrix][group][8 columns] (a 32-K row of u8 = 8 columns)
   static constexpr int D_SLOT = SG * NA * DC;
   static constexpr int DSLOTS = 256 / D_SLOT;
   static constexpr int A_SLOT = NA * NG * 8;
-  static constexpr int ASLOTS = GATED ? 2 : 4;
+  static constexpr int ASLOTS = NA == 2 ? 2 : 4;
   static constexpr int A_COL0 = DSLOTS * D_SLOT;
   static_assert(A_COL0 + ASLOTS * A_SLOT <= 512, "TMEM has 512 columns");
   static constexpr int OFF_BAR = ST * STAGE;
@@ -91,6 +100,7 @@ struct Cfg {
 
 struct Params {
   int K, E, rows_per_expert, I, m_tiles;
+  int row_off2;          // NA = 2: rows of the second tile after the first (I for gate/up, 128 for down)
   const uint16_t* w_s;   // bf16 [E*rows_per_expert, K/32]
   int scales_tma;        // 1: weight scales by TMA (K % 256 == 0), else by cp.async
   TileSched sched;
@@ -191,7 +201,8 @@ struct Promo {
 // Tokens [0, NP) of one D slot (groups g0 .. g0+SG-1 x NA matrices, the first `ngs` of them
 // present): loads their 2*NP columns of every (group, matrix) in batches of at most 32
 // registers, one wait per batch.  swg/swu: weight scales of this thread's rows per group;
-// meta: the stage's meta words per token.
+// meta: the stage's meta words per token.  (Handing the slot back right after the last batch
+// is in registers, before the arithmetic, measured 4-5% slower on the decode gate/up GEMM.)
 template <int NA, int SG, int NP>
 __device__ __forceinline__ void promote_slot(uint32_t slot_addr, const int* meta, int g0, int ngs,
                                              const float (&swg)[SG], const float (&swu)[SG], Promo<NP>& P) {
@@ -232,13 +243,13 @@ __device__ __forceinline__ float bf16_at(const uint4& v, int g) {
 }
 
 // The K loop of one work item for the promotion warps, specialised on the live-token bound NP.
-template <bool GATED, int NP>
+template <bool GATED, int NA_, int NP>
 __device__ __forceinline__ bool promote_item(const Params& p, const Item& I, int mrow, int lane, uint32_t lane_base,
                                              const uint8_t* smem, int& s, uint32_t& ph, uint64_t* full,
                                              uint64_t* empty, int& ds, uint32_t& ph_d, uint64_t* d_full,
                                              uint64_t* d_empty, volatile int* abort_flag, int kb0, int kb1,
                                              Promo<NP>& P) {
-  using C = Cfg<GATED>;
+  using C = Cfg<GATED, NA_>;
   constexpr int NA = C::NA, DSL = C::DSLOTS, ST = C::ST, SG = C::SG;
   const int K = p.K;
   const uint64_t lim = p.wait_limit;
@@ -250,7 +261,7 @@ __device__ __forceinline__ bool promote_item(const Params& p, const Item& I, int
     const uint8_t* st = smem + s * C::STAGE;
     const int* meta = reinterpret_cast<const int*>(st + C::META);
     const uint4 sgv = *reinterpret_cast<const uint4*>(st + C::SCL + mrow * 16);
-    const uint4 suv = GATED ? *reinterpret_cast<const uint4*>(st + C::SCL + C::S_TILE + mrow * 16) : sgv;
+    const uint4 suv = NA == 2 ? *reinterpret_cast<const uint4*>(st + C::SCL + C::S_TILE + mrow * 16) : sgv;
 #pragma unroll
     for (int g0 = 0; g0 < NG; g0 += SG) {  // unrolled: scale registers are indexed statically
       if (g0 >= ng) break;
@@ -272,7 +283,7 @@ __device__ __forceinline__ bool promote_item(const Params& p, const Item& I, int
       }
     }
     __syncwarp();
-    if (lane == 0) mbar_arrive(&empty[s]);  // meta words read
+    if (lane == 0) mbar_arrive(&empty[s]);  // meta words and scales read, the stage's MMAs done
     if (++s == ST) {
       s = 0;
       ph ^= 1u;
@@ -282,8 +293,9 @@ __device__ __forceinline__ bool promote_item(const Params& p, const Item& I, int
 }
 
 // One work item of the promotion warps: the K loop, then the epilogue (GATED: h = SiLU(gate)
-// * up as fixed-point planes with one scale per (token, tile); else fp32 or bf16 rows).
-template <bool GATED, int NP>
+// * up as fixed-point planes with one scale per (token, tile); else fp32 or bf16 rows of the
+// item's NA tiles).
+template <bool GATED, int NA_, int NP>
 __device__ __forceinline__ bool epi_item(const Params& p, const Item& I, int it, int ew, int lane, uint32_t lane_base,
                                          const uint8_t* smem, int& s, uint32_t& ph, uint64_t* full, uint64_t* empty,
                                          int& ds, uint32_t& ph_d, uint64_t* d_full, uint64_t* d_empty,
@@ -294,8 +306,8 @@ __device__ __forceinline__ bool epi_item(const Params& p, const Item& I, int it,
   for (int c = 0; c < NP; ++c) P.ag[c] = P.au[c] = 0.f;
   int kb0, kb1;
   split_range(it, ceil_div(p.K, KB), p.splits, kb0, kb1);
-  if (!promote_item<GATED, NP>(p, I, mrow, lane, lane_base, smem, s, ph, full, empty, ds, ph_d, d_full, d_empty,
-                               abort_flag, kb0, kb1, P))
+  if (!promote_item<GATED, NA_, NP>(p, I, mrow, lane, lane_base, smem, s, ph, full, empty, ds, ph_d, d_full,
+                                    d_empty, abort_flag, kb0, kb1, P))
     return false;
   if constexpr (GATED) {
 #pragma unroll
@@ -333,33 +345,36 @@ __device__ __forceinline__ bool epi_item(const Params& p, const Item& I, int it,
     }
     return epi_sync(epi_bar, ph_e, abort_flag, p.wait_limit);  // red[] is reused by the next item
   } else {
-    const int n = I.m * BM + mrow;
-    if (p.splits > 1) {  // this split's partial sum, reduced in split order by another kernel
-      float* y = p.part + (size_t)(it % p.splits) * p.act_rows * p.out_ld;
 #pragma unroll
-      for (int c = 0; c < NP; ++c)
-        if (c < nv) y[(size_t)(I.r0 + c) * p.out_ld + n] = P.ag[c];
-    } else if (p.out_kind == OUT_F32) {
-      float* y = reinterpret_cast<float*>(p.out);
+    for (int mat = 0; mat < NA_; ++mat) {
+      const int n = I.m * (NA_ * BM) + mat * BM + mrow;
+      if (p.splits > 1) {  // this split's partial sum, reduced in split order by another kernel
+        float* y = p.part + (size_t)(it % p.splits) * p.act_rows * p.out_ld;
 #pragma unroll
-      for (int c = 0; c < NP; ++c)
-        if (c < nv) y[(size_t)(I.r0 + c) * p.out_ld + n] = P.ag[c];
-    } else {
-      __nv_bfloat16* y = reinterpret_cast<__nv_bfloat16*>(p.out);
+        for (int c = 0; c < NP; ++c)
+          if (c < nv) y[(size_t)(I.r0 + c) * p.out_ld + n] = mat ? P.au[c] : P.ag[c];
+      } else if (p.out_kind == OUT_F32) {
+        float* y = reinterpret_cast<float*>(p.out);
 #pragma unroll
-      for (int c = 0; c < NP; ++c)
-        if (c < nv) y[(size_t)(I.r0 + c) * p.out_ld + n] = __float2bfloat16_rn(P.ag[c]);
+        for (int c = 0; c < NP; ++c)
+          if (c < nv) y[(size_t)(I.r0 + c) * p.out_ld + n] = mat ? P.au[c] : P.ag[c];
+      } else {
+        __nv_bfloat16* y = reinterpret_cast<__nv_bfloat16*>(p.out);
+#pragma unroll
+        for (int c = 0; c < NP; ++c)
+          if (c < nv) y[(size_t)(I.r0 + c) * p.out_ld + n] = __float2bfloat16_rn(mat ? P.au[c] : P.ag[c]);
+      }
     }
     return true;
   }
 }
 
-template <bool GATED>
+template <bool GATED, int NA_>
 __global__ void __launch_bounds__(kThreads, 1)
     w4i8_gemm_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CUtensorMap tm_x,
                      const __grid_constant__ CUtensorMap tm_m, const __grid_constant__ CUtensorMap tm_s,
                      const Params p) {
-  using C = Cfg<GATED>;
+  using C = Cfg<GATED, NA_>;
   constexpr int NA = C::NA, ST = C::ST, ASL = C::ASLOTS, DSL = C::DSLOTS, SG = C::SG;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -428,8 +443,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     bool ok = true;
     for (int it = blockIdx.x; it < total && ok; it += gridDim.x) {
       const Item I = decode_item(it, sprefix, p);
-      const int row_g = I.e * p.rows_per_expert + I.m * BM;
-      const int row_u = row_g + p.I;
+      const int row_g = I.e * p.rows_per_expert + I.m * (GATED ? BM : NA * BM);  // first tile
+      const int row_u = row_g + p.row_off2;                                      // second tile
       int kb0, kb1;
       split_range(it, nkb, p.splits, kb0, kb1);
       for (int kb = kb0; kb < kb1; ++kb) {
@@ -441,13 +456,13 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (p.scales_tma) bytes += NA * C::S_TILE;
           mbar_arrive_expect_tx(&full[s], bytes);
           tma_load_2d_hint(st, &tm_w, &full[s], kb * (KB / 8), row_g, pol_w);
-          if (GATED) tma_load_2d_hint(st + C::W_TILE, &tm_w, &full[s], kb * (KB / 8), row_u, pol_w);
+          if (NA == 2) tma_load_2d_hint(st + C::W_TILE, &tm_w, &full[s], kb * (KB / 8), row_u, pol_w);
           for (int a = 0; a < natom; ++a)
             tma_load_2d_hint(st + C::STAGE_B + a * C::B_ATOM, &tm_x, &full[s], kb * KB + a * 128, 2 * I.r0, pol_b);
           tma_load_2d_hint(st + C::META, &tm_m, &full[s], kb * kMetaWords, I.r0, pol_b);
           if (p.scales_tma) {
             tma_load_2d_hint(st + C::SCL, &tm_s, &full[s], kb * NG, row_g, pol_w);
-            if (GATED) tma_load_2d_hint(st + C::SCL + C::S_TILE, &tm_s, &full[s], kb * NG, row_u, pol_w);
+            if (NA == 2) tma_load_2d_hint(st + C::SCL + C::S_TILE, &tm_s, &full[s], kb * NG, row_u, pol_w);
           }
         }
         if (!p.scales_tma) {  // scale rows 8-byte aligned: 8 or 4 bf16 per row by cp.async
@@ -582,8 +597,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       const Item I = decode_item(it, sprefix, p);
       const int nv = I.nvalid;
 #define MOE_EPI_ITEM(NP_)                                                                                           \
-  epi_item<GATED, NP_>(p, I, it, ew, lane, lane_base, smem, s, ph, full, empty, ds, ph_d, d_full, d_empty, red, epi_bar, \
-                       ph_e, abort_flag)
+  epi_item<GATED, NA_, NP_>(p, I, it, ew, lane, lane_base, smem, s, ph, full, empty, ds, ph_d, d_full, d_empty, red,  \
+                            epi_bar, ph_e, abort_flag)
       if (nv <= 1)
         ok = MOE_EPI_ITEM(1);
       else if (nv <= 2)
@@ -596,14 +611,14 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   } else if (warp >= kUnpackWarp0) {
     // ---------------------------------------------------------------- INT4 -> u8 rows of TMEM
-    // GATED: warps 8-11 gate rows, 12-15 up rows, a thread = a row, the whole stage;
-    // plain: a thread = a row and one 128-K half of the stage.
+    // two tiles: warps 8-11 rows of the first (gate) tile, 12-15 of the second (up), a thread =
+    // a row, the whole stage; one tile: a thread = a row and one 128-K half of the stage.
     const int uw = warp - kUnpackWarp0;
     const int row = (uw & 3) * 32 + lane;
     const int sw = row & 7;
-    const int mat = GATED ? (uw >> 2) : 0;
-    const int half = GATED ? 0 : (uw >> 2);
-    constexpr int CHK = GATED ? 8 : 4;  // 16-byte chunks (32 K each) this thread unpacks per stage
+    const int mat = NA == 2 ? (uw >> 2) : 0;
+    const int half = NA == 2 ? 0 : (uw >> 2);
+    constexpr int CHK = NA == 2 ? 8 : 4;  // 16-byte chunks (32 K each) this thread unpacks per stage
     const uint32_t lane_base = tmem_base + ((uint32_t)((uw & 3) * 32) << 16);
     int s = 0, as = 0;
     uint32_t ph = 0, ph_a = 0;
@@ -619,7 +634,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         uint4 wv[CHK];
 #pragma unroll
         for (int c = 0; c < CHK; ++c) {
-          const int lc = GATED ? c : 4 * half + c;  // logical 16-byte chunk = 32-K group
+          const int lc = NA == 2 ? c : 4 * half + c;  // logical 16-byte chunk = 32-K group
           wv[c] = *reinterpret_cast<const uint4*>(wrow + ((lc ^ sw) << 4));
         }
         __syncwarp();
@@ -644,8 +659,8 @@ __global__ void __launch_bounds__(kThreads, 1)
             r[c * 8 + 2 * w + 1] = (n >> 4) & 0x0F0F0F0Fu;
           }
         }
-        const uint32_t col0 = (uint32_t)(C::A_COL0 + as * C::A_SLOT + mat * NG * 8 + (GATED ? 0 : half * 32));
-        if constexpr (GATED) {
+        const uint32_t col0 = (uint32_t)(C::A_COL0 + as * C::A_SLOT + mat * NG * 8 + (NA == 2 ? 0 : half * 32));
+        if constexpr (NA == 2) {
           uint32_t r0[32], r1[32];
 #pragma unroll
           for (int i = 0; i < 32; ++i) r0[i] = r[i], r1[i] = r[32 + i];
@@ -677,9 +692,9 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
 }
 
-template <bool GATED>
+template <bool GATED, int NA_>
 cudaError_t launch_t(const W4I8Problem& pr, cudaStream_t s) {
-  using C = Cfg<GATED>;
+  using C = Cfg<GATED, NA_>;
   CUtensorMap tm_w, tm_x, tm_m, tm_s;
   const uint64_t wrows = (uint64_t)pr.E * pr.rows_per_expert;
   if (encode_tmap_2d(&tm_w, pr.w_q, CU_TENSOR_MAP_DATA_TYPE_INT32, pr.K / 8, wrows, (uint64_t)pr.K / 2, KB / 8, BM,
@@ -706,7 +721,8 @@ cudaError_t launch_t(const W4I8Problem& pr, cudaStream_t s) {
   p.E = pr.E;
   p.rows_per_expert = pr.rows_per_expert;
   p.I = pr.I;
-  p.m_tiles = GATED ? pr.I / BM : pr.rows_per_expert / BM;
+  p.m_tiles = GATED ? pr.I / BM : pr.rows_per_expert / (NA_ * BM);
+  p.row_off2 = GATED ? pr.I : BM;
   p.w_s = pr.w_s;
   p.sched = pr.sched;
   p.out_kind = pr.out_kind;
@@ -718,7 +734,7 @@ cudaError_t launch_t(const W4I8Problem& pr, cudaStream_t s) {
   p.act_rows = pr.act_rows;
   p.wait_limit = wait_limit_ns();
   const size_t smem = C::smem_bytes(pr.E);
-  auto kern = w4i8_gemm_kernel<GATED>;
+  auto kern = w4i8_gemm_kernel<GATED, NA_>;
   cudaError_t err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (err != cudaSuccess) return err;
   const char* name = GATED ? "w4i8_gemm_gate_up" : "w4i8_gemm_down";
@@ -730,8 +746,12 @@ cudaError_t launch_t(const W4I8Problem& pr, cudaStream_t s) {
 
 }  // namespace w4i8
 
+int w4i8_tiles_per_item(bool gated, int rows_per_expert) { return gated || rows_per_expert % 256 == 0 ? 2 : 1; }
+
 cudaError_t launch_w4i8_gemm(const W4I8Problem& p, cudaStream_t s) {
-  return p.gated ? w4i8::launch_t<true>(p, s) : w4i8::launch_t<false>(p, s);
+  if (p.gated) return w4i8::launch_t<true, 2>(p, s);
+  return w4i8_tiles_per_item(false, p.rows_per_expert) == 2 ? w4i8::launch_t<false, 2>(p, s)
+                                                            : w4i8::launch_t<false, 1>(p, s);
 }
 
 }  // namespace moe
