@@ -145,7 +145,7 @@ bool use_i8(int max_rows_per_expert) { return max_rows_per_expert <= 64; }
 
 // Larger layer calls choose per expert, from its actual token count: an expert with at most
 // kThinRows rows runs on the int8 GEMM (8-row token tiles; its cost is streaming the weights
-// plus a promotion step per live token), one with more on the fp16 GEMM (tiles of up to 256
+// plus a promotion step per live token), one with more on the fp16 GEMM (tiles of up to 192
 // rows, where dequantizing a weight tile once serves many tokens, but a tile of few tokens
 // costs as much dequantization as a full one).  Measured on the 384-expert model with skewed
 // routing at T = 128 ... 8192, switch points of 16, 32, 48 and 64 rows: 16 was fastest at
@@ -154,7 +154,6 @@ bool use_i8(int max_rows_per_expert) { return max_rows_per_expert <= 64; }
 #define MOE_THIN_ROWS 16
 #endif
 constexpr int kThinRows = MOE_THIN_ROWS;
-constexpr int kWideTileRows = 256;
 
 // 16-bit fixed-point planes of an activation matrix [rows, K]
 struct Planes {
@@ -214,7 +213,7 @@ FwdWs carve_w4_forward(void* ws, int T, int H, int I, int E, int k) {
 // so that items x splits ~ 148 (at least one 256-K stage per split, at most 32 splits); a
 // shape-only rule, so the workspace size needs no device.
 int gemm_splits(int M, int K, int N) {
-  const int tile_rows = use_i8(M) ? kI8TileRows : 256;
+  const int tile_rows = use_i8(M) ? kI8TileRows : kWideTileRows;
   const int weight_rows = use_i8(M) ? 128 * w4i8_tiles_per_item(false, N) : 128;  // per work item
   const int nkb = (K + 255) / 256;
   const int items = (N / weight_rows) * ((M + tile_rows - 1) / tile_rows);

@@ -1,8 +1,8 @@
-// a5-a7 for prefill-sized experts: W4A16 grouped expert GEMM on the 5th-generation tensor
+// a5-a7 for experts with many rows: W4A16 grouped expert GEMM on the 5th-generation tensor
 // cores (tcgen05 kind::f16, sm_100a).
 //
 // One persistent CTA per SM walks a static round-robin list of work items.  An item is
-// (expert e, weight tile m of 128 output rows, token tile t of up to NMAX = 256 activation
+// (expert e, weight tile m of 128 output rows, token tile t of up to NMAX = 192 activation
 // rows); the item list is ordered expert-major, then weight tile, then token tile, so that CTAs
 // running at the same time share weight tiles through L2 when an expert has several token
 // tiles.  The MMA runs "swapped": the 128 weight rows are the M operand and the token rows the
@@ -11,21 +11,33 @@
 // transposition of the AWS and Helion articles, on tcgen05's M=128 instead of Hopper's 64-row
 // WGMMA).
 //
-// Warp roles (512 threads):
-//   warp 0      idle after setup;
-//   warp 1      TMEM allocator and single-thread tcgen05.mma issuer; it never waits on an
-//               mbarrier (see bar_red_and) and is released step by step by
+// The dequantized weights (the MMA's A operand) live in tensor memory, not shared memory: per
+// 64-K step a 128-row fp16 tile staged in shared memory would be written once and read once per
+// matrix, which next to the activation tile's copy and two reads asks more of shared memory than
+// it delivers; from tensor memory the MMA reads A without touching it.  The accumulators and the
+// A ring then share the 512 TMEM columns, which sets the token tile to 192 rows.
+//
+// Warp roles (512 threads, 544 for the gate/up GEMM):
+//   warp 0      TMA producer of the packed INT4 weight tiles (NA x 128 rows x 256 K, 128-byte
+//               swizzle) and their bf16 scales (TMA; cp.async when a scale row is not 16-byte
+//               aligned), WST-deep ring of 256-K stages;
+//   warp 1      TMEM allocator and single-thread tcgen05.mma issuer (A from tensor memory, B
+//               from shared memory) of the gate (or only) matrix, and for the gate/up GEMM
+//   warp 16     the issuer of the up matrix's MMAs: a thread with MMAs in flight stalls at its
+//               next synchronisation until they drain, so with one issuer the tensor core idles
+//               at every step's hand-off; with two, one's MMAs run while the other waits.  The
+//               issuers never wait on an mbarrier (see bar_red_and) and are released step by
+//               step by
 //   warp 2      the MMA scheduler, which waits for the accumulator, the dequantized A tile and
 //               the activation tile of each 64-K step;
 //   warp 3      TMA producer of the fp16 activation tiles (N rows x 64 K), BST-deep ring;
-//   warps 4-7   epilogue: tcgen05.ld of the fp32 accumulators, SiLU(gate)*up for the gate/up
-//               GEMM (fp16 h) or a plain store (fp32 / bf16) for the down GEMM;
-//   warps 8-15  dequantization: each thread loads its weight row's packed INT4 words and bf16
-//               scales straight from global memory into registers one 256-K stage ahead (the
-//               weights are read once, so staging them in shared memory bought nothing and
-//               took the room the activation ring needs), and writes INT4 -> fp16 = q * s
-//               exactly (|q| <= 8 has 3 significant bits, a bf16 scale 8, fp16 holds 11) in
-//               the 128-byte swizzled K-major layout the MMA reads, ABUF-deep per 64-K step.
+//   warps 4-7   epilogue: tcgen05.ld of the fp32 accumulators, times each row's power-of-two
+//               exponent, SiLU(gate)*up for the gate/up GEMM (fp16 h) or a plain store (fp32 /
+//               bf16) for the down GEMM;
+//   warps 8-15  dequantization: each thread copies its weight row's words and scales of a stage
+//               into registers (freeing the stage at once), then per 64-K step writes
+//               INT4 -> fp16 = q * s exactly (|q| <= 8 has 3 significant bits, a bf16 scale 8,
+//               fp16 holds 11) into an A slot of tensor memory (tcgen05.st), ABUF-deep.
 // The gate/up GEMM keeps two accumulators (gate rows m*128.., up rows I+m*128..) so each
 // epilogue thread holds gate_j and up_j of the same j.
 //
@@ -36,46 +48,57 @@
 namespace moe {
 namespace w4 {
 
-constexpr int BM = 128;    // weight rows per tile (MMA M)
-constexpr int KB = 256;    // K per weight stage
-constexpr int KS = 64;     // K per MMA step (one 128-byte swizzle atom of fp16)
-constexpr int NMAX = 256;  // token rows per tile
+constexpr int BM = 128;             // weight rows per tile (MMA M)
+constexpr int KB = 256;             // K per weight stage
+constexpr int KS = 64;              // K per MMA step (one 128-byte swizzle atom of fp16)
+constexpr int NMAX = kWideTileRows; // token rows per tile
+constexpr int kWProdWarp = 0;
 constexpr int kMmaWarp = 1;
 constexpr int kSchedWarp = 2;
 constexpr int kActWarp = 3;
 constexpr int kEpiWarp0 = 4;  // warps 4-7: epilogue
 constexpr int kDqWarp0 = 8;   // warps 8-15: dequantization
 constexpr int kNumDq = 8;
-constexpr int kThreads = (kDqWarp0 + kNumDq) * 32;
-constexpr int kMmaBarrier = 1;  // named barrier of the MMA and scheduler warps (0 is __syncthreads)
+constexpr int kMmaWarpUp = kDqWarp0 + kNumDq;  // warp 16 (gate/up GEMM only)
+template <bool GATED>
+constexpr int threads() { return (kDqWarp0 + kNumDq + (GATED ? 1 : 0)) * 32; }
+constexpr int kMmaBarrier = 1;  // named barriers 1 (gate/only) and 2 (up) of an MMA warp and the
+                                // scheduler warp (0 is __syncthreads)
+static_assert(NMAX % 32 == 0 && NMAX <= 256, "token tile");
 
 template <bool GATED>
 struct Cfg {
   static constexpr int NA = GATED ? 2 : 1;
-  // ring depths: activation tiles, dequantized A tiles
-  static constexpr int BST = GATED ? 3 : 5;
-  static constexpr int ABUF = GATED ? 3 : 2;
   static constexpr int NSUB = KB / KS;               // 64-K steps per weight stage
-  static constexpr int A_TILE = BM * KS * 2;         // dequantized fp16 operand
+  static constexpr int W_TILE = BM * KB / 2;         // packed INT4 bytes of one 128-row tile
+  static constexpr int S_TILE = BM * (KB / 32) * 2;  // its bf16 scales
+  static constexpr int W_STAGE = NA * (W_TILE + S_TILE);
   static constexpr int B_ATOM = NMAX * KS * 2;       // activation tile of one 64-K step
+  // ring depths: weight stages, activation tiles, A slots in tensor memory
+  static constexpr int WST = GATED ? 3 : 4;
+  static constexpr int BST = GATED ? 4 : 6;
+  static constexpr int ABUF = GATED ? 2 : 4;
   static constexpr int ACC_COLS = NA * NMAX;         // [matrix][NMAX] fp32 columns
-  static constexpr int ACC_BUFS = (2 * ACC_COLS <= 512) ? 2 : 1;
-  static constexpr int TMEM_COLS = 512;
-  static constexpr int OFF_A = 0;
-  static constexpr int OFF_B = OFF_A + ABUF * NA * A_TILE;
+  static constexpr int ACC_BUFS = (2 * ACC_COLS + ABUF * NA * (KS / 2) <= 512) ? 2 : 1;
+  static constexpr int A_COLS = KS / 2;              // a 64-K fp16 row of one tile = 32 TMEM columns
+  static constexpr int A_COL0 = ACC_BUFS * ACC_COLS; // first TMEM column of the A ring
+  static constexpr int OFF_W = 0;
+  static constexpr int OFF_B = OFF_W + WST * W_STAGE;
   static constexpr int OFF_BAR = OFF_B + BST * B_ATOM;
-  static constexpr int NUM_BARS = 2 * BST + 2 * ABUF + 2 * ACC_BUFS + 1;
+  static constexpr int NUM_BARS = 2 * WST + 2 * BST + 2 * ABUF + 2 * ACC_BUFS + 1;
   static constexpr int OFF_MISC = OFF_BAR + NUM_BARS * 8;
   static constexpr int OFF_PREFIX = OFF_MISC + 16;
-  static_assert(OFF_A % 1024 == 0 && OFF_B % 1024 == 0, "swizzled tiles need 1024-byte alignment");
-  static_assert(ACC_BUFS * ACC_COLS <= TMEM_COLS, "TMEM has 512 columns");
-  static constexpr size_t smem_bytes(int E) { return (size_t)OFF_PREFIX + 4 * (size_t)(E + 1) + 1024; }
+  static_assert(W_STAGE % 1024 == 0 && W_TILE % 1024 == 0 && OFF_B % 1024 == 0 && B_ATOM % 1024 == 0,
+                "swizzled tiles need 1024-byte alignment");
+  static_assert(A_COL0 + ABUF * NA * A_COLS <= 512, "TMEM has 512 columns");
+  // then the tile prefix [E+1] and the epilogue warps' row exponents [4][NMAX]
+  static constexpr size_t smem_bytes(int E) { return (size_t)OFF_PREFIX + 4 * (size_t)(E + 1 + 4 * NMAX) + 1024; }
   static_assert(smem_bytes(1024) <= 232448, "shared memory budget");
 };
 
 struct Params {
   int K, E, rows_per_expert, I, m_tiles;
-  const int32_t* w_q;
+  int scales_tma;  // 1: weight scales by TMA (K % 256 == 0), else by cp.async
   const uint16_t* w_s;
   TileSched sched;
   void* out;
@@ -162,14 +185,17 @@ __device__ __forceinline__ int interleave_pos(int j) {
 }
 
 template <bool GATED>
-__global__ void __launch_bounds__(kThreads, 1)
-    w4a16_gemm_kernel(const __grid_constant__ CUtensorMap tm_b, const __grid_constant__ CUtensorMap tm_b128,
+__global__ void __launch_bounds__(threads<GATED>(), 1)
+    w4a16_gemm_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CUtensorMap tm_s,
+                      const __grid_constant__ CUtensorMap tm_b, const __grid_constant__ CUtensorMap tm_b128,
                       const Params p) {
   using C = Cfg<GATED>;
-  constexpr int NA = C::NA, BST = C::BST, ABUF = C::ABUF, ACCB = C::ACC_BUFS, NSUB = C::NSUB;
+  constexpr int NA = C::NA, WST = C::WST, BST = C::BST, ABUF = C::ABUF, ACCB = C::ACC_BUFS, NSUB = C::NSUB;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  uint64_t* full_b = reinterpret_cast<uint64_t*>(smem + C::OFF_BAR);
+  uint64_t* full_w = reinterpret_cast<uint64_t*>(smem + C::OFF_BAR);
+  uint64_t* empty_w = full_w + WST;
+  uint64_t* full_b = empty_w + WST;
   uint64_t* empty_b = full_b + BST;
   uint64_t* a_full = empty_b + BST;
   uint64_t* a_empty = a_full + ABUF;
@@ -185,28 +211,35 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   for (int i = threadIdx.x; i <= p.E; i += blockDim.x) sprefix[i] = __ldg(p.sched.tile_prefix + i);
   if (threadIdx.x == 0) {
+    for (int i = 0; i < WST; ++i) {
+      mbar_init(&full_w[i], p.scales_tma ? 1 : 1 + 32);
+      mbar_init(&empty_w[i], kNumDq);
+    }
     for (int i = 0; i < BST; ++i) {
       mbar_init(&full_b[i], 1);
-      mbar_init(&empty_b[i], 1);
+      mbar_init(&empty_b[i], NA);
     }
+    // the A slot, the activation tile and the accumulator are released by a commit of each MMA warp
     for (int i = 0; i < ABUF; ++i) {
       mbar_init(&a_full[i], kNumDq);
-      mbar_init(&a_empty[i], 1);
+      mbar_init(&a_empty[i], NA);
     }
     for (int i = 0; i < ACCB; ++i) {
-      mbar_init(&acc_full[i], 1);
+      mbar_init(&acc_full[i], NA);
       mbar_init(&acc_empty[i], 4);
     }
-    mbar_init(drain, 1);
+    mbar_init(drain, NA);
     *abort_flag = 0;
     fence_mbar_init();
   }
   if (warp == 0 && lane == 0) {
+    prefetch_tmap(&tm_w);
+    if (p.scales_tma) prefetch_tmap(&tm_s);
     prefetch_tmap(&tm_b);
     prefetch_tmap(&tm_b128);
   }
   if (warp == kMmaWarp) {
-    tmem_alloc(tmem_slot, C::TMEM_COLS);
+    tmem_alloc(tmem_slot, 512);
     tmem_relinquish();
   }
   tc_fence_before();
@@ -217,34 +250,80 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int K = p.K;
   const int nkb = ceil_div(K, KB);
 
-  if (warp == 0) {
-    // idle: the dequantization warps load the weights themselves
-  } else if (warp == kMmaWarp) {
-    // ---------------------------------------------------------------- MMA issuer
-    // Released step by step by the scheduler warp; identical loop bounds on both sides.
+  if (warp == kWProdWarp) {
+    // ---------------------------------------------------------------- weight producer
+    const uint64_t pol_w = policy_evict_first();
+    const int kg = K / 32;
+    int ws = 0, issued = 0;
+    uint32_t ph = 0;
+    bool ok = true;
+    for (int it = blockIdx.x; it < total && ok; it += gridDim.x) {
+      const Item I = decode_item(it, sprefix, p);
+      const int row_g = I.e * p.rows_per_expert + I.m * BM;
+      const int row_u = row_g + p.I;  // gated: the up tile
+      int kb0, kb1;
+      split_range(it, nkb, p.splits, kb0, kb1);
+      for (int kb = kb0; kb < kb1; ++kb) {
+        if (!(ok = __all_sync(0xffffffffu, mbar_wait(&empty_w[ws], ph ^ 1u, abort_flag, lim)))) break;
+        uint8_t* st = smem + C::OFF_W + ws * C::W_STAGE;
+        if (lane == 0) {
+          mbar_arrive_expect_tx(&full_w[ws], (uint32_t)(NA * C::W_TILE + (p.scales_tma ? NA * C::S_TILE : 0)));
+          tma_load_2d_hint(st, &tm_w, &full_w[ws], kb * (KB / 8), row_g, pol_w);
+          if (GATED) tma_load_2d_hint(st + C::W_TILE, &tm_w, &full_w[ws], kb * (KB / 8), row_u, pol_w);
+          if (p.scales_tma) {
+            tma_load_2d_hint(st + NA * C::W_TILE, &tm_s, &full_w[ws], kb * (KB / 32), row_g, pol_w);
+            if (GATED) tma_load_2d_hint(st + NA * C::W_TILE + C::S_TILE, &tm_s, &full_w[ws], kb * (KB / 32), row_u, pol_w);
+          }
+        }
+        if (!p.scales_tma) {  // scale rows 8-byte aligned: 8 or 4 bf16 per row by cp.async
+          const int ngrp = min(KB, K - kb * KB) / 32;
+#pragma unroll
+          for (int mat = 0; mat < NA; ++mat) {
+            const int row0 = mat ? row_u : row_g;
+            for (int rr = lane; rr < BM; rr += 32) {
+              const uint16_t* src = p.w_s + (size_t)(row0 + rr) * kg + kb * (KB / 32);
+              uint8_t* dst = st + NA * C::W_TILE + mat * C::S_TILE + rr * 16;
+              cp_async_8(dst, src);
+              if (ngrp > 4) cp_async_8(dst + 8, src + 4);
+            }
+          }
+          cp_async_arrive_noinc(&full_w[ws]);
+        }
+        ++issued;
+        if (++ws == WST) {
+          ws = 0;
+          ph ^= 1u;
+        }
+      }
+    }
+    if (lane == 0)
+      for (int i = max(0, issued - WST); i < issued; ++i) mbar_wait_plain(&full_w[i % WST], (i / WST) & 1, lim);
+  } else if (warp == kMmaWarp || (GATED && warp == kMmaWarpUp)) {
+    // ---------------------------------------------------------------- MMA issuers
+    // One per matrix, each released step by step by the scheduler warp on its own named barrier;
+    // identical loop bounds on all three sides.
+    const int mat = warp == kMmaWarp ? 0 : 1;
     int ab = 0, bs = 0, acc = 0;
     bool ok = true;
     for (int it = blockIdx.x; it < total && ok; it += gridDim.x) {
       const Item I = decode_item(it, sprefix, p);
       const uint32_t idesc = make_idesc(BM, I.nmma, 0, 0);
-      const uint32_t d0 = tmem_base + (uint32_t)(acc * C::ACC_COLS);  // [matrix][NMAX] columns
-      const uint32_t d1 = d0 + NMAX;
+      const uint32_t d = tmem_base + (uint32_t)(acc * C::ACC_COLS + mat * NMAX);  // [matrix][NMAX] columns
       int kb0, kb1;
       split_range(it, nkb, p.splits, kb0, kb1);
       for (int kb = kb0; kb < kb1 && ok; ++kb) {
         const int nsub = min(NSUB, (K - kb * KB) / KS);
         for (int j = 0; j < nsub; ++j) {
-          if (!(ok = bar_red_and(kMmaBarrier, 64, true))) break;
+          if (!(ok = bar_red_and(kMmaBarrier + mat, 64, true))) break;
           if (lane == 0) {
             tc_fence_after();
             const uint64_t b = sw128_kmajor_desc(smem_u32(smem + C::OFF_B + bs * C::B_ATOM));
-            const uint64_t a0 = sw128_kmajor_desc(smem_u32(smem + C::OFF_A + (ab * NA + 0) * C::A_TILE));
-            const uint64_t a1 = sw128_kmajor_desc(smem_u32(smem + C::OFF_A + (ab * NA + (NA - 1)) * C::A_TILE));
+            const uint32_t a0 = tmem_base + (uint32_t)(C::A_COL0 + (ab * NA + mat) * C::A_COLS);
 #pragma unroll
             for (int kk = 0; kk < KS / 16; ++kk) {
               const uint32_t accum = (kb != kb0) || j != 0 || kk != 0;  // fresh at the split's first K
-              umma_f16(d0, a0 + 2 * kk, b + 2 * kk, idesc, accum);  // +32 bytes along K
-              if (GATED) umma_f16(d1, a1 + 2 * kk, b + 2 * kk, idesc, accum);
+              // 16 K = 8 TMEM columns of A, 32 bytes of the activation atom
+              umma_f16_ts(d, a0 + 8 * kk, b + 2 * kk, idesc, accum);
             }
             umma_commit(&a_empty[ab]);
             umma_commit(&empty_b[bs]);
@@ -279,7 +358,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int j = 0; j < nsub; ++j) {
           ready = ready && __all_sync(0xffffffffu, mbar_wait(&a_full[ab], ph_a, abort_flag, lim)) &&
                   __all_sync(0xffffffffu, mbar_wait(&full_b[bs], ph_b, abort_flag, lim));
-          if (!(ok = bar_red_and(kMmaBarrier, 64, ready))) break;
+          ok = bar_red_and(kMmaBarrier, 64, ready);
+          if (GATED) bar_red_and(kMmaBarrier + 1, 64, ok);  // the up issuer takes the same step
+          if (!ok) break;
           if (++ab == ABUF) {
             ab = 0;
             ph_a ^= 1u;
@@ -329,19 +410,20 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   } else if (warp >= kEpiWarp0 && warp < kEpiWarp0 + 4) {
     // ---------------------------------------------------------------- epilogue
+    // Per chunk of 16 token columns the arithmetic of all 16 values is done first and the stores
+    // after it, with the rare h beyond fp16 handled out of line, so that the 16 independent
+    // SiLU chains overlap their latencies (one per thread at a time took ~10x longer).
     const int ew = warp - kEpiWarp0;  // == warp % 4: this warp may read TMEM lanes 32*ew..32*ew+31
     const int mrow = ew * 32 + lane;
+    int* rexp = sprefix + p.E + 1 + ew * NMAX;  // this warp's copy of the item's row exponents
     int acc = 0;
     uint32_t ph = 0;
     for (int it = blockIdx.x; it < total; it += gridDim.x) {
       const Item I = decode_item(it, sprefix, p);
-      // the item's row exponents, loaded while the MMAs run: lane l holds rows l + 32j
-      int rexp[NMAX / 32];
-#pragma unroll
-      for (int j = 0; j < NMAX / 32; ++j) {
-        const int rr = lane + 32 * j;
-        rexp[j] = (p.acc_exp && rr < I.nvalid) ? __ldg(p.acc_exp + I.r0 + rr) : 0;
-      }
+      // the item's row exponents, loaded while the MMAs run
+      if (p.acc_exp)
+        for (int rr = lane; rr < I.nmma; rr += 32) rexp[rr] = rr < I.nvalid ? __ldg(p.acc_exp + I.r0 + rr) : 0;
+      __syncwarp();
       if (!__all_sync(0xffffffffu, mbar_wait(&acc_full[acc], ph, abort_flag, lim))) break;
       tc_fence_after();
       const uint32_t tb = tmem_base + ((uint32_t)(ew * 32) << 16) + (uint32_t)(acc * C::ACC_COLS);
@@ -353,12 +435,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         tmem_ld_wait();
         const int nv = min(16, I.nvalid - c0);
         if (p.acc_exp) {  // rows whose fp16 operand was scaled by 2^-e to fit fp16: undo it
-          int ej = rexp[0];  // the exponents of rows c0 .. c0+15 sit in register c0 / 32
-#pragma unroll
-          for (int j = 1; j < NMAX / 32; ++j) ej = (c0 >> 5) == j ? rexp[j] : ej;
 #pragma unroll
           for (int i = 0; i < 16; ++i) {
-            const float sc = exp2_int(__shfl_sync(0xffffffffu, ej, (c0 & 16) + i));
+            const float sc = exp2_int(rexp[c0 + i]);  // the same word for every lane: a broadcast
             g[i] = __float_as_uint(__uint_as_float(g[i]) * sc);
             if (GATED) u[i] = __float_as_uint(__uint_as_float(u[i]) * sc);
           }
@@ -366,24 +445,36 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (GATED) {
           const int pos = interleave_pos(col);
           __half* out = reinterpret_cast<__half*>(p.out) + (size_t)(I.r0 + c0) * p.out_ld + pos;
-          bool huge = false;  // an h beyond even the prescaled fp16 range (2^32)
+          float hv[16];
+          bool over = false;
 #pragma unroll
           for (int i = 0; i < 16; ++i) {
-            if (i < nv) {
-              const float gv = __uint_as_float(g[i]), uv = __uint_as_float(u[i]);
-              const float hv = gv / (1.0f + __expf(-gv)) * uv;
-              if (fabsf(hv) < 65520.0f) {
-                out[(size_t)i * p.out_ld] = __float2half_rn(hv);
-              } else {  // beyond fp16: stored as h * 2^-16 and marked; h_rescale fixes its row
-                const int r = I.r0 + c0 + i;
-                out[(size_t)i * p.out_ld] = __float2half_rn(hv * (1.0f / 65536.0f));
-                atomicOr(p.ovf_mask + (size_t)r * (p.out_ld / 32) + pos / 32, 1u << (pos & 31));
-                p.ovf_flag[r] = 1;
-                huge |= !(fabsf(hv) < 65520.0f * 65536.0f);
+            const float gv = __uint_as_float(g[i]), uv = __uint_as_float(u[i]);
+            hv[i] = __fdividef(gv, 1.0f + __expf(-gv)) * uv;  // SiLU(g) * u; fp16 rounding follows
+            over |= i < nv && !(fabsf(hv[i]) < 65520.0f);
+          }
+          if (!__any_sync(0xffffffffu, over)) {
+#pragma unroll
+            for (int i = 0; i < 16; ++i)
+              if (i < nv) out[(size_t)i * p.out_ld] = __float2half_rn(hv[i]);
+          } else {
+            bool huge = false;  // an h beyond even the prescaled fp16 range (2^32)
+#pragma unroll
+            for (int i = 0; i < 16; ++i) {
+              if (i < nv) {
+                if (fabsf(hv[i]) < 65520.0f) {
+                  out[(size_t)i * p.out_ld] = __float2half_rn(hv[i]);
+                } else {  // beyond fp16: stored as h * 2^-16 and marked; h_rescale fixes its row
+                  const int r = I.r0 + c0 + i;
+                  out[(size_t)i * p.out_ld] = __float2half_rn(hv[i] * (1.0f / 65536.0f));
+                  atomicOr(p.ovf_mask + (size_t)r * (p.out_ld / 32) + pos / 32, 1u << (pos & 31));
+                  p.ovf_flag[r] = 1;
+                  huge |= !(fabsf(hv[i]) < 65520.0f * 65536.0f);
+                }
               }
             }
+            if (huge) set_status(MOE_ERR_DEVICE_CHECK);
           }
-          if (huge) set_status(MOE_ERR_DEVICE_CHECK);
         } else if (p.splits > 1) {  // this split's partial sum, reduced in split order by another kernel
           float* out = p.part + (size_t)(it % p.splits) * p.act_rows * p.out_ld + (size_t)(I.r0 + c0) * p.out_ld + col;
 #pragma unroll
@@ -409,84 +500,76 @@ __global__ void __launch_bounds__(kThreads, 1)
         ph ^= 1u;
       }
     }
-  } else if (warp >= kDqWarp0) {
-    // ---------------------------------------------------------------- dequantization -> SMEM
+  } else if (warp >= kDqWarp0 && warp < kDqWarp0 + kNumDq) {
+    // ---------------------------------------------------------------- dequantization -> TMEM
     // GATED: thread = one row of the gate (warps 8-11) or up (warps 12-15) tile, all 64 K of
-    // each step; plain: thread = one row, half of each 64-K step.  The thread's packed words
-    // and scales of the next (item, stage) are loaded while the current stage is written.
-    const int dt = threadIdx.x - kDqWarp0 * 32;  // 0..255
-    const int mat = GATED ? (dt >> 7) : 0;
-    const int half = GATED ? 0 : (dt >> 7);
-    const int row = dt & 127;
+    // each step (8 words -> 32 TMEM columns); plain: thread = one row and one 32-K half of each
+    // step (warps 8-11 the first half, 12-15 the second; 4 words -> 16 columns).  Warp 8 + q
+    // and 12 + q write TMEM lanes 32q .. 32q+31, the rows they own.
+    const int dw = warp - kDqWarp0;
+    const int row = (dw & 3) * 32 + lane;
     const int sw = row & 7;
+    const int mat = GATED ? (dw >> 2) : 0;
+    const int half = GATED ? 0 : (dw >> 2);
     constexpr int CHK = GATED ? 8 : 4;  // 16-byte chunks of packed words this thread takes per stage
-    const int kw = K / 8, kg = K / 32;  // int32 words and scales per weight row
-    const bool scl16 = (K % KB) == 0;   // scale rows are 16-byte aligned
-    // loads of stage kb of the item whose weight row is wr (chunks past K are not read)
-    auto load_stage = [&](int wr, int kb, uint4 (&wv)[CHK], uint4& sc) {
-      const uint4* wrow = reinterpret_cast<const uint4*>(p.w_q + (size_t)wr * kw + kb * (KB / 8));
-      const int nchunk = min(KB, K - kb * KB) / 32;  // 16-byte chunks (32 K) present: 8 or 4
-#pragma unroll
-      for (int c = 0; c < CHK; ++c) {
-        const int lc = GATED ? c : 2 * c + half;  // logical 16-byte chunk (32 K) of the stage
-        wv[c] = lc < nchunk ? __ldcs(wrow + lc) : make_uint4(0, 0, 0, 0);
-      }
-      const uint16_t* srow = p.w_s + (size_t)wr * kg + kb * 8;
-      if (scl16) {
-        sc = __ldcs(reinterpret_cast<const uint4*>(srow));
-      } else {
-        const uint2 lo = __ldcs(reinterpret_cast<const uint2*>(srow));
-        const uint2 hi = nchunk == 8 ? __ldcs(reinterpret_cast<const uint2*>(srow + 4)) : make_uint2(0, 0);
-        sc = make_uint4(lo.x, lo.y, hi.x, hi.y);
-      }
-    };
-    auto weight_row = [&](int it) {
-      const Item I = decode_item(it, sprefix, p);
-      return I.e * p.rows_per_expert + I.m * BM + (mat ? p.I : 0) + row;
-    };
-    int ab = 0;
-    uint32_t ph_a = 0;
+    const uint32_t lane_base = tmem_base + ((uint32_t)((dw & 3) * 32) << 16);
+    int ws = 0, ab = 0;
+    uint32_t ph_w = 0, ph_a = 0;
     bool ok = true;
-    uint4 wn[CHK], sn;
-    int wr = blockIdx.x < total ? weight_row(blockIdx.x) : 0;
-    if (blockIdx.x < total) {
-      int f0, f1;
-      split_range(blockIdx.x, nkb, p.splits, f0, f1);
-      load_stage(wr, f0, wn, sn);
-    }
     for (int it = blockIdx.x; it < total && ok; it += gridDim.x) {
-      const bool has_next = it + (int)gridDim.x < total;
-      const int wr_next = has_next ? weight_row(it + gridDim.x) : wr;
-      int kb0, kb1, nkb0, nkb1;
+      int kb0, kb1;
       split_range(it, nkb, p.splits, kb0, kb1);
-      split_range(it + gridDim.x, nkb, p.splits, nkb0, nkb1);
       for (int kb = kb0; kb < kb1 && ok; ++kb) {
-        uint4 wv[CHK], sc = sn;
+        ok = __all_sync(0xffffffffu, mbar_wait(&full_w[ws], ph_w, abort_flag, lim));
+        if (!ok) break;
+        const uint8_t* st = smem + C::OFF_W + ws * C::W_STAGE;
+        const uint8_t* wrow = st + mat * C::W_TILE + row * 128;
+        const uint4 sc = *reinterpret_cast<const uint4*>(st + NA * C::W_TILE + mat * C::S_TILE + row * 16);
+        uint4 wv[CHK];
 #pragma unroll
-        for (int c = 0; c < CHK; ++c) wv[c] = wn[c];
-        if (kb + 1 < kb1)
-          load_stage(wr, kb + 1, wn, sn);
-        else if (has_next)
-          load_stage(wr_next, nkb0, wn, sn);
+        for (int c = 0; c < CHK; ++c) {
+          const int lc = GATED ? c : 2 * c + half;  // logical 16-byte chunk (32 K) of the stage
+          wv[c] = *reinterpret_cast<const uint4*>(wrow + ((lc ^ sw) << 4));
+        }
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&empty_w[ws]);  // words and scales are in registers
+        if (++ws == WST) {
+          ws = 0;
+          ph_w ^= 1u;
+        }
         const int nsub = min(NSUB, (K - kb * KB) / KS);
 #pragma unroll
         for (int j = 0; j < NSUB; ++j) {
           if (j < nsub) {
             ok = __all_sync(0xffffffffu, mbar_wait(&a_empty[ab], ph_a ^ 1u, abort_flag, lim));
             if (!ok) break;
-            uint8_t* arow = smem + C::OFF_A + (ab * NA + mat) * C::A_TILE + row * 128;
+            tc_fence_after();  // the MMAs that last read this A slot have completed
+            const uint32_t col = (uint32_t)(C::A_COL0 + (ab * NA + mat) * C::A_COLS);
+            if constexpr (GATED) {
+              uint32_t r[32];
 #pragma unroll
-            for (int q = 0; q < 2; ++q) {
-              if (GATED || q == half) {
-                const uint4 w = GATED ? wv[2 * j + q] : wv[j];
+              for (int q = 0; q < 2; ++q) {
+                const uint4 w = wv[2 * j + q];
                 const __half2 s2 = scale_h2(sc, 2 * j + q);
-                *reinterpret_cast<uint4*>(arow + (((4 * q + 0) ^ sw) << 4)) = dequant_word(w.x, s2);
-                *reinterpret_cast<uint4*>(arow + (((4 * q + 1) ^ sw) << 4)) = dequant_word(w.y, s2);
-                *reinterpret_cast<uint4*>(arow + (((4 * q + 2) ^ sw) << 4)) = dequant_word(w.z, s2);
-                *reinterpret_cast<uint4*>(arow + (((4 * q + 3) ^ sw) << 4)) = dequant_word(w.w, s2);
+                const uint4 d0 = dequant_word(w.x, s2), d1 = dequant_word(w.y, s2);
+                const uint4 d2 = dequant_word(w.z, s2), d3 = dequant_word(w.w, s2);
+                const uint32_t v[16] = {d0.x, d0.y, d0.z, d0.w, d1.x, d1.y, d1.z, d1.w,
+                                        d2.x, d2.y, d2.z, d2.w, d3.x, d3.y, d3.z, d3.w};
+#pragma unroll
+                for (int i = 0; i < 16; ++i) r[16 * q + i] = v[i];
               }
+              tmem_st32(lane_base + col, r);
+            } else {
+              const uint4 w = wv[j];
+              const __half2 s2 = scale_h2(sc, 2 * j + half);
+              const uint4 d0 = dequant_word(w.x, s2), d1 = dequant_word(w.y, s2);
+              const uint4 d2 = dequant_word(w.z, s2), d3 = dequant_word(w.w, s2);
+              const uint32_t r[16] = {d0.x, d0.y, d0.z, d0.w, d1.x, d1.y, d1.z, d1.w,
+                                      d2.x, d2.y, d2.z, d2.w, d3.x, d3.y, d3.z, d3.w};
+              tmem_st16(lane_base + col + 16 * half, r);
             }
-            fence_proxy_async_smem();  // generic-proxy smem writes -> visible to the tensor core
+            tmem_st_wait();
+            tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(&a_full[ab]);
             if (++ab == ABUF) {
@@ -496,7 +579,6 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
         }
       }
-      wr = wr_next;
     }
   }
 
@@ -504,14 +586,26 @@ __global__ void __launch_bounds__(kThreads, 1)
   __syncthreads();
   if (warp == kMmaWarp) {
     tc_fence_after();
-    tmem_dealloc(tmem_base, C::TMEM_COLS);
+    tmem_dealloc(tmem_base, 512);
   }
 }
 
 template <bool GATED>
 cudaError_t launch_t(const W4GemmProblem& pr, cudaStream_t s) {
   using C = Cfg<GATED>;
-  CUtensorMap tm_b, tm_b128;
+  CUtensorMap tm_w, tm_s, tm_b, tm_b128;
+  const uint64_t wrows = (uint64_t)pr.E * pr.rows_per_expert;
+  if (encode_tmap_2d(&tm_w, pr.w_q, CU_TENSOR_MAP_DATA_TYPE_INT32, pr.K / 8, wrows, (uint64_t)pr.K / 2, KB / 8, BM,
+                     CU_TENSOR_MAP_SWIZZLE_128B) != CUDA_SUCCESS)
+    return cudaErrorInvalidValue;
+  const int scales_tma = (pr.K % KB) == 0;  // scale rows are then a multiple of 16 bytes
+  if (scales_tma) {
+    if (encode_tmap_2d(&tm_s, pr.w_s, CU_TENSOR_MAP_DATA_TYPE_UINT16, pr.K / 32, wrows, (uint64_t)pr.K / 16, KB / 32,
+                       BM, CU_TENSOR_MAP_SWIZZLE_NONE) != CUDA_SUCCESS)
+      return cudaErrorInvalidValue;
+  } else {
+    tm_s = tm_w;  // unused
+  }
   if (encode_tmap_2d(&tm_b, pr.act, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, pr.K, (uint64_t)pr.act_rows, (uint64_t)pr.K * 2,
                      KS, 16, CU_TENSOR_MAP_SWIZZLE_128B) != CUDA_SUCCESS)
     return cudaErrorInvalidValue;
@@ -524,7 +618,7 @@ cudaError_t launch_t(const W4GemmProblem& pr, cudaStream_t s) {
   p.rows_per_expert = pr.rows_per_expert;
   p.I = pr.I;
   p.m_tiles = GATED ? pr.I / BM : pr.rows_per_expert / BM;
-  p.w_q = pr.w_q;
+  p.scales_tma = scales_tma;
   p.w_s = pr.w_s;
   p.sched = pr.sched;
   p.out = pr.out;
@@ -544,7 +638,7 @@ cudaError_t launch_t(const W4GemmProblem& pr, cudaStream_t s) {
   if (err != cudaSuccess) return err;
   const char* name = GATED ? "w4a16_gemm_gate_up" : "w4a16_gemm_down";
   timing_before(name, s);
-  kern<<<sm_count(), kThreads, smem, s>>>(tm_b, tm_b128, p);
+  kern<<<sm_count(), threads<GATED>(), smem, s>>>(tm_w, tm_s, tm_b, tm_b128, p);
   timing_after(name, s);
   return cudaGetLastError();
 }

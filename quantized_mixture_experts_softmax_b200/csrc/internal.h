@@ -68,7 +68,9 @@ cudaError_t launch_convert_rows(const uint16_t* a, int a_is_bf16, int M, int K, 
 cudaError_t launch_combine(const float* y_perm, const int32_t* inv_pos, const float* topk_w, int T, int k, int H,
                            void* out, int out_fp32, cudaStream_t s);
 
-// W4A16 grouped GEMM (gemm_w4a16.cu)
+// W4A16 grouped GEMM (gemm_w4a16.cu): token tiles of at most this many rows (the accumulators
+// and the A ring share tensor memory)
+constexpr int kWideTileRows = 192;
 enum OutKind { OUT_H_F16_INTERLEAVED = 0, OUT_F32 = 1, OUT_BF16 = 2, OUT_PLANES = 3 };
 struct W4GemmProblem {
   const int32_t* w_q;  // [E, rows_per_expert, K/8]

@@ -83,6 +83,16 @@ def test_expert_counts_straddling_the_kernel_choice():
     run_and_check(W4Layer(14, len(assign), 256, 256, E, 1, logits=lg), what="mixed kernels")
 
 
+def test_expert_counts_at_the_fp16_tile_height():
+    """Experts on the fp16 GEMM take token tiles of at most 192 rows: counts around one, two
+    and three tiles."""
+    counts = [191, 192, 193, 384, 385, 577, 17]
+    assign = np.repeat(np.arange(len(counts)), counts)
+    E = 8
+    lg = _onehot_logits(assign, E, 1, 15)
+    run_and_check(W4Layer(15, len(assign), 256, 128, E, 1, logits=lg), what="192-row tiles")
+
+
 def test_all_tokens_one_expert_top2():
     T, E = 300, 8
     lg = synth.logits(9, T, E)
