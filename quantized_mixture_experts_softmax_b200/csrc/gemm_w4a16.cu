@@ -30,7 +30,8 @@
 //               step by
 //   warp 2      the MMA scheduler, which waits for the accumulator, the dequantized A tile and
 //               the activation tile of each 64-K step;
-//   warp 3      TMA producer of the fp16 activation tiles (N rows x 64 K), BST-deep ring;
+//   warp 3      TMA producer of the fp16 activation tiles (N rows x 64 K, boxes of 128, 64, 32
+//               and 16 rows), BST-deep ring;
 //   warps 4-7   epilogue: tcgen05.ld of the fp32 accumulators, times each row's power-of-two
 //               exponent, SiLU(gate)*up for the gate/up GEMM (fp16 h) or a plain store (fp32 /
 //               bf16) for the down GEMM;
@@ -75,8 +76,8 @@ struct Cfg {
   static constexpr int W_STAGE = NA * (W_TILE + S_TILE);
   static constexpr int B_ATOM = NMAX * KS * 2;       // activation tile of one 64-K step
   // ring depths: weight stages, activation tiles, A slots in tensor memory
-  static constexpr int WST = GATED ? 3 : 4;
-  static constexpr int BST = GATED ? 4 : 6;
+  static constexpr int WST = GATED ? 3 : 2;
+  static constexpr int BST = GATED ? 4 : 7;
   static constexpr int ABUF = GATED ? 2 : 4;
   static constexpr int ACC_COLS = NA * NMAX;         // [matrix][NMAX] fp32 columns
   static constexpr int ACC_BUFS = (2 * ACC_COLS + ABUF * NA * (KS / 2) <= 512) ? 2 : 1;
@@ -94,6 +95,12 @@ struct Cfg {
   // then the tile prefix [E+1] and the epilogue warps' row exponents [4][NMAX]
   static constexpr size_t smem_bytes(int E) { return (size_t)OFF_PREFIX + 4 * (size_t)(E + 1 + 4 * NMAX) + 1024; }
   static_assert(smem_bytes(1024) <= 232448, "shared memory budget");
+};
+
+// tensor maps of the activation matrix with boxes of 128, 64, 32 and 16 rows (64 K each)
+struct BoxMaps {
+  CUtensorMap m[4];
+  __device__ const CUtensorMap& operator[](int i) const { return m[i]; }
 };
 
 struct Params {
@@ -187,8 +194,7 @@ __device__ __forceinline__ int interleave_pos(int j) {
 template <bool GATED>
 __global__ void __launch_bounds__(threads<GATED>(), 1)
     w4a16_gemm_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CUtensorMap tm_s,
-                      const __grid_constant__ CUtensorMap tm_b, const __grid_constant__ CUtensorMap tm_b128,
-                      const Params p) {
+                      const __grid_constant__ BoxMaps tm_b, const Params p) {
   using C = Cfg<GATED>;
   constexpr int NA = C::NA, WST = C::WST, BST = C::BST, ABUF = C::ABUF, ACCB = C::ACC_BUFS, NSUB = C::NSUB;
   extern __shared__ uint8_t smem_raw[];
@@ -235,8 +241,7 @@ __global__ void __launch_bounds__(threads<GATED>(), 1)
   if (warp == 0 && lane == 0) {
     prefetch_tmap(&tm_w);
     if (p.scales_tma) prefetch_tmap(&tm_s);
-    prefetch_tmap(&tm_b);
-    prefetch_tmap(&tm_b128);
+    for (int b = 0; b < 4; ++b) prefetch_tmap(&tm_b[b]);
   }
   if (warp == kMmaWarp) {
     tmem_alloc(tmem_slot, 512);
@@ -393,12 +398,13 @@ __global__ void __launch_bounds__(threads<GATED>(), 1)
         for (int ks = kb0 * (KB / KS); ks < ks1; ++ks) {
           if (!(ok = mbar_wait(&empty_b[bs], ph ^ 1u, abort_flag, lim))) break;
           mbar_arrive_expect_tx(&full_b[bs], (uint32_t)(I.nmma * KS * 2));
-          // 128-row boxes, then 16-row boxes for the rest (few large copies per step)
+          // boxes of 128, 64, 32 and 16 rows, largest first (at most 4 copies per tile)
+          uint8_t* dst = smem + C::OFF_B + bs * C::B_ATOM;
           int r = 0;
-          for (; r + 128 <= I.nmma; r += 128)
-            tma_load_2d_hint(smem + C::OFF_B + bs * C::B_ATOM + r * 128, &tm_b128, &full_b[bs], ks * KS, I.r0 + r, pol);
-          for (; r < I.nmma; r += 16)
-            tma_load_2d_hint(smem + C::OFF_B + bs * C::B_ATOM + r * 128, &tm_b, &full_b[bs], ks * KS, I.r0 + r, pol);
+          for (int b = 0; b < 4; ++b) {
+            const int h = 128 >> b;
+            for (; r + h <= I.nmma; r += h) tma_load_2d_hint(dst + r * 128, &tm_b[b], &full_b[bs], ks * KS, I.r0 + r, pol);
+          }
           ++issued;
           if (++bs == BST) {
             bs = 0;
@@ -593,7 +599,8 @@ __global__ void __launch_bounds__(threads<GATED>(), 1)
 template <bool GATED>
 cudaError_t launch_t(const W4GemmProblem& pr, cudaStream_t s) {
   using C = Cfg<GATED>;
-  CUtensorMap tm_w, tm_s, tm_b, tm_b128;
+  CUtensorMap tm_w, tm_s;
+  BoxMaps tm_b;
   const uint64_t wrows = (uint64_t)pr.E * pr.rows_per_expert;
   if (encode_tmap_2d(&tm_w, pr.w_q, CU_TENSOR_MAP_DATA_TYPE_INT32, pr.K / 8, wrows, (uint64_t)pr.K / 2, KB / 8, BM,
                      CU_TENSOR_MAP_SWIZZLE_128B) != CUDA_SUCCESS)
@@ -606,12 +613,10 @@ cudaError_t launch_t(const W4GemmProblem& pr, cudaStream_t s) {
   } else {
     tm_s = tm_w;  // unused
   }
-  if (encode_tmap_2d(&tm_b, pr.act, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, pr.K, (uint64_t)pr.act_rows, (uint64_t)pr.K * 2,
-                     KS, 16, CU_TENSOR_MAP_SWIZZLE_128B) != CUDA_SUCCESS)
-    return cudaErrorInvalidValue;
-  if (encode_tmap_2d(&tm_b128, pr.act, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, pr.K, (uint64_t)pr.act_rows,
-                     (uint64_t)pr.K * 2, KS, 128, CU_TENSOR_MAP_SWIZZLE_128B) != CUDA_SUCCESS)
-    return cudaErrorInvalidValue;
+  for (int b = 0; b < 4; ++b)
+    if (encode_tmap_2d(&tm_b.m[b], pr.act, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, pr.K, (uint64_t)pr.act_rows,
+                       (uint64_t)pr.K * 2, KS, 128 >> b, CU_TENSOR_MAP_SWIZZLE_128B) != CUDA_SUCCESS)
+      return cudaErrorInvalidValue;
   Params p;
   p.K = pr.K;
   p.E = pr.E;
@@ -638,7 +643,7 @@ cudaError_t launch_t(const W4GemmProblem& pr, cudaStream_t s) {
   if (err != cudaSuccess) return err;
   const char* name = GATED ? "w4a16_gemm_gate_up" : "w4a16_gemm_down";
   timing_before(name, s);
-  kern<<<sm_count(), threads<GATED>(), smem, s>>>(tm_w, tm_s, tm_b, tm_b128, p);
+  kern<<<sm_count(), threads<GATED>(), smem, s>>>(tm_w, tm_s, tm_b, p);
   timing_after(name, s);
   return cudaGetLastError();
 }
