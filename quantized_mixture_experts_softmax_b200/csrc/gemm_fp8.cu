@@ -329,31 +329,47 @@ __global__ void __launch_bounds__(Cfg<GATED, NMAX>::kThreads, 1)
       if (!ok) break;
       if constexpr (GATED) {
         // h = SiLU(gate) * up; requantize each token's 128 values of this tile (one 1x128 group):
-        // the token's amax over the tile's rows comes from the four warps of its half
+        // the token's amax over the tile's rows comes from the four warps of its half.  All
+        // arithmetic of the 32 tokens first, then the stores (independent chains overlap).
+        float hv[NH];
 #pragma unroll
-        for (int c = 0; c < NH; ++c) {
-          const float h = ag[c] / (1.0f + __expf(-ag[c])) * au[c];
-          ag[c] = h;
-          float m = fabsf(h);
+        for (int c = 0; c < NH; ++c) hv[c] = __fdividef(ag[c], 1.0f + __expf(-ag[c])) * au[c];
+        // the warp's max |h| per token, by recursive halving: after the step that exchanges
+        // `half` values, lane l holds maxima of the tokens whose index agrees with l in the bits
+        // above; in the end lane l holds token l's max over the warp's 32 rows (31 shuffles)
+        float m[NH];
 #pragma unroll
-          for (int off = 16; off; off >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, off));
-          if (lane == 0) red[ew * NMAX + tok0 + c] = m;
-        }
-        if (!(ok = epi_sync(epi_bar, ph_e, abort_flag, lim))) break;
-        uint8_t* hq = reinterpret_cast<uint8_t*>(p.out);
-        const int j = I.m * BM + mrow;
+        for (int c = 0; c < NH; ++c) m[c] = fabsf(hv[c]);
 #pragma unroll
-        for (int c = 0; c < NH; ++c) {
-          if (c < nv) {
-            const int t = tok0 + c;
-            const float a = fmaxf(fmaxf(red[t], red[NMAX + t]), fmaxf(red[2 * NMAX + t], red[3 * NMAX + t]));
-            const float sc = __fdiv_rn(fmaxf(a, 1e-10f), 448.0f);
-            const __nv_fp8_e4m3 q(__fdiv_rn(ag[c], sc));  // round to nearest even, saturating
-            hq[(size_t)(I.r0 + t) * p.out_ld + j] = *reinterpret_cast<const uint8_t*>(&q);
-            if (mrow == 0) p.h_scale[(size_t)I.m * p.act_rows + I.r0 + t] = sc;
+        for (int half = NH / 2; half >= 1; half >>= 1) {
+          const bool up = (lane & half) != 0;
+#pragma unroll
+          for (int i = 0; i < half; ++i) {
+            const float give = up ? m[i] : m[half + i];
+            const float keep = up ? m[half + i] : m[i];
+            m[i] = fmaxf(keep, __shfl_xor_sync(0xffffffffu, give, half));
           }
         }
-        if (!(ok = epi_sync(epi_bar, ph_e, abort_flag, lim))) break;  // red[] is reused by the next item
+        red[ew * NMAX + tok0 + lane] = m[0];
+        if (!(ok = epi_sync(epi_bar, ph_e, abort_flag, lim))) break;
+        // token tok0 + lane's scale, computed once per lane and read back by every lane
+        const int t = tok0 + lane;
+        const float a = fmaxf(fmaxf(red[t], red[NMAX + t]), fmaxf(red[2 * NMAX + t], red[3 * NMAX + t]));
+        const float sc_l = __fdiv_rn(fmaxf(a, 1e-10f), 448.0f);
+        cs[lane] = sc_l;  // the block-scale area is free after the K loop
+        if (ew == 0 && lane < nv) p.h_scale[(size_t)I.m * p.act_rows + I.r0 + t] = sc_l;
+        __syncwarp();
+        uint8_t q[NH];
+#pragma unroll
+        for (int c = 0; c < NH; ++c) {
+          const __nv_fp8_e4m3 e(__fdiv_rn(hv[c], cs[c]));  // round to nearest even, saturating
+          q[c] = *reinterpret_cast<const uint8_t*>(&e);
+        }
+        uint8_t* hq = reinterpret_cast<uint8_t*>(p.out) + (size_t)(I.r0 + tok0) * p.out_ld + I.m * BM + mrow;
+#pragma unroll
+        for (int c = 0; c < NH; ++c)
+          if (c < nv) hq[(size_t)c * p.out_ld] = q[c];
+        if (!(ok = epi_sync(epi_bar, ph_e, abort_flag, lim))) break;  // red[] and cs are reused next
       } else {
         float* y = reinterpret_cast<float*>(p.out);
         const int n = I.m * BM + mrow;
