@@ -41,16 +41,20 @@ constexpr int kMmaBarrier = 1;  // named barrier of the MMA and scheduler warps 
 constexpr int kEpiWarp0 = 3;    // warps 3..: promotion; lane quarter warp % 4, token part (warp - 3) / 4
 
 // NMAX = token rows per tile (32 or 64): 4 promotion warps per 32 tokens
-template <bool GATED, int NMAX>
+// NA_ = 128-row weight tiles per work item: the gate and up tiles (gate/up GEMM), or two
+// adjacent output tiles (down GEMM with rows in 256s: twice the MMAs per hand-off and per
+// activation tile, half the items), else one.
+template <bool GATED, int NMAX, int NA_>
 struct Cfg {
   static_assert(NMAX % NH == 0 && NMAX <= 64, "32 or 64 token rows per tile");
   static constexpr int kNumEpi = 4 * (NMAX / NH);
   static constexpr int kThreads = (kEpiWarp0 + kNumEpi) * 32;
-  static constexpr int NA = GATED ? 2 : 1;
+  static_assert(!GATED || NA_ == 2, "gate and up tiles");
+  static constexpr int NA = NA_;
   static constexpr int W_TILE = BM * KB;    // e4m3 bytes
   static constexpr int B_TILE = NMAX * KB;  // activation bytes
   static constexpr int STAGE = NA * W_TILE + B_TILE;
-  static constexpr int ST = NMAX == 32 ? (GATED ? 6 : 10) : (GATED ? 5 : 9);
+  static constexpr int ST = NMAX == 32 ? (NA == 2 ? 6 : 10) : (NA == 2 ? 5 : 9);
   static constexpr int P_COLS = NA * NMAX;  // one partial-product tile: [matrix][NMAX] columns
   // partial-product tiles in flight between the MMA and the promotion warps (as many as fit)
   static constexpr int NPB = 4 * P_COLS <= 512 ? 4 : 2;
@@ -70,6 +74,7 @@ struct Cfg {
 
 struct Params {
   int K, E, rows_per_expert, I, m_tiles;
+  int row_off2;          // NA = 2: rows of the second tile after the first (I for gate/up, 128 for down)
   const float* w_scale;  // [E, rows_per_expert/128, K/128]
   const float* x_scale;  // transposed activation scales [K/128, act_rows]
   int act_rows;
@@ -117,11 +122,11 @@ __device__ __forceinline__ bool epi_sync(uint64_t* bar, uint32_t& phase, volatil
   return ok;
 }
 
-template <bool GATED, int NMAX>
-__global__ void __launch_bounds__(Cfg<GATED, NMAX>::kThreads, 1)
+template <bool GATED, int NMAX, int NA_>
+__global__ void __launch_bounds__(Cfg<GATED, NMAX, NA_>::kThreads, 1)
     fp8_gemm_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CUtensorMap tm_b,
                     const Params p) {
-  using C = Cfg<GATED, NMAX>;
+  using C = Cfg<GATED, NMAX, NA_>;
   constexpr int NA = C::NA, ST = C::ST, kNumEpi = C::kNumEpi;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -180,14 +185,14 @@ __global__ void __launch_bounds__(Cfg<GATED, NMAX>::kThreads, 1)
       bool ok = true;
       for (int it = blockIdx.x; it < total && ok; it += gridDim.x) {
         const Item I = decode_item(it, sprefix, p);
-        const int row_g = I.e * p.rows_per_expert + I.m * BM;
-        const int row_u = row_g + p.I;
+        const int row_g = I.e * p.rows_per_expert + I.m * (GATED ? BM : NA * BM);  // first tile
+        const int row_u = row_g + p.row_off2;                                        // second tile
         for (int kb = 0; kb < nkb; ++kb) {
           if (!(ok = mbar_wait(&empty[s], ph ^ 1u, abort_flag, lim))) break;
           uint8_t* st = smem + s * C::STAGE;
           mbar_arrive_expect_tx(&full[s], (uint32_t)(NA * C::W_TILE + I.nmma * KB));
           tma_load_2d_hint(st, &tm_w, &full[s], kb * KB, row_g, pol_w);
-          if (GATED) tma_load_2d_hint(st + C::W_TILE, &tm_w, &full[s], kb * KB, row_u, pol_w);
+          if (NA == 2) tma_load_2d_hint(st + C::W_TILE, &tm_w, &full[s], kb * KB, row_u, pol_w);
           for (int r = 0; r < I.nmma; r += 16)
             tma_load_2d_hint(st + NA * C::W_TILE + r * 128, &tm_b, &full[s], kb * KB, I.r0 + r, pol_b);
           ++issued;
@@ -219,7 +224,7 @@ __global__ void __launch_bounds__(Cfg<GATED, NMAX>::kThreads, 1)
 #pragma unroll
           for (int kk = 0; kk < KB / 32; ++kk) {  // K = 32 e4m3 = 32 bytes per MMA
             umma_f8(d, a0 + 2 * kk, b + 2 * kk, idesc, kk != 0);
-            if (GATED) umma_f8(d + NMAX, a1 + 2 * kk, b + 2 * kk, idesc, kk != 0);
+            if (NA == 2) umma_f8(d + NMAX, a1 + 2 * kk, b + 2 * kk, idesc, kk != 0);
           }
           umma_commit(&p_full[pb]);
           umma_commit(&empty[s]);
@@ -270,20 +275,20 @@ __global__ void __launch_bounds__(Cfg<GATED, NMAX>::kThreads, 1)
       float ag[NH], au[NH];
 #pragma unroll
       for (int c = 0; c < NH; ++c) ag[c] = au[c] = 0.f;
-      const float* wsg = p.w_scale + ((size_t)I.e * (p.rows_per_expert / BM) + I.m) * GK;
-      const float* wsu = GATED ? wsg + (size_t)(p.I / BM) * GK : wsg;
+      const float* wsg = p.w_scale + ((size_t)I.e * (p.rows_per_expert / BM) + I.m * (GATED ? 1 : NA)) * GK;
+      const float* wsu = NA == 2 ? wsg + (size_t)(p.row_off2 / BM) * GK : wsg;
       // per-token activation scales (lane c holds token tok0+c's) and weight-block scales, one
       // block ahead so that their load latency hides behind the current block
       auto xs_at = [&](int kb) {
         return (lane < nv && kb < nkb) ? __ldg(p.x_scale + (size_t)kb * p.act_rows + I.r0 + tok0 + lane) : 0.f;
       };
-      float xs_n = xs_at(0), sg_n = __ldg(wsg), su_n = GATED ? __ldg(wsu) : 0.f;
+      float xs_n = xs_at(0), sg_n = __ldg(wsg), su_n = NA == 2 ? __ldg(wsu) : 0.f;
       for (int kb = 0; kb < nkb; ++kb) {
         const float xs_l = xs_n, sg = sg_n, su = su_n;
         xs_n = xs_at(kb + 1);
         if (kb + 1 < nkb) {
           sg_n = __ldg(wsg + kb + 1);
-          if (GATED) su_n = __ldg(wsu + kb + 1);
+          if (NA == 2) su_n = __ldg(wsu + kb + 1);
         }
         ok = __all_sync(0xffffffffu, mbar_wait(&p_full[pb], ph_p, abort_flag, lim));
         if (!ok) break;
@@ -291,7 +296,7 @@ __global__ void __launch_bounds__(Cfg<GATED, NMAX>::kThreads, 1)
         // the scale of (row block, token) is uniform over the warp's rows: one product per token,
         // read back by every lane as float4 broadcasts
         cs[lane] = sg * xs_l;
-        if (GATED) cs[NH + lane] = su * xs_l;
+        if (NA == 2) cs[NH + lane] = su * xs_l;
         __syncwarp();
         const uint32_t tb = tmem_base + ((uint32_t)(ew * 32) << 16) + (uint32_t)(pb * C::P_COLS + tok0);
         uint32_t pg[16], pu[16];
@@ -299,7 +304,7 @@ __global__ void __launch_bounds__(Cfg<GATED, NMAX>::kThreads, 1)
         for (int c0 = 0; c0 < NH; c0 += 16) {
           if (tok0 + c0 < I.nmma) {
             tmem_ld16(tb + c0, pg);
-            if (GATED) tmem_ld16(tb + NMAX + c0, pu);
+            if (NA == 2) tmem_ld16(tb + NMAX + c0, pu);
             tmem_ld_wait();
 #pragma unroll
             for (int i = 0; i < 16; i += 4) {
@@ -308,7 +313,7 @@ __global__ void __launch_bounds__(Cfg<GATED, NMAX>::kThreads, 1)
               ag[c0 + i + 1] = fmaf(__uint_as_float(pg[i + 1]), g4.y, ag[c0 + i + 1]);
               ag[c0 + i + 2] = fmaf(__uint_as_float(pg[i + 2]), g4.z, ag[c0 + i + 2]);
               ag[c0 + i + 3] = fmaf(__uint_as_float(pg[i + 3]), g4.w, ag[c0 + i + 3]);
-              if (GATED) {
+              if (NA == 2) {
                 const float4 u4 = *reinterpret_cast<const float4*>(cs + NH + c0 + i);
                 au[c0 + i + 0] = fmaf(__uint_as_float(pu[i + 0]), u4.x, au[c0 + i + 0]);
                 au[c0 + i + 1] = fmaf(__uint_as_float(pu[i + 1]), u4.y, au[c0 + i + 1]);
@@ -372,10 +377,13 @@ __global__ void __launch_bounds__(Cfg<GATED, NMAX>::kThreads, 1)
         if (!(ok = epi_sync(epi_bar, ph_e, abort_flag, lim))) break;  // red[] and cs are reused next
       } else {
         float* y = reinterpret_cast<float*>(p.out);
-        const int n = I.m * BM + mrow;
 #pragma unroll
-        for (int c = 0; c < NH; ++c)
-          if (c < nv) y[(size_t)(I.r0 + tok0 + c) * p.out_ld + n] = ag[c];
+        for (int mat = 0; mat < NA; ++mat) {
+          const int n = I.m * (NA * BM) + mat * BM + mrow;
+#pragma unroll
+          for (int c = 0; c < NH; ++c)
+            if (c < nv) y[(size_t)(I.r0 + tok0 + c) * p.out_ld + n] = mat ? au[c] : ag[c];
+        }
       }
     }
   }
@@ -388,9 +396,9 @@ __global__ void __launch_bounds__(Cfg<GATED, NMAX>::kThreads, 1)
   }
 }
 
-template <bool GATED, int NMAX>
+template <bool GATED, int NMAX, int NA_>
 cudaError_t launch_t(const F8GemmProblem& pr, cudaStream_t s) {
-  using C = Cfg<GATED, NMAX>;
+  using C = Cfg<GATED, NMAX, NA_>;
   CUtensorMap tm_w, tm_b;
   const uint64_t wrows = (uint64_t)pr.E * pr.rows_per_expert;
   if (encode_tmap_2d(&tm_w, pr.w, CU_TENSOR_MAP_DATA_TYPE_UINT8, pr.K, wrows, (uint64_t)pr.K, KB, BM,
@@ -404,7 +412,8 @@ cudaError_t launch_t(const F8GemmProblem& pr, cudaStream_t s) {
   p.E = pr.E;
   p.rows_per_expert = pr.rows_per_expert;
   p.I = pr.I;
-  p.m_tiles = GATED ? pr.I / BM : pr.rows_per_expert / BM;
+  p.m_tiles = GATED ? pr.I / BM : pr.rows_per_expert / (NA_ * BM);
+  p.row_off2 = GATED ? pr.I : BM;
   p.w_scale = pr.w_scale;
   p.x_scale = pr.x_scale;
   p.act_rows = pr.act_rows;
@@ -414,7 +423,7 @@ cudaError_t launch_t(const F8GemmProblem& pr, cudaStream_t s) {
   p.h_scale = pr.h_scale;
   p.wait_limit = wait_limit_ns();
   const size_t smem = C::smem_bytes(pr.E);
-  auto kern = fp8_gemm_kernel<GATED, NMAX>;
+  auto kern = fp8_gemm_kernel<GATED, NMAX, NA_>;
   cudaError_t err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (err != cudaSuccess) return err;
   const char* name = GATED ? "fp8_gemm_gate_up" : "fp8_gemm_down";
@@ -427,8 +436,13 @@ cudaError_t launch_t(const F8GemmProblem& pr, cudaStream_t s) {
 }  // namespace f8
 
 cudaError_t launch_fp8_gemm(const F8GemmProblem& p, cudaStream_t s) {
-  if (p.nmax == 32) return p.gated ? f8::launch_t<true, 32>(p, s) : f8::launch_t<false, 32>(p, s);
-  if (p.nmax == 64) return p.gated ? f8::launch_t<true, 64>(p, s) : f8::launch_t<false, 64>(p, s);
+  const bool two = p.rows_per_expert % 256 == 0;  // the down GEMM: two output tiles per item
+  if (p.nmax == 32)
+    return p.gated ? f8::launch_t<true, 32, 2>(p, s)
+                   : (two ? f8::launch_t<false, 32, 2>(p, s) : f8::launch_t<false, 32, 1>(p, s));
+  if (p.nmax == 64)
+    return p.gated ? f8::launch_t<true, 64, 2>(p, s)
+                   : (two ? f8::launch_t<false, 64, 2>(p, s) : f8::launch_t<false, 64, 1>(p, s));
   return cudaErrorInvalidValue;
 }
 
