@@ -123,11 +123,16 @@ moe_status_t moe_align_noalloc(const int32_t* topk_ids, int T, int k, int E, int
  *     accumulated in fp32; h is stored the same way (one scale per token per 128 rows of I).
  *     The only rounding besides fp32 accumulation is X (at most s / 2 per element); any finite
  *     x is taken.
- *   fp16 GEMM: activations and dequantized weights are fed to the tensor cores in fp16, which is
- *     exact for bf16 x inside the fp16 normal range and for |q*s| inside it (scales in
- *     [2^-14/8... , 65504/8]); accumulation is fp32; h is rounded to fp16.  An x or an h
- *     beyond the fp16 range (|v| >= 65520) becomes +-inf there and records
- *     MOE_ERR_DEVICE_CHECK.
+ *   fp16 GEMM: activations and dequantized weights are fed to the tensor cores in fp16 with fp32
+ *     accumulation.  Each permuted row of x is multiplied by an exact power of two 2^-c (c >= 0
+ *     the smallest that brings the row's largest magnitude inside fp16, so c = 0 for every row
+ *     already inside it) and the row's accumulators are multiplied by 2^c, so any finite x is
+ *     taken; the conversion is exact for values inside the fp16 normal range after that
+ *     scaling.  The dequantized weights q*s are exact in fp16 while |q*s| is inside its normal
+ *     range.  h is rounded to fp16; a value of h beyond fp16 is stored times 2^-16 and its row
+ *     is then brought to one power-of-two scale 2^-c (c >= 1) before the down projection,
+ *     which multiplies that row's accumulators by 2^c.  An h beyond even that (|h| >= 65520 *
+ *     2^16, about 4.3e9) and a non-finite x record MOE_ERR_DEVICE_CHECK.
  * The combine sums the k slots in fp32 in slot order, so the result is deterministic run to
  * run.
  * ws: moe_w4a16_workspace_size(T, H, I, E, k) bytes. */

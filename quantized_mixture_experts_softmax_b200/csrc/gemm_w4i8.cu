@@ -56,6 +56,10 @@ constexpr int kEpiWarp0 = 4;
 constexpr int kUnpackWarp0 = 8;
 constexpr int kNumUnpack = 8;
 static_assert(NT == 8, "the promotion code handles up to 8 tokens per tile");
+// The producer decodes each work item (a binary search of the tile prefix plus three global
+// loads, ~1300 cycles with shared memory busy) and publishes it in a ring that the promotion
+// warps read once the item's first stage has landed, so the decode never holds the D slots.
+constexpr int kItemRing = 16;
 
 // A work item covers NA weight tiles of 128 rows: the gate and up tiles of the same 128
 // columns of h (gate/up GEMM), or two adjacent 128-row tiles of the output (down GEMM, when the
@@ -91,8 +95,11 @@ struct Cfg {
   static constexpr int OFF_BAR = ST * STAGE;
   static constexpr int NUM_BARS = 2 * ST + 2 * ASLOTS + 2 * DSLOTS + 2;
   static constexpr int OFF_MISC = OFF_BAR + NUM_BARS * 8;
-  static constexpr int OFF_RED = OFF_MISC + 16;  // [4 warps][NT] amax partials
-  static constexpr int OFF_PREFIX = OFF_RED + 4 * NT * 4;
+  static constexpr int OFF_RED = OFF_MISC + 16;  // [2 items][4 warps][NT] amax partials
+  static constexpr int OFF_ITEMS = OFF_RED + 2 * 4 * NT * 4;  // [kItemRing] decoded items
+  static constexpr int OFF_PREFIX = OFF_ITEMS + kItemRing * 16;
+  // the producer runs at most ST stages (so at most ST items) ahead of the promotion warps
+  static_assert(kItemRing > ST + 1, "item ring deeper than the stage ring");
   static_assert(STAGE % 1024 == 0 && STAGE_B % 1024 == 0, "swizzled tiles need 1024-byte alignment");
   static constexpr size_t smem_bytes(int E) { return (size_t)OFF_PREFIX + 4 * (size_t)(E + 1) + 1024; }
   static_assert(smem_bytes(1024) <= 232448, "shared memory budget");
@@ -117,6 +124,7 @@ struct Params {
 struct Item {
   int e, m, r0, nvalid;
 };
+static_assert(sizeof(Item) == 16, "ring entry");
 
 __device__ __forceinline__ Item decode_item(int it_, const int* __restrict__ sprefix, const Params& p) {
   Item I;
@@ -312,12 +320,13 @@ __device__ __forceinline__ bool epi_item(const Params& p, const Item& I, int it,
   if constexpr (GATED) {
 #pragma unroll
     for (int c = 0; c < NP; ++c) {
-      const float h = P.ag[c] / (1.0f + __expf(-P.ag[c])) * P.au[c];
+      const float h = __fdividef(P.ag[c], 1.0f + __expf(-P.ag[c])) * P.au[c];
       P.ag[c] = h;
-      float m = fabsf(h);
-#pragma unroll
-      for (int off = 16; off; off >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, off));
-      if (lane == 0) red[ew * NT + c] = m;
+      // the bit patterns of non-negative floats order like the values: one warp reduction (a NaN
+      // counts as 0, as fmaxf would skip it)
+      const float ah = fabsf(h);
+      const uint32_t m = __reduce_max_sync(0xffffffffu, ah == ah ? __float_as_uint(ah) : 0u);
+      if (lane == 0) red[ew * NT + c] = __uint_as_float(m);
     }
     if (!epi_sync(epi_bar, ph_e, abort_flag, p.wait_limit)) return false;
     const int j = I.m * BM + mrow;
@@ -328,22 +337,27 @@ __device__ __forceinline__ bool epi_item(const Params& p, const Item& I, int it,
     for (int c = 0; c < NP; ++c) {
       if (c < nv) {
         const float a = fmaxf(fmaxf(red[c], red[NT + c]), fmaxf(red[2 * NT + c], red[3 * NT + c]));
-        const float sc = fmaxf(a, 1e-30f) * (1.0f / kFixMax);
-        const int X = __float2int_rn(__fdiv_rn(P.ag[c], sc));
+        const float af = fmaxf(a, 1e-30f);
+        const float sc = af * (1.0f / kFixMax);
+        // |h| <= a and inv is within 2 ulps of kFixMax / a, so |X| <= kFixMax; the fast divide
+        // holds for divisors below 2^126
+        const float inv = af < 8.5e37f ? __fdividef((float)kFixMax, af) : (float)kFixMax / af;
+        const int X = __float2int_rn(P.ag[c] * inv);
         const int h8 = (X + 128) >> 8;
         const size_t o = (size_t)(2 * (I.r0 + c)) * p.out_ld + pos;
         planes[o] = (int8_t)h8;
         planes[o + p.out_ld] = (int8_t)(X - 256 * h8);
-        int sum = X;  // the 32 rows of this warp are one 32-group of h's K
-#pragma unroll
-        for (int off = 16; off; off >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, off);
+        const int sum = __reduce_add_sync(0xffffffffu, X);  // the warp's 32 rows: one 32-group of h's K
         // h's meta: stage I.m / 2, group (I.m & 1) * 4 + ew, block scale 8 + (I.m & 1)
         int32_t* m = p.out_meta + (size_t)(I.r0 + c) * mw_h + (I.m >> 1) * kMetaWords;
         if (lane == 0) m[(I.m & 1) * 4 + ew] = kFixBias - 8 * sum;
         if (mrow == 0) m[8 + (I.m & 1)] = __float_as_int(sc);
       }
     }
-    return epi_sync(epi_bar, ph_e, abort_flag, p.wait_limit);  // red[] is reused by the next item
+    // no second barrier: red[] alternates between two buffers by item, and a warp can write this
+    // buffer again (two items on) only after every warp has passed the next item's barrier,
+    // that is, after every warp finished the reads above
+    return true;
   } else {
 #pragma unroll
     for (int mat = 0; mat < NA_; ++mat) {
@@ -389,6 +403,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::OFF_MISC);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::OFF_MISC + 4);
   float* red = reinterpret_cast<float*>(smem + C::OFF_RED);
+  Item* items = reinterpret_cast<Item*>(smem + C::OFF_ITEMS);
   int* sprefix = reinterpret_cast<int*>(smem + C::OFF_PREFIX);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -438,10 +453,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint64_t pol_w = policy_evict_first();
     const uint64_t pol_b = policy_evict_last();
     const int kg = K / G;
-    int s = 0, issued = 0;
+    int s = 0, issued = 0, local = 0;
     uint32_t ph = 0;
     bool ok = true;
-    for (int it = blockIdx.x; it < total && ok; it += gridDim.x) {
+    for (int it = blockIdx.x; it < total && ok; it += gridDim.x, ++local) {
       const Item I = decode_item(it, sprefix, p);
       const int row_g = I.e * p.rows_per_expert + I.m * (GATED ? BM : NA * BM);  // first tile
       const int row_u = row_g + p.row_off2;                                      // second tile
@@ -452,6 +467,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         uint8_t* st = smem + s * C::STAGE;
         const int natom = min(KB, K - kb * KB) / 128;  // 2, or 1 for a half stage
         if (lane == 0) {
+          // the item's entry, released to the promotion warps by this stage's full barrier (its
+          // slot was last read for item local - kItemRing, whose stages are all done: the empty
+          // wait above)
+          if (kb == kb0) items[local & (kItemRing - 1)] = I;
           uint32_t bytes = NA * C::W_TILE + natom * C::B_ATOM + C::META_BYTES;
           if (p.scales_tma) bytes += NA * C::S_TILE;
           mbar_arrive_expect_tx(&full[s], bytes);
@@ -593,12 +612,16 @@ __global__ void __launch_bounds__(kThreads, 1)
     int ds = 0, s = 0;
     uint32_t ph_d = 0, ph_e = 0, ph = 0;
     bool ok = true;
-    for (int it = blockIdx.x; it < total && ok; it += gridDim.x) {
-      const Item I = decode_item(it, sprefix, p);
+    for (int it = blockIdx.x, local = 0; it < total && ok; it += gridDim.x, ++local) {
+      // the item's first stage has landed, so its entry is published (the same wait opens the
+      // K loop below)
+      if (!(ok = __all_sync(0xffffffffu, mbar_wait(&full[s], ph, abort_flag, lim)))) break;
+      const Item I = items[local & (kItemRing - 1)];
       const int nv = I.nvalid;
+      float* red_it = red + (local & 1) * (4 * NT);
 #define MOE_EPI_ITEM(NP_)                                                                                           \
-  epi_item<GATED, NA_, NP_>(p, I, it, ew, lane, lane_base, smem, s, ph, full, empty, ds, ph_d, d_full, d_empty, red,  \
-                            epi_bar, ph_e, abort_flag)
+  epi_item<GATED, NA_, NP_>(p, I, it, ew, lane, lane_base, smem, s, ph, full, empty, ds, ph_d, d_full, d_empty,      \
+                            red_it, epi_bar, ph_e, abort_flag)
       if (nv <= 1)
         ok = MOE_EPI_ITEM(1);
       else if (nv <= 2)
