@@ -64,8 +64,13 @@ struct Cfg {
   static constexpr int NUM_BARS = 2 * ST + 2 * NPB + 2;
   static constexpr int OFF_MISC = OFF_BAR + NUM_BARS * 8;
   static constexpr int OFF_RED = OFF_MISC + 16;              // [4 lane quarters][NMAX] amax partials
-  static constexpr int OFF_CS = OFF_RED + 4 * NMAX * 4;      // [promotion warp][matrix][NH] block scales
-  static constexpr int OFF_PREFIX = OFF_CS + kNumEpi * NA * NH * 4;
+  // [promotion warp][2][NH] block scales of gate and up (gate/up epilogue: h scales and their
+  // reciprocals)
+  static constexpr int OFF_CS = OFF_RED + 4 * NMAX * 4;
+  // gate/up: per promotion warp a [NH tokens][32 rows] byte tile, the e4m3 codes transposed so
+  // that each token's 32 bytes leave in two 16-byte stores
+  static constexpr int OFF_TR = OFF_CS + kNumEpi * 2 * NH * 4;
+  static constexpr int OFF_PREFIX = OFF_TR + (GATED ? kNumEpi * NH * 32 : 0);
   static_assert(OFF_CS % 16 == 0, "float4 reads of the block scales");
   static_assert(STAGE % 1024 == 0, "swizzled tiles need 1024-byte alignment");
   static constexpr size_t smem_bytes(int E) { return (size_t)OFF_PREFIX + 4 * (size_t)(E + 1) + 1024; }
@@ -140,6 +145,7 @@ __global__ void __launch_bounds__(Cfg<GATED, NMAX, NA_>::kThreads, 1)
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::OFF_MISC + 4);
   float* red = reinterpret_cast<float*>(smem + C::OFF_RED);
   float* cscale = reinterpret_cast<float*>(smem + C::OFF_CS);
+  uint8_t* trbuf = smem + C::OFF_TR;
   int* sprefix = reinterpret_cast<int*>(smem + C::OFF_PREFIX);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -336,15 +342,17 @@ __global__ void __launch_bounds__(Cfg<GATED, NMAX, NA_>::kThreads, 1)
         // h = SiLU(gate) * up; requantize each token's 128 values of this tile (one 1x128 group):
         // the token's amax over the tile's rows comes from the four warps of its half.  All
         // arithmetic of the 32 tokens first, then the stores (independent chains overlap).
-        float hv[NH];
+        // h overwrites the gate accumulators and |h| the up ones
+        float* hv = ag;
+        float* m = au;
 #pragma unroll
-        for (int c = 0; c < NH; ++c) hv[c] = __fdividef(ag[c], 1.0f + __expf(-ag[c])) * au[c];
+        for (int c = 0; c < NH; ++c) {
+          hv[c] = __fdividef(ag[c], 1.0f + __expf(-ag[c])) * au[c];
+          m[c] = fabsf(hv[c]);
+        }
         // the warp's max |h| per token, by recursive halving: after the step that exchanges
         // `half` values, lane l holds maxima of the tokens whose index agrees with l in the bits
         // above; in the end lane l holds token l's max over the warp's 32 rows (31 shuffles)
-        float m[NH];
-#pragma unroll
-        for (int c = 0; c < NH; ++c) m[c] = fabsf(hv[c]);
 #pragma unroll
         for (int half = NH / 2; half >= 1; half >>= 1) {
           const bool up = (lane & half) != 0;
@@ -362,19 +370,28 @@ __global__ void __launch_bounds__(Cfg<GATED, NMAX, NA_>::kThreads, 1)
         const float a = fmaxf(fmaxf(red[t], red[NMAX + t]), fmaxf(red[2 * NMAX + t], red[3 * NMAX + t]));
         const float sc_l = __fdiv_rn(fmaxf(a, 1e-10f), 448.0f);
         cs[lane] = sc_l;  // the block-scale area is free after the K loop
+        cs[NH + lane] = __frcp_rn(sc_l);
         if (ew == 0 && lane < nv) p.h_scale[(size_t)I.m * p.act_rows + I.r0 + t] = sc_l;
         __syncwarp();
-        uint8_t q[NH];
+        // q = e4m3(h / s), round to nearest even, saturating; h times the correctly rounded
+        // reciprocal of s differs from the quotient by at most an ulp of fp32, which moves a
+        // code only for a value that close to a rounding boundary of e4m3 (three mantissa bits)
+        uint8_t* tr = trbuf + (warp - kEpiWarp0) * (NH * 32);
 #pragma unroll
         for (int c = 0; c < NH; ++c) {
-          const __nv_fp8_e4m3 e(__fdiv_rn(hv[c], cs[c]));  // round to nearest even, saturating
-          q[c] = *reinterpret_cast<const uint8_t*>(&e);
+          const __nv_fp8_e4m3 e(hv[c] * cs[NH + c]);
+          tr[c * 32 + lane] = *reinterpret_cast<const uint8_t*>(&e);
         }
-        uint8_t* hq = reinterpret_cast<uint8_t*>(p.out) + (size_t)(I.r0 + tok0) * p.out_ld + I.m * BM + mrow;
-#pragma unroll
-        for (int c = 0; c < NH; ++c)
-          if (c < nv) hq[(size_t)c * p.out_ld] = q[c];
-        if (!(ok = epi_sync(epi_bar, ph_e, abort_flag, lim))) break;  // red[] and cs are reused next
+        __syncwarp();
+        if (lane < nv) {  // token tok0 + lane: its bytes of this warp's 32 rows
+          const uint4* src = reinterpret_cast<const uint4*>(tr + lane * 32);
+          uint4* dst = reinterpret_cast<uint4*>(reinterpret_cast<uint8_t*>(p.out) +
+                                                (size_t)(I.r0 + tok0 + lane) * p.out_ld + I.m * BM + ew * 32);
+          dst[0] = src[0];
+          dst[1] = src[1];
+        }
+        // red[], cs and the transpose tile are reused by the next item
+        if (!(ok = epi_sync(epi_bar, ph_e, abort_flag, lim))) break;
       } else {
         float* y = reinterpret_cast<float*>(p.out);
 #pragma unroll
