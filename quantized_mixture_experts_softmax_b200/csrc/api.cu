@@ -373,20 +373,27 @@ moe_status_t moe_w4a16_forward(const moe_w4a16_args* a, void* ws, size_t ws_byte
     so.tile_prefix = w.thin_tile_prefix;
     so.chunk = w.thin_chunk;
   }
-  cudaError_t e = launch_align(a->topk_ids, T, k, E, 1, w.counts, w.offsets, w.sorted, w.inv, w.blockcnt, &so, stream);
-  const TileSched thin{w.offsets, mixed ? w.thin_row_count : w.counts, w.thin_tile_prefix, w.thin_chunk};
-  const TileSched wide{w.offsets, w.row_count, w.tile_prefix, w.chunk};
   const uint16_t* x = static_cast<const uint16_t*>(a->x);
   const uint16_t* w13_s = static_cast<const uint16_t*>(a->w13_s);
   const uint16_t* w2_s = static_cast<const uint16_t*>(a->w2_s);
-  // activations of each class of experts in the form its GEMM reads
-  if (e == cudaSuccess) {
-    if (mixed)  // the rows of the thin experts only: at most kThinRows per expert
-      e = launch_planes_list(x, w.thin_row_prefix, w.offsets, w.sorted, E, k, std::min(P, kThinRows * E), H, w.xq.x,
-                             w.xq.meta, stream);
-    else
-      e = launch_planes(x, 1, w.inv, P, k, H, w.xq.x, w.xq.meta, stream);
+  cudaError_t e = cudaSuccess;
+  if (!mixed && fused_align_planes_ok(T, k, E)) {
+    // a decode-sized batch: alignment, schedule and planes in one launch
+    e = launch_align_planes(a->topk_ids, T, k, E, x, H, w.counts, w.offsets, w.sorted, w.inv, so.tile_prefix,
+                            so.chunk, so.nmax, w.xq.x, w.xq.meta, stream);
+  } else {
+    e = launch_align(a->topk_ids, T, k, E, 1, w.counts, w.offsets, w.sorted, w.inv, w.blockcnt, &so, stream);
+    // activations of each class of experts in the form its GEMM reads
+    if (e == cudaSuccess) {
+      if (mixed)  // the rows of the thin experts only: at most kThinRows per expert
+        e = launch_planes_list(x, w.thin_row_prefix, w.offsets, w.sorted, E, k, std::min(P, kThinRows * E), H,
+                               w.xq.x, w.xq.meta, stream);
+      else
+        e = launch_planes(x, 1, w.inv, P, k, H, w.xq.x, w.xq.meta, stream);
+    }
   }
+  const TileSched thin{w.offsets, mixed ? w.thin_row_count : w.counts, w.thin_tile_prefix, w.thin_chunk};
+  const TileSched wide{w.offsets, w.row_count, w.tile_prefix, w.chunk};
   if (e == cudaSuccess && mixed)
     e = launch_permute_w4(x, w.inv, a->topk_ids, w.row_count, T, k, H, w.x_perm, w.x_exp, w.ovf_flag, w.ovf_mask, I,
                           stream);

@@ -142,6 +142,13 @@ cudaError_t launch_reduce_splits(const float* part, int splits, int rows, int N,
                                  const int32_t* row_count, int E, void* out, int out_fp32, cudaStream_t s);
 // Planes of the K-vectors x_src: plane row r takes source row r (inv_pos == null, k == 1),
 // or for every pair p plane row inv_pos[p] takes source row p / k.
+// Alignment (align = 1) with the int8 GEMM's tile schedule and the fixed-point planes of every
+// pair's row, in one launch, for batches where fused_align_planes_ok(T, k, E).
+bool fused_align_planes_ok(int T, int k, int E);
+cudaError_t launch_align_planes(const int32_t* ids, int T, int k, int E, const uint16_t* x_bf16, int K,
+                                int32_t* counts, int32_t* offsets, int32_t* sorted_ids, int32_t* inv_pos,
+                                int32_t* tile_prefix, int32_t* chunk, int nmax, int8_t* planes, int32_t* meta,
+                                cudaStream_t s);
 cudaError_t launch_planes(const uint16_t* a, int a_is_bf16, const int32_t* inv_pos, int n_pairs, int k, int K,
                           int8_t* planes, int32_t* meta, cudaStream_t s);
 // Planes of the rows of the thin schedule's experts: row_prefix [E+1] is the exclusive scan of

@@ -206,11 +206,19 @@ cudaError_t launch_permute_fp8(const uint8_t* x, const float* xs, const int32_t*
 // word unpacks); the sum of X over every 32-K group (for the MMA's offset correction) and the
 // block scales go to the row's meta words.  Called by whole warps (two units of 16 lanes); a
 // lane with r < 0 takes part in the shuffles and writes nothing.
-__device__ __forceinline__ void planes_unit(const uint4* __restrict__ a, int a_is_bf16, int r, int src, int blk,
-                                            int i, int K, uint2* __restrict__ planes, int32_t* __restrict__ meta) {
+// One 128-K block of a source row, the caller's 8 elements: packed hi and lo bytes, the 32-K
+// group sum of X (valid on every lane) and the block scale.
+struct PlaneBits {
+  uint32_t hb[2], lb[2];
+  int sum;
+  float sc;
+};
+
+__device__ __forceinline__ PlaneBits planes_compute(const uint4* __restrict__ a, int a_is_bf16, bool live, int src,
+                                                    int blk, int i, int K) {
   float x[8];
   float amax = 0.f;
-  if (r >= 0) {
+  if (live) {
     const uint4 v = __ldg(a + ((size_t)src * K + blk * 128 + 8 * i) / 8);
     const uint32_t w[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
@@ -233,32 +241,179 @@ __device__ __forceinline__ void planes_unit(const uint4* __restrict__ a, int a_i
 #pragma unroll
   for (int off = 8; off; off >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, off));  // 16 lanes
   if (!(amax <= 3.402823466e38f) && i == 0) set_status(MOE_ERR_DEVICE_CHECK);  // an inf or NaN input
-  const float sc = fmaxf(amax, 1e-30f) * (1.0f / kFixMax);
+  PlaneBits pb;
+  pb.sc = fmaxf(amax, 1e-30f) * (1.0f / kFixMax);
   int X[8], sum = 0;
 #pragma unroll
   for (int j = 0; j < 8; ++j) {
-    X[j] = __float2int_rn(__fdiv_rn(x[j], sc));
+    X[j] = __float2int_rn(__fdiv_rn(x[j], pb.sc));
     sum += X[j];
   }
   sum += __shfl_xor_sync(0xffffffffu, sum, 1);
   sum += __shfl_xor_sync(0xffffffffu, sum, 2);  // 4 threads = one 32-K group
-  if (r < 0) return;
+  pb.sum = sum;
   constexpr int ord[8] = {0, 2, 4, 6, 1, 3, 5, 7};
-  uint32_t hb[2] = {0, 0}, lb[2] = {0, 0};
+  pb.hb[0] = pb.hb[1] = pb.lb[0] = pb.lb[1] = 0;
 #pragma unroll
   for (int q = 0; q < 8; ++q) {
     const int v = X[ord[q]];
     const int h8 = (v + 128) >> 8;
     const int l8 = v - 256 * h8;
-    hb[q >> 2] |= (uint32_t)(h8 & 0xFF) << (8 * (q & 3));
-    lb[q >> 2] |= (uint32_t)(l8 & 0xFF) << (8 * (q & 3));
+    pb.hb[q >> 2] |= (uint32_t)(h8 & 0xFF) << (8 * (q & 3));
+    pb.lb[q >> 2] |= (uint32_t)(l8 & 0xFF) << (8 * (q & 3));
   }
+  return pb;
+}
+
+__device__ __forceinline__ void planes_write(const PlaneBits& pb, int r, int blk, int i, int K,
+                                             uint2* __restrict__ planes, int32_t* __restrict__ meta) {
   const size_t o = ((size_t)(2 * r) * K + blk * 128 + 8 * i) / 8;
-  planes[o] = make_uint2(hb[0], hb[1]);
-  planes[o + K / 8] = make_uint2(lb[0], lb[1]);
+  planes[o] = make_uint2(pb.hb[0], pb.hb[1]);
+  planes[o + K / 8] = make_uint2(pb.lb[0], pb.lb[1]);
   int32_t* m = meta + (size_t)r * meta_words_per_row(K) + (blk >> 1) * kMetaWords;
-  if ((i & 3) == 0) m[(blk & 1) * 4 + (i >> 2)] = kFixBias - 8 * sum;
-  if (i == 0) m[8 + (blk & 1)] = __float_as_int(sc);
+  if ((i & 3) == 0) m[(blk & 1) * 4 + (i >> 2)] = kFixBias - 8 * pb.sum;
+  if (i == 0) m[8 + (blk & 1)] = __float_as_int(pb.sc);
+}
+
+__device__ __forceinline__ void planes_unit(const uint4* __restrict__ a, int a_is_bf16, int r, int src, int blk,
+                                            int i, int K, uint2* __restrict__ planes, int32_t* __restrict__ meta) {
+  const PlaneBits pb = planes_compute(a, a_is_bf16, r >= 0, src, blk, i, K);
+  if (r >= 0) planes_write(pb, r, blk, i, K, planes, meta);
+}
+
+// ------------------------------------------------------------------ alignment + planes, one launch
+// For small batches (P = T*k <= kFusedMaxPairs pairs, E <= kFusedMaxExperts): every CTA computes the
+// whole stable alignment in shared memory (a few microseconds for a decode batch), so no CTA waits
+// for another; each CTA writes its slice of inv_pos / sorted_ids (CTA 0 also the counts, offsets
+// and the int8 GEMM's tile schedule) and the fixed-point planes of its (token, 128-K block) units,
+// computed once per token and written to each of the token's k rows.  The same results as
+// moe_align (align = 1) followed by the planes kernel.
+constexpr int kFusedThreads = 512;
+constexpr int kFusedWarps = kFusedThreads / 32;
+constexpr int kFusedMaxPairs = 4096;
+constexpr int kFusedMaxExperts = kFusedThreads;  // one expert per thread in the block scans
+
+__global__ void __launch_bounds__(kFusedThreads) align_planes_kernel(
+    const int32_t* __restrict__ ids, int T, int k, int E, const uint4* __restrict__ x, int K,
+    int32_t* __restrict__ counts, int32_t* __restrict__ offsets, int32_t* __restrict__ sorted_ids,
+    int32_t* __restrict__ inv_pos, int32_t* __restrict__ tile_prefix, int32_t* __restrict__ chunk, int nmax,
+    uint2* __restrict__ planes, int32_t* __restrict__ meta) {
+  extern __shared__ int fsm[];
+  int* wcnt = fsm;                          // [kFusedWarps][E]: a warp's count, then its base
+  int* offs = wcnt + kFusedWarps * E;       // [E] first row of each expert
+  int* inv_s = offs + E;                    // [P] row of each pair (-1: out-of-range id)
+  __shared__ int warp_tot[32];
+  __shared__ int total;
+  const int P = T * k;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  for (int i = threadIdx.x; i < kFusedWarps * E; i += blockDim.x) wcnt[i] = 0;
+  __syncthreads();
+  // each warp takes a contiguous run of pairs, 32 at a time in order, so that ranks within an
+  // expert follow the pair order (a stable sort)
+  const int run = (P + kFusedWarps - 1) / kFusedWarps;
+  const int q0 = warp * run, q1 = min(P, q0 + run);
+  int* my = wcnt + warp * E;
+  for (int b = q0; b < q1; b += 32) {
+    const int p = b + lane;
+    const int e = p < q1 ? ids[p] : -1;
+    const bool valid = e >= 0 && e < E;
+    if (p < q1 && !valid && blockIdx.x == 0) set_status(MOE_ERR_DEVICE_CHECK);
+    const unsigned peers = __match_any_sync(0xffffffffu, valid ? e : -(lane + 2));
+    if (valid && lane == __ffs(peers) - 1) my[e] += __popc(peers);
+    __syncwarp();
+  }
+  __syncthreads();
+  // per expert: bases of the warps' runs, the count, then offsets and tiles by block scans
+  const int e = threadIdx.x;
+  int c = 0;
+  if (e < E)
+    for (int w = 0; w < kFusedWarps; ++w) {
+      const int v = wcnt[w * E + e];
+      wcnt[w * E + e] = c;
+      c += v;
+    }
+  const int off = block_exclusive_scan(e < E ? c : 0, warp_tot, &total);
+  const int n_rows = total;  // read by every thread before the next scan writes it
+  int nt = 0, ch = 16;
+  if (e < E) {
+    offs[e] = off;
+    expert_tiles(c, nmax, &nt, &ch);
+  }
+  const int tp = block_exclusive_scan(nt, warp_tot, &total);
+  if (blockIdx.x == 0) {
+    if (e < E) {
+      counts[e] = c;
+      offsets[e] = off;
+      tile_prefix[e] = tp;
+      chunk[e] = ch;
+    }
+    if (e == 0) {
+      offsets[E] = n_rows;
+      tile_prefix[E] = total;
+    }
+  }
+  __syncthreads();
+  // scatter: the same walk, now placing each pair
+  for (int b = q0; b < q1; b += 32) {
+    const int p = b + lane;
+    const int ee = p < q1 ? ids[p] : -1;
+    const bool valid = ee >= 0 && ee < E;
+    const unsigned peers = __match_any_sync(0xffffffffu, valid ? ee : -(lane + 2));
+    int pos = -1;
+    if (valid) pos = offs[ee] + my[ee] + __popc(peers & ((1u << lane) - 1u));
+    __syncwarp();
+    if (valid && lane == __ffs(peers) - 1) my[ee] += __popc(peers);
+    if (p < q1) inv_s[p] = pos;
+    __syncwarp();
+  }
+  __syncthreads();
+  // this CTA's slice of the pair arrays
+  const int slice = (P + gridDim.x - 1) / gridDim.x;
+  for (int p = blockIdx.x * slice + threadIdx.x; p < min(P, (int)(blockIdx.x + 1) * slice); p += blockDim.x) {
+    const int r = inv_s[p];
+    inv_pos[p] = r;
+    if (r >= 0) sorted_ids[r] = p;
+  }
+  // planes: units (token, 128-K block), 16 lanes each, this CTA's share of them
+  const int nblk = K / 128;
+  const int units = T * nblk;
+  const int per = (units + gridDim.x - 1) / gridDim.x;
+  const int u0 = blockIdx.x * per, u1 = min(units, u0 + per);
+  const int i = threadIdx.x & 15;
+  for (int ub = u0; ub < u1; ub += kFusedThreads / 16) {
+    const int u = ub + (threadIdx.x >> 4);
+    const bool live = u < u1;
+    const int t = live ? u / nblk : 0, blk = live ? u % nblk : 0;
+    const PlaneBits pb = planes_compute(x, 1, live, t, blk, i, K);
+    if (live)
+      for (int s = 0; s < k; ++s) {
+        const int r = inv_s[t * k + s];
+        if (r >= 0) planes_write(pb, r, blk, i, K, planes, meta);
+      }
+  }
+}
+
+bool fused_align_planes_ok(int T, int k, int E) { return (long long)T * k <= kFusedMaxPairs && E <= kFusedMaxExperts; }
+
+cudaError_t launch_align_planes(const int32_t* ids, int T, int k, int E, const uint16_t* x_bf16, int K,
+                                int32_t* counts, int32_t* offsets, int32_t* sorted_ids, int32_t* inv_pos,
+                                int32_t* tile_prefix, int32_t* chunk, int nmax, int8_t* planes, int32_t* meta,
+                                cudaStream_t s) {
+  const int P = T * k;
+  const size_t smem = (size_t)(kFusedWarps * E + E + P) * sizeof(int);
+  if (smem > 48 * 1024) {
+    const cudaError_t e = cudaFuncSetAttribute(align_planes_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                               (int)smem);
+    if (e != cudaSuccess) return e;
+  }
+  const int units = T * (K / 128);
+  const int grid = std::max(1, std::min(sm_count(), ceil_div(units, kFusedThreads / 16)));
+  timing_before("align_planes", s);
+  align_planes_kernel<<<grid, kFusedThreads, smem, s>>>(ids, T, k, E, reinterpret_cast<const uint4*>(x_bf16), K,
+                                                         counts, offsets, sorted_ids, inv_pos, tile_prefix, chunk,
+                                                         nmax, reinterpret_cast<uint2*>(planes), meta);
+  timing_after("align_planes", s);
+  return cudaGetLastError();
 }
 
 // every pair p: plane row inv_pos[p] from source row p / k (or, without inv_pos, row p from row p)
