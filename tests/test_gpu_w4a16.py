@@ -117,6 +117,14 @@ def test_k_equals_e():
     run_and_check(W4Layer(13, 9, 256, 128, 4, 4), what="k=E")
 
 
+@pytest.mark.parametrize("T,k,E", [(64, 64, 64), (64, 65, 65), (64, 8, 512), (8, 2, 600)])
+def test_decode_prologue_paths(T, k, E):
+    """T <= 64: batches of at most 4096 (token, slot) pairs and 512 experts take the alignment,
+    tile schedule and planes in one launch, larger ones the separate kernels; both sides of
+    each limit."""
+    run_and_check(W4Layer(14, T, 128, 128, E, k), what=f"T={T} k={k} E={E}")
+
+
 # ---------------------------------------------------------------------- full-size model
 @pytest.fixture(scope="module")
 def big_weights():
