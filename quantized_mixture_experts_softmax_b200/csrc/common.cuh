@@ -18,6 +18,23 @@ __device__ int g_device_status = 0;  // the library is one translation unit (lib
 
 __device__ __forceinline__ void set_status(int code) { atomicCAS(&g_device_status, 0, code); }
 
+// ------------------------------------------------------------------ dependent launches
+// Every kernel of the library is launched with programmatic stream serialization
+// (launch_kernel): it may be dispatched while the kernel before it on the stream is still
+// running, does its setup (barriers, tensor memory, tensor-map prefetch), then waits here until
+// that kernel has completed and its memory is visible, before it reads anything an earlier
+// kernel wrote or writes anything at all.  The short kernels then let the next kernel be
+// dispatched at once; the grouped GEMMs do not (the next kernel starts when they end).  Without
+// the launch attribute the wait returns at once.
+__device__ __forceinline__ void grid_dependency_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void grid_dependents_launch() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+__device__ __forceinline__ void grid_dependency_sync() {
+  grid_dependency_wait();
+  grid_dependents_launch();
+}
+
 // ------------------------------------------------------------------ smem addressing
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));

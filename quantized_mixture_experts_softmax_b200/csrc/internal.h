@@ -8,6 +8,25 @@
 
 namespace moe {
 
+// Launches `kernel` on stream s with programmatic stream serialization: the kernel may be
+// dispatched while the previous kernel on the stream still runs, and orders itself after it with
+// grid_dependency_wait (common.cuh) once its setup is done.
+template <typename... KArgs, typename... Args>
+cudaError_t launch_kernel(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t s,
+                          Args&&... args) {
+  cudaLaunchConfig_t cfg{};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kernel, static_cast<Args&&>(args)...);
+}
+
 // Kernel launch bookkeeping (per-kernel event timing for benchmarks).
 void timing_before(const char* name, cudaStream_t s);
 void timing_after(const char* name, cudaStream_t s);

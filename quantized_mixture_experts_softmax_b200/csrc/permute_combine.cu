@@ -74,6 +74,7 @@ __global__ void __launch_bounds__(256) permute_w4_kernel(const uint4* __restrict
                                                          uint4* __restrict__ x_perm, int32_t* __restrict__ x_exp,
                                                          int32_t* __restrict__ ovf_flag, uint32_t* __restrict__ ovf_mask,
                                                          int mask_words) {
+  grid_dependency_sync();  // see common.cuh
   const int p = (int)((blockIdx.x * blockDim.x + threadIdx.x) >> 5);
   const int lane = threadIdx.x & 31;
   if (p >= P) return;
@@ -101,7 +102,7 @@ cudaError_t launch_permute_w4(const uint16_t* x_bf16, const int32_t* inv_pos, co
                               int32_t* ovf_flag, uint32_t* ovf_mask, int I, cudaStream_t s) {
   const int P = T * k;
   timing_before("permute", s);
-  permute_w4_kernel<<<ceil_div(P, 8), 256, 0, s>>>(reinterpret_cast<const uint4*>(x_bf16), inv_pos, ids, cls_rows, P,
+  (void)launch_kernel(permute_w4_kernel, dim3(ceil_div(P, 8)), dim3(256), 0, s, reinterpret_cast<const uint4*>(x_bf16), inv_pos, ids, cls_rows, P,
                                                   k, H / 8, reinterpret_cast<uint4*>(x_perm), x_exp, ovf_flag, ovf_mask,
                                                   I / 32);
   timing_after("permute", s);
@@ -118,6 +119,7 @@ __global__ void __launch_bounds__(256) h_rescale_kernel(uint4* __restrict__ h, i
                                                         const int32_t* __restrict__ ovf_flag,
                                                         const uint32_t* __restrict__ ovf_mask,
                                                         int32_t* __restrict__ h_exp) {
+  grid_dependency_sync();  // see common.cuh
   const int lane = threadIdx.x & 31;
   const int mask_words = I8 / 4;
   for (int r = (int)((blockIdx.x * blockDim.x + threadIdx.x) >> 5); r < rows;
@@ -167,7 +169,7 @@ cudaError_t launch_h_rescale(__half* h, int rows, int I, const int32_t* ovf_flag
   const size_t want = ((size_t)rows + 7) / 8;
   const unsigned blocks = (unsigned)std::min<size_t>(want, (size_t)sm_count() * 16);
   timing_before("h_rescale", s);
-  h_rescale_kernel<<<blocks, 256, 0, s>>>(reinterpret_cast<uint4*>(h), rows, I / 8, ovf_flag, ovf_mask, h_exp);
+  (void)launch_kernel(h_rescale_kernel, dim3(blocks), dim3(256), 0, s, reinterpret_cast<uint4*>(h), rows, I / 8, ovf_flag, ovf_mask, h_exp);
   timing_after("h_rescale", s);
   return cudaGetLastError();
 }
@@ -177,6 +179,7 @@ __global__ void __launch_bounds__(256) permute_fp8_kernel(const uint4* __restric
                                                           const int32_t* __restrict__ inv_pos, int Pn, int k, int H,
                                                           uint4* __restrict__ x_perm, float* __restrict__ xs_t,
                                                           int P) {
+  grid_dependency_sync();  // see common.cuh
   const int p = (int)((blockIdx.x * blockDim.x + threadIdx.x) >> 5);
   const int lane = threadIdx.x & 31;
   if (p >= Pn) return;
@@ -193,7 +196,7 @@ cudaError_t launch_permute_fp8(const uint8_t* x, const float* xs, const int32_t*
                                uint8_t* x_perm, float* xs_t, int P, cudaStream_t s) {
   const int Pn = T * k;
   timing_before("permute_fp8", s);
-  permute_fp8_kernel<<<ceil_div(Pn, 8), 256, 0, s>>>(reinterpret_cast<const uint4*>(x), xs, inv_pos, Pn, k, H,
+  (void)launch_kernel(permute_fp8_kernel, dim3(ceil_div(Pn, 8)), dim3(256), 0, s, reinterpret_cast<const uint4*>(x), xs, inv_pos, Pn, k, H,
                                                     reinterpret_cast<uint4*>(x_perm), xs_t, P);
   timing_after("permute_fp8", s);
   return cudaGetLastError();
@@ -298,6 +301,7 @@ __global__ void __launch_bounds__(kFusedThreads) align_planes_kernel(
     int32_t* __restrict__ counts, int32_t* __restrict__ offsets, int32_t* __restrict__ sorted_ids,
     int32_t* __restrict__ inv_pos, int32_t* __restrict__ tile_prefix, int32_t* __restrict__ chunk, int nmax,
     uint2* __restrict__ planes, int32_t* __restrict__ meta) {
+  grid_dependency_sync();  // see common.cuh
   extern __shared__ int fsm[];
   int* wcnt = fsm;                          // [kFusedWarps][E]: a warp's count, then its base
   int* offs = wcnt + kFusedWarps * E;       // [E] first row of each expert
@@ -409,7 +413,7 @@ cudaError_t launch_align_planes(const int32_t* ids, int T, int k, int E, const u
   const int units = T * (K / 128);
   const int grid = std::max(1, std::min(sm_count(), ceil_div(units, kFusedThreads / 16)));
   timing_before("align_planes", s);
-  align_planes_kernel<<<grid, kFusedThreads, smem, s>>>(ids, T, k, E, reinterpret_cast<const uint4*>(x_bf16), K,
+  (void)launch_kernel(align_planes_kernel, dim3(grid), dim3(kFusedThreads), smem, s, ids, T, k, E, reinterpret_cast<const uint4*>(x_bf16), K,
                                                          counts, offsets, sorted_ids, inv_pos, tile_prefix, chunk,
                                                          nmax, reinterpret_cast<uint2*>(planes), meta);
   timing_after("align_planes", s);
@@ -420,6 +424,7 @@ cudaError_t launch_align_planes(const int32_t* ids, int T, int k, int E, const u
 __global__ void __launch_bounds__(256) planes_kernel(const uint4* __restrict__ a, int a_is_bf16,
                                                      const int32_t* __restrict__ inv_pos, int n_pairs, int k, int K,
                                                      uint2* __restrict__ planes, int32_t* __restrict__ meta) {
+  grid_dependency_sync();  // see common.cuh
   const int nblk = K / 128;
   const size_t unit = (blockIdx.x * (size_t)blockDim.x + threadIdx.x) >> 4;  // (pair, block)
   const int i = threadIdx.x & 15;                                             // 8-group within the block
@@ -434,7 +439,7 @@ cudaError_t launch_planes(const uint16_t* a, int a_is_bf16, const int32_t* inv_p
                           int8_t* planes, int32_t* meta, cudaStream_t s) {
   const size_t threads = (size_t)n_pairs * (K / 128) * 16;
   timing_before("planes", s);
-  planes_kernel<<<(unsigned)((threads + 255) / 256), 256, 0, s>>>(reinterpret_cast<const uint4*>(a), a_is_bf16,
+  (void)launch_kernel(planes_kernel, dim3((unsigned)((threads + 255) / 256)), dim3(256), 0, s, reinterpret_cast<const uint4*>(a), a_is_bf16,
                                                                   inv_pos, n_pairs, k, K,
                                                                   reinterpret_cast<uint2*>(planes), meta);
   timing_after("planes", s);
@@ -449,6 +454,7 @@ __global__ void __launch_bounds__(256) planes_list_kernel(const uint4* __restric
                                                           const int32_t* __restrict__ offsets,
                                                           const int32_t* __restrict__ sorted_ids, int E, int k, int K,
                                                           uint2* __restrict__ planes, int32_t* __restrict__ meta) {
+  grid_dependency_sync();  // see common.cuh
   const int nblk = K / 128;
   const size_t unit = (blockIdx.x * (size_t)blockDim.x + threadIdx.x) >> 4;  // (list row, block)
   const int i = threadIdx.x & 15;
@@ -477,7 +483,7 @@ cudaError_t launch_planes_list(const uint16_t* x_bf16, const int32_t* row_prefix
                                int32_t* meta, cudaStream_t s) {
   const size_t threads = (size_t)max_rows * (K / 128) * 16;
   timing_before("planes", s);
-  planes_list_kernel<<<(unsigned)((threads + 255) / 256), 256, 0, s>>>(
+  (void)launch_kernel(planes_list_kernel, dim3((unsigned)((threads + 255) / 256)), dim3(256), 0, s, 
       reinterpret_cast<const uint4*>(x_bf16), row_prefix, offsets, sorted_ids, E, k, K,
       reinterpret_cast<uint2*>(planes), meta);
   timing_after("planes", s);
@@ -493,6 +499,7 @@ __global__ void __launch_bounds__(256) reduce_splits_kernel(const float4* __rest
                                                             int N, const int32_t* __restrict__ row_start,
                                                             const int32_t* __restrict__ row_count,
                                                             void* __restrict__ out, int out_fp32) {
+  grid_dependency_sync();  // see common.cuh
   const int e = blockIdx.y;
   const int cnt = __ldg(row_count + e);
   if (cnt <= 0) return;
@@ -524,7 +531,7 @@ cudaError_t launch_reduce_splits(const float* part, int splits, int rows, int N,
   const size_t cap = (size_t)sm_count() * 8;
   const unsigned bx = (unsigned)std::max<size_t>(1, std::min(want, cap) / (size_t)E);
   timing_before("reduce_splits", s);
-  reduce_splits_kernel<<<dim3(bx, (unsigned)E), 256, 0, s>>>(reinterpret_cast<const float4*>(part), splits, rows, N,
+  (void)launch_kernel(reduce_splits_kernel, dim3(dim3(bx, (unsigned)E)), dim3(256), 0, s, reinterpret_cast<const float4*>(part), splits, rows, N,
                                                               row_start, row_count, out, out_fp32);
   timing_after("reduce_splits", s);
   return cudaGetLastError();
@@ -535,6 +542,7 @@ cudaError_t launch_reduce_splits(const float* part, int splits, int rows, int N,
 // fp16 (always 0 for fp16 input); a non-finite input is recorded as MOE_ERR_DEVICE_CHECK.
 __global__ void __launch_bounds__(256) convert_rows_kernel(const uint4* __restrict__ a, int a_is_bf16, int M, int K8,
                                                            uint4* __restrict__ out, int32_t* __restrict__ x_exp) {
+  grid_dependency_sync();  // see common.cuh
   const int lane = threadIdx.x & 31;
   for (int r = (int)((blockIdx.x * (size_t)blockDim.x + threadIdx.x) >> 5); r < M;
        r += (int)(((size_t)gridDim.x * blockDim.x) >> 5)) {
@@ -559,7 +567,7 @@ cudaError_t launch_convert_rows(const uint16_t* a, int a_is_bf16, int M, int K, 
                                 cudaStream_t s) {
   const int blocks = (int)std::min<size_t>(((size_t)M + 7) / 8, (size_t)sm_count() * 16);
   timing_before("convert", s);
-  convert_rows_kernel<<<blocks, 256, 0, s>>>(reinterpret_cast<const uint4*>(a), a_is_bf16, M, K / 8,
+  (void)launch_kernel(convert_rows_kernel, dim3(blocks), dim3(256), 0, s, reinterpret_cast<const uint4*>(a), a_is_bf16, M, K / 8,
                                              reinterpret_cast<uint4*>(out), x_exp);
   timing_after("convert", s);
   return cudaGetLastError();
@@ -569,6 +577,7 @@ cudaError_t launch_convert_rows(const uint16_t* a, int a_is_bf16, int M, int K, 
 __global__ void __launch_bounds__(256) combine_kernel(const float4* __restrict__ y, const int32_t* __restrict__ inv_pos,
                                                       const float* __restrict__ w, int T, int k, int H4,
                                                       void* __restrict__ out, int out_fp32) {
+  grid_dependency_sync();  // see common.cuh
   const size_t i = blockIdx.x * (size_t)blockDim.x + threadIdx.x;
   if (i >= (size_t)T * H4) return;
   const int t = (int)(i / H4), c = (int)(i % H4);
@@ -598,7 +607,7 @@ cudaError_t launch_combine(const float* y_perm, const int32_t* inv_pos, const fl
                            void* out, int out_fp32, cudaStream_t s) {
   const size_t n = (size_t)T * (H / 4);
   timing_before("combine", s);
-  combine_kernel<<<(unsigned)((n + 255) / 256), 256, 0, s>>>(reinterpret_cast<const float4*>(y_perm), inv_pos, topk_w,
+  (void)launch_kernel(combine_kernel, dim3((unsigned)((n + 255) / 256)), dim3(256), 0, s, reinterpret_cast<const float4*>(y_perm), inv_pos, topk_w,
                                                               T, k, H / 4, out, out_fp32);
   timing_after("combine", s);
   return cudaGetLastError();

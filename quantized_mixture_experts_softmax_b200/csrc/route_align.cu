@@ -24,6 +24,7 @@ template <int EPL>
 __global__ void __launch_bounds__(256) route_kernel(const float* __restrict__ logits, int T, int E, int k,
                                                     int renormalize, int32_t* __restrict__ ids,
                                                     float* __restrict__ w) {
+  grid_dependency_sync();  // see common.cuh
   const int warp = (int)((blockIdx.x * blockDim.x + threadIdx.x) >> 5);
   const int lane = threadIdx.x & 31;
   if (warp >= T) return;
@@ -89,17 +90,17 @@ cudaError_t launch_route(const float* logits, int T, int E, int k, int renormali
   timing_before("route", s);
   const int epl = ceil_div(E, 32);
   if (epl <= 1)
-    route_kernel<1><<<blocks, 256, 0, s>>>(logits, T, E, k, renormalize, ids, w);
+    (void)launch_kernel(route_kernel<1>, dim3(blocks), dim3(256), 0, s, logits, T, E, k, renormalize, ids, w);
   else if (epl <= 2)
-    route_kernel<2><<<blocks, 256, 0, s>>>(logits, T, E, k, renormalize, ids, w);
+    (void)launch_kernel(route_kernel<2>, dim3(blocks), dim3(256), 0, s, logits, T, E, k, renormalize, ids, w);
   else if (epl <= 4)
-    route_kernel<4><<<blocks, 256, 0, s>>>(logits, T, E, k, renormalize, ids, w);
+    (void)launch_kernel(route_kernel<4>, dim3(blocks), dim3(256), 0, s, logits, T, E, k, renormalize, ids, w);
   else if (epl <= 8)
-    route_kernel<8><<<blocks, 256, 0, s>>>(logits, T, E, k, renormalize, ids, w);
+    (void)launch_kernel(route_kernel<8>, dim3(blocks), dim3(256), 0, s, logits, T, E, k, renormalize, ids, w);
   else if (epl <= 16)
-    route_kernel<16><<<blocks, 256, 0, s>>>(logits, T, E, k, renormalize, ids, w);
+    (void)launch_kernel(route_kernel<16>, dim3(blocks), dim3(256), 0, s, logits, T, E, k, renormalize, ids, w);
   else
-    route_kernel<32><<<blocks, 256, 0, s>>>(logits, T, E, k, renormalize, ids, w);
+    (void)launch_kernel(route_kernel<32>, dim3(blocks), dim3(256), 0, s, logits, T, E, k, renormalize, ids, w);
   timing_after("route", s);
   return cudaGetLastError();
 }
@@ -151,6 +152,7 @@ __device__ __forceinline__ void expert_tiles(int c, int nmax, int* nt, int* ch) 
 // ------------------------------------------------------------------ align kernels
 __global__ void __launch_bounds__(256) align_hist_kernel(const int32_t* __restrict__ ids, int P, int E,
                                                          int32_t* __restrict__ blockcnt) {
+  grid_dependency_sync();  // see common.cuh
   __shared__ int cnt[1024];
   for (int e = threadIdx.x; e < E; e += blockDim.x) cnt[e] = 0;
   __syncthreads();
@@ -171,6 +173,7 @@ __global__ void __launch_bounds__(1024) align_scan_kernel(int32_t* __restrict__ 
                                                           int P, int32_t* __restrict__ counts,
                                                           int32_t* __restrict__ offsets,
                                                           int32_t* __restrict__ sorted_ids, SchedOut sch) {
+  grid_dependency_sync();  // see common.cuh
   __shared__ int warp_tot[32];
   __shared__ int total;
   const int e = threadIdx.x;
@@ -230,6 +233,7 @@ __global__ void __launch_bounds__(32) align_scatter_kernel(const int32_t* __rest
                                                            const int32_t* __restrict__ offsets,
                                                            int32_t* __restrict__ sorted_ids,
                                                            int32_t* __restrict__ inv_pos) {
+  grid_dependency_sync();  // see common.cuh
   __shared__ int cur[1024];
   const int lane = threadIdx.x;
   for (int e = lane; e < E; e += 32) cur[e] = offsets[e] + blockbase[(size_t)blockIdx.x * E + e];
@@ -261,14 +265,14 @@ cudaError_t launch_align(const int32_t* ids, int T, int k, int E, int align, int
   const int P = T * k;
   const int nb = align_blocks(T, k);
   timing_before("align_hist", s);
-  align_hist_kernel<<<nb, 256, 0, s>>>(ids, P, E, blockcnt);
+  (void)launch_kernel(align_hist_kernel, dim3(nb), dim3(256), 0, s, ids, P, E, blockcnt);
   timing_after("align_hist", s);
   timing_before("align_scan", s);
   SchedOut none{};
-  align_scan_kernel<<<1, 1024, 0, s>>>(blockcnt, nb, E, align, P, counts, offsets, sorted_ids, sched ? *sched : none);
+  (void)launch_kernel(align_scan_kernel, dim3(1), dim3(1024), 0, s, blockcnt, nb, E, align, P, counts, offsets, sorted_ids, sched ? *sched : none);
   timing_after("align_scan", s);
   timing_before("align_scatter", s);
-  align_scatter_kernel<<<nb, 32, 0, s>>>(ids, P, E, blockcnt, offsets, sorted_ids, inv_pos);
+  (void)launch_kernel(align_scatter_kernel, dim3(nb), dim3(32), 0, s, ids, P, E, blockcnt, offsets, sorted_ids, inv_pos);
   timing_after("align_scatter", s);
   return cudaGetLastError();
 }
@@ -278,6 +282,7 @@ __global__ void __launch_bounds__(1024) sched_from_offsets_kernel(const int32_t*
                                                                   int nmax, int32_t* __restrict__ row_count,
                                                                   int32_t* __restrict__ tile_prefix,
                                                                   int32_t* __restrict__ chunk) {
+  grid_dependency_sync();  // see common.cuh
   __shared__ int warp_tot[32];
   __shared__ int total;
   const int e = threadIdx.x;
@@ -304,7 +309,7 @@ __global__ void __launch_bounds__(1024) sched_from_offsets_kernel(const int32_t*
 cudaError_t launch_sched_from_offsets(const int32_t* offsets, int E, int M, int nmax, int32_t* row_count,
                                       int32_t* tile_prefix, int32_t* chunk, cudaStream_t s) {
   timing_before("sched", s);
-  sched_from_offsets_kernel<<<1, 1024, 0, s>>>(offsets, E, M, nmax, row_count, tile_prefix, chunk);
+  (void)launch_kernel(sched_from_offsets_kernel, dim3(1), dim3(1024), 0, s, offsets, E, M, nmax, row_count, tile_prefix, chunk);
   timing_after("sched", s);
   return cudaGetLastError();
 }
