@@ -56,6 +56,20 @@ W13_BYTES_PER_EXPERT = 2 * 2048 * 7168 // 2 + 2 * 2048 * (7168 // 32) * 2   # IN
 W2_BYTES_PER_EXPERT = 7168 * 2048 // 2 + 7168 * (2048 // 32) * 2
 
 
+# Datasheet figures of a B200 (HGX): HBM3e 8 TB/s; dense tensor 2.25 PFLOP/s bf16/fp16, 4.5 fp8.
+# Every fraction is reported against the measured peak (`frac`) and against these (`frac_spec`).
+SPEC = dict(hbm=8000.0, bf16=2250.0, fp8=4500.0, src="vendor datasheet (HGX B200)")
+
+
+def with_spec(roof: dict, spec_peak: float) -> dict:
+    """`roof` plus the same achieved figure as a fraction of the datasheet peak."""
+    roof = dict(roof)
+    roof["spec_peak"] = spec_peak
+    roof["frac_spec"] = round(roof["achieved"] / spec_peak, 4)
+    roof["spec_source"] = SPEC["src"]
+    return roof
+
+
 def load_peaks():
     p = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(p):
@@ -312,14 +326,16 @@ def run_gemm(args, world, rank):
     hbm_bound = flops / bytes_ < peaks["bf16"] * 1e3 / peaks["hbm"]
     if hbm_bound:
         ach = bytes_ / s_ / 1e9
-        roof = dict(kernel="all", bound="hbm", achieved=round(ach, 1), peak=peaks["hbm"], unit="GB/s",
-                    frac=round(ach / peaks["hbm"], 4), traffic=None, peak_source=peaks["src"] + " (copy, burst)",
-                    algorithmic_bytes_per_launch=int(bytes_))
+        roof = with_spec(dict(kernel="all", bound="hbm", achieved=round(ach, 1), peak=peaks["hbm"], unit="GB/s",
+                              frac=round(ach / peaks["hbm"], 4), traffic=None,
+                              peak_source=peaks["src"] + " (copy, burst)", algorithmic_bytes_per_launch=int(bytes_)),
+                         SPEC["hbm"])
     else:
         ach = flops / s_ / 1e12
-        roof = dict(kernel="all", bound="tensor", achieved=round(ach, 1), peak=peaks["bf16"], unit="TFLOP/s",
-                    frac=round(ach / peaks["bf16"], 4), traffic=None, peak_source=peaks["src"] + " bf16 GEMM, burst",
-                    algorithmic_flops_per_launch=flops)
+        roof = with_spec(dict(kernel="all", bound="tensor", achieved=round(ach, 1), peak=peaks["bf16"],
+                              unit="TFLOP/s", frac=round(ach / peaks["bf16"], 4), traffic=None,
+                              peak_source=peaks["src"] + " bf16 GEMM, burst", algorithmic_flops_per_launch=flops),
+                         SPEC["bf16"])
     return {
         "metric": GEMM_METRIC, "value": round(ms_step * 1e3, 2), "unit": "µs/GEMM", "n_gpus": world,
         "steps": steps, "warmup": warmup, "ms_per_step": round(ms_step, 4), "higher_is_better": False,
@@ -332,7 +348,7 @@ def run_gemm(args, world, rank):
     }
 
 
-def _phase_roofline(kern, suffix, alg_bytes, alg_flops, t_peak, t_peak_src, peaks, traffic):
+def _phase_roofline(kern, suffix, alg_bytes, alg_flops, t_peak, t_peak_src, peaks, traffic, t_spec):
     """Roofline of one GEMM phase (gate/up or down): the kernels whose names end with `suffix`
     (one launch each per step: the int8-MMA kernel for experts with few rows, the fp16 one for
     the rest), algorithmic bytes / flops of the phase over their summed time per step."""
@@ -348,11 +364,12 @@ def _phase_roofline(kern, suffix, alg_bytes, alg_flops, t_peak, t_peak_src, peak
                   traffic=traffic, algorithmic_bytes_per_launch=int(alg_bytes), algorithmic_flops_per_launch=alg_flops)
     if hbm_bound:
         ach = alg_bytes / per_s / 1e9
-        return dict(bound="hbm", achieved=round(ach, 1), peak=peaks["hbm"], unit="GB/s",
-                    frac=round(ach / peaks["hbm"], 4), peak_source=peaks["src"] + " (copy, burst)", **common)
+        return with_spec(dict(bound="hbm", achieved=round(ach, 1), peak=peaks["hbm"], unit="GB/s",
+                              frac=round(ach / peaks["hbm"], 4), peak_source=peaks["src"] + " (copy, burst)",
+                              **common), SPEC["hbm"])
     ach = alg_flops / per_s / 1e12
-    return dict(bound="tensor", achieved=round(ach, 1), peak=t_peak, unit="TFLOP/s", frac=round(ach / t_peak, 4),
-                peak_source=t_peak_src, **common)
+    return with_spec(dict(bound="tensor", achieved=round(ach, 1), peak=t_peak, unit="TFLOP/s",
+                          frac=round(ach / t_peak, 4), peak_source=t_peak_src, **common), t_spec)
 
 
 def measure_layer(args, workload, W, world):
@@ -528,7 +545,8 @@ def measure_layer(args, workload, W, world):
         traffic = None
         if len(names) == 1 and not no_traffic:
             traffic = load_traffic(workload, names[0], family)
-        phases[suffix] = _phase_roofline(kern, suffix, alg_b, alg_f, t_peak, t_peak_src, peaks, traffic)
+        phases[suffix] = _phase_roofline(kern, suffix, alg_b, alg_f, t_peak, t_peak_src, peaks, traffic,
+                                         SPEC["fp8" if kind == "fp8" else "bf16"])
     dom = max((v for v in phases.values() if v), key=lambda r: r["launch_ms"], default=None)
     launches = sum(n for (_, n) in kern.values())
     res = {
@@ -545,6 +563,9 @@ def measure_layer(args, workload, W, world):
                   "hbm_gbs": round(layer_bytes / (ms_step * 1e-3) / 1e9, 1),
                   "hbm_frac": round(layer_bytes / (ms_step * 1e-3) / 1e9 / peaks["hbm"], 4),
                   "tensor_frac": round(flops / (ms_step * 1e-3) / 1e12 / t_peak, 4),
+                  "hbm_frac_spec": round(layer_bytes / (ms_step * 1e-3) / 1e9 / SPEC["hbm"], 4),
+                  "tensor_frac_spec": round(flops / (ms_step * 1e-3) / 1e12 / SPEC["fp8" if kind == "fp8" else "bf16"],
+                                            4),
                   "algorithmic_bytes": int(layer_bytes), "flops": flops},
         "kernels_ms_per_step": {n: round(v[0] / steps, 4) for n, v in sorted(kern.items(), key=lambda kv: -kv[1][0])},
         "e2e": {"value": round(ms_e2e * 1e3, 2), "unit": "µs/layer", "h2d_bytes_per_step": h2d,

@@ -115,3 +115,14 @@ def test_reference_arm_gemm_line():
     line = bench.run_reference(_args("gemm_m1_k7168_n512"), 1, 0)
     _check_reference_line(line, bench.GEMM_METRIC, "µs/GEMM")
     assert line["config"] == bench.gemm_config(1, 7168, 512)
+
+
+def test_fractions_against_measured_and_datasheet_peaks():
+    """Every roofline object carries the achieved figure over the measured peak and over the
+    datasheet peak, each named."""
+    import bench
+    r = bench.with_spec(dict(bound="hbm", achieved=6000.0, peak=6534.8, unit="GB/s", frac=round(6000 / 6534.8, 4)),
+                        bench.SPEC["hbm"])
+    assert r["frac"] == round(6000 / 6534.8, 4)
+    assert r["frac_spec"] == 0.75 and r["spec_peak"] == 8000.0 and "datasheet" in r["spec_source"]
+    assert bench.SPEC["bf16"] == 2250.0 and bench.SPEC["fp8"] == 2 * bench.SPEC["bf16"]
