@@ -157,8 +157,11 @@ def moe_w4a16_gemm(a, w_q, w_s, expert_offsets, out=None, out_fp32: bool = False
     E, N = w_q.shape[0], w_q.shape[1]
     if a.dtype not in (torch.bfloat16, torch.float16):
         raise ValueError("a must be bf16 or fp16")
+    want = torch.float32 if out_fp32 else torch.bfloat16
     if out is None:
-        out = torch.empty(M, N, dtype=torch.float32 if out_fp32 else torch.bfloat16, device=a.device)
+        out = torch.empty(M, N, dtype=want, device=a.device)
+    elif out.dtype != want or tuple(out.shape) != (M, N):
+        raise ValueError(f"out must be {want} [{M}, {N}] (out_fp32={out_fp32})")
     nbytes = lib.moe_w4a16_gemm_workspace_size(M, K, N, E)
     ws = _workspace(nbytes, workspace, a.device)
     check(lib.moe_w4a16_gemm(_p(a), int(a.dtype == torch.bfloat16), _p(w_q), _p(w_s), _p(expert_offsets), M, K, N,

@@ -214,7 +214,7 @@ FwdWs carve_w4_forward(void* ws, int T, int H, int I, int E, int k) {
 // shape-only rule, so the workspace size needs no device.
 int gemm_splits(int M, int K, int N) {
   const int tile_rows = use_i8(M) ? kI8TileRows : kWideTileRows;
-  const int weight_rows = use_i8(M) ? 128 * w4i8_tiles_per_item(false, N) : 128;  // per work item
+  const int weight_rows = 128 * (use_i8(M) ? w4i8_tiles_per_item(false, N) : w4a16_tiles_per_item(N));  // per item
   const int nkb = (K + 255) / 256;
   const int items = (N / weight_rows) * ((M + tile_rows - 1) / tile_rows);
   int s = 148 / (items > 0 ? items : 1);

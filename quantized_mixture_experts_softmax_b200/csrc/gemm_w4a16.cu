@@ -60,25 +60,30 @@ constexpr int kActWarp = 3;
 constexpr int kEpiWarp0 = 4;  // warps 4-7: epilogue
 constexpr int kDqWarp0 = 8;   // warps 8-15: dequantization
 constexpr int kNumDq = 8;
-constexpr int kMmaWarpUp = kDqWarp0 + kNumDq;  // warp 16 (gate/up GEMM only)
-template <bool GATED>
-constexpr int threads() { return (kDqWarp0 + kNumDq + (GATED ? 1 : 0)) * 32; }
+constexpr int kMmaWarpUp = kDqWarp0 + kNumDq;  // warp 16: the second tile's issuer (NA = 2)
+template <int NA>
+constexpr int threads() { return (kDqWarp0 + kNumDq + (NA == 2 ? 1 : 0)) * 32; }
 constexpr int kMmaBarrier = 1;  // named barriers 1 (gate/only) and 2 (up) of an MMA warp and the
                                 // scheduler warp (0 is __syncthreads)
 static_assert(NMAX % 32 == 0 && NMAX <= 256, "token tile");
 
-template <bool GATED>
+// NA_ = 128-row weight tiles per work item: gate and up (gate/up GEMM), or two adjacent tiles
+// of the output (down GEMM with rows in 256s: twice the MMAs per 64-K hand-off, whose fixed cost
+// made the one-tile down GEMM the less efficient of the two), else one.
+template <bool GATED, int NA_>
 struct Cfg {
-  static constexpr int NA = GATED ? 2 : 1;
+  static_assert(NA_ == 1 || NA_ == 2, "one or two weight tiles per item");
+  static_assert(!GATED || NA_ == 2, "gate and up tiles");
+  static constexpr int NA = NA_;
   static constexpr int NSUB = KB / KS;               // 64-K steps per weight stage
   static constexpr int W_TILE = BM * KB / 2;         // packed INT4 bytes of one 128-row tile
   static constexpr int S_TILE = BM * (KB / 32) * 2;  // its bf16 scales
   static constexpr int W_STAGE = NA * (W_TILE + S_TILE);
   static constexpr int B_ATOM = NMAX * KS * 2;       // activation tile of one 64-K step
   // ring depths: weight stages, activation tiles, A slots in tensor memory
-  static constexpr int WST = GATED ? 3 : 2;
-  static constexpr int BST = GATED ? 4 : 7;
-  static constexpr int ABUF = GATED ? 2 : 4;
+  static constexpr int WST = NA == 2 ? 3 : 2;
+  static constexpr int BST = NA == 2 ? 4 : 7;
+  static constexpr int ABUF = NA == 2 ? 2 : 4;
   static constexpr int ACC_COLS = NA * NMAX;         // [matrix][NMAX] fp32 columns
   static constexpr int ACC_BUFS = (2 * ACC_COLS + ABUF * NA * (KS / 2) <= 512) ? 2 : 1;
   static constexpr int A_COLS = KS / 2;              // a 64-K fp16 row of one tile = 32 TMEM columns
@@ -105,6 +110,7 @@ struct BoxMaps {
 
 struct Params {
   int K, E, rows_per_expert, I, m_tiles;
+  int row_off2;    // NA = 2: rows of the second tile after the first (I for gate/up, 128 for down)
   int scales_tma;  // 1: weight scales by TMA (K % 256 == 0), else by cp.async
   const uint16_t* w_s;
   TileSched sched;
@@ -191,11 +197,11 @@ __device__ __forceinline__ int interleave_pos(int j) {
   return (j & ~7) | (r < 4 ? 2 * r : 2 * (r - 4) + 1);
 }
 
-template <bool GATED>
-__global__ void __launch_bounds__(threads<GATED>(), 1)
+template <bool GATED, int NA_>
+__global__ void __launch_bounds__(threads<NA_>(), 1)
     w4a16_gemm_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CUtensorMap tm_s,
                       const __grid_constant__ BoxMaps tm_b, const Params p) {
-  using C = Cfg<GATED>;
+  using C = Cfg<GATED, NA_>;
   constexpr int NA = C::NA, WST = C::WST, BST = C::BST, ABUF = C::ABUF, ACCB = C::ACC_BUFS, NSUB = C::NSUB;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -268,8 +274,8 @@ __global__ void __launch_bounds__(threads<GATED>(), 1)
     bool ok = true;
     for (int it = blockIdx.x; it < total && ok; it += gridDim.x) {
       const Item I = decode_item(it, sprefix, p);
-      const int row_g = I.e * p.rows_per_expert + I.m * BM;
-      const int row_u = row_g + p.I;  // gated: the up tile
+      const int row_g = I.e * p.rows_per_expert + I.m * (GATED ? BM : NA * BM);  // first tile
+      const int row_u = row_g + p.row_off2;                                      // second tile
       int kb0, kb1;
       split_range(it, nkb, p.splits, kb0, kb1);
       for (int kb = kb0; kb < kb1; ++kb) {
@@ -278,10 +284,11 @@ __global__ void __launch_bounds__(threads<GATED>(), 1)
         if (lane == 0) {
           mbar_arrive_expect_tx(&full_w[ws], (uint32_t)(NA * C::W_TILE + (p.scales_tma ? NA * C::S_TILE : 0)));
           tma_load_2d_hint(st, &tm_w, &full_w[ws], kb * (KB / 8), row_g, pol_w);
-          if (GATED) tma_load_2d_hint(st + C::W_TILE, &tm_w, &full_w[ws], kb * (KB / 8), row_u, pol_w);
+          if (NA == 2) tma_load_2d_hint(st + C::W_TILE, &tm_w, &full_w[ws], kb * (KB / 8), row_u, pol_w);
           if (p.scales_tma) {
             tma_load_2d_hint(st + NA * C::W_TILE, &tm_s, &full_w[ws], kb * (KB / 32), row_g, pol_w);
-            if (GATED) tma_load_2d_hint(st + NA * C::W_TILE + C::S_TILE, &tm_s, &full_w[ws], kb * (KB / 32), row_u, pol_w);
+            if (NA == 2)
+              tma_load_2d_hint(st + NA * C::W_TILE + C::S_TILE, &tm_s, &full_w[ws], kb * (KB / 32), row_u, pol_w);
           }
         }
         if (!p.scales_tma) {  // scale rows 8-byte aligned: 8 or 4 bf16 per row by cp.async
@@ -307,7 +314,7 @@ __global__ void __launch_bounds__(threads<GATED>(), 1)
     }
     if (lane == 0)
       for (int i = max(0, issued - WST); i < issued; ++i) mbar_wait_plain(&full_w[i % WST], (i / WST) & 1, lim);
-  } else if (warp == kMmaWarp || (GATED && warp == kMmaWarpUp)) {
+  } else if (warp == kMmaWarp || (NA == 2 && warp == kMmaWarpUp)) {
     // ---------------------------------------------------------------- MMA issuers
     // One per matrix, each released step by step by the scheduler warp on its own named barrier;
     // identical loop bounds on all three sides.
@@ -368,7 +375,7 @@ __global__ void __launch_bounds__(threads<GATED>(), 1)
           ready = ready && __all_sync(0xffffffffu, mbar_wait(&a_full[ab], ph_a, abort_flag, lim)) &&
                   __all_sync(0xffffffffu, mbar_wait(&full_b[bs], ph_b, abort_flag, lim));
           ok = bar_red_and(kMmaBarrier, 64, ready);
-          if (GATED) bar_red_and(kMmaBarrier + 1, 64, ok);  // the up issuer takes the same step
+          if (NA == 2) bar_red_and(kMmaBarrier + 1, 64, ok);  // the second issuer takes the same step
           if (!ok) break;
           if (++ab == ABUF) {
             ab = 0;
@@ -441,7 +448,7 @@ __global__ void __launch_bounds__(threads<GATED>(), 1)
       for (int c0 = 0; c0 < I.nmma; c0 += 16) {
         uint32_t g[16], u[16];
         tmem_ld16(tb + c0, g);
-        if (GATED) tmem_ld16(tb + NMAX + c0, u);
+        if (NA == 2) tmem_ld16(tb + NMAX + c0, u);
         tmem_ld_wait();
         const int nv = min(16, I.nvalid - c0);
         if (p.acc_exp) {  // rows whose fp16 operand was scaled by 2^-e to fit fp16: undo it
@@ -449,7 +456,7 @@ __global__ void __launch_bounds__(threads<GATED>(), 1)
           for (int i = 0; i < 16; ++i) {
             const float sc = exp2_int(rexp[c0 + i]);  // the same word for every lane: a broadcast
             g[i] = __float_as_uint(__uint_as_float(g[i]) * sc);
-            if (GATED) u[i] = __float_as_uint(__uint_as_float(u[i]) * sc);
+            if (NA == 2) u[i] = __float_as_uint(__uint_as_float(u[i]) * sc);
           }
         }
         if (GATED) {
@@ -485,21 +492,30 @@ __global__ void __launch_bounds__(threads<GATED>(), 1)
             }
             if (huge) set_status(MOE_ERR_DEVICE_CHECK);
           }
-        } else if (p.splits > 1) {  // this split's partial sum, reduced in split order by another kernel
-          float* out = p.part + (size_t)(it % p.splits) * p.act_rows * p.out_ld + (size_t)(I.r0 + c0) * p.out_ld + col;
-#pragma unroll
-          for (int i = 0; i < 16; ++i)
-            if (i < nv) out[(size_t)i * p.out_ld] = __uint_as_float(g[i]);
-        } else if (p.out_kind == OUT_F32) {
-          float* out = reinterpret_cast<float*>(p.out) + (size_t)(I.r0 + c0) * p.out_ld + col;
-#pragma unroll
-          for (int i = 0; i < 16; ++i)
-            if (i < nv) out[(size_t)i * p.out_ld] = __uint_as_float(g[i]);
         } else {
-          __nv_bfloat16* out = reinterpret_cast<__nv_bfloat16*>(p.out) + (size_t)(I.r0 + c0) * p.out_ld + col;
+          // plain output: the item's NA tiles, output columns m * NA * 128 + mat * 128 + row
 #pragma unroll
-          for (int i = 0; i < 16; ++i)
-            if (i < nv) out[(size_t)i * p.out_ld] = __float2bfloat16_rn(__uint_as_float(g[i]));
+          for (int mat = 0; mat < NA; ++mat) {
+            const uint32_t* v = mat ? u : g;
+            const int ncol = I.m * (NA * BM) + mat * BM + mrow;
+            if (p.splits > 1) {  // this split's partial sum, reduced in split order by another kernel
+              float* out =
+                  p.part + (size_t)(it % p.splits) * p.act_rows * p.out_ld + (size_t)(I.r0 + c0) * p.out_ld + ncol;
+#pragma unroll
+              for (int i = 0; i < 16; ++i)
+                if (i < nv) out[(size_t)i * p.out_ld] = __uint_as_float(v[i]);
+            } else if (p.out_kind == OUT_F32) {
+              float* out = reinterpret_cast<float*>(p.out) + (size_t)(I.r0 + c0) * p.out_ld + ncol;
+#pragma unroll
+              for (int i = 0; i < 16; ++i)
+                if (i < nv) out[(size_t)i * p.out_ld] = __uint_as_float(v[i]);
+            } else {
+              __nv_bfloat16* out = reinterpret_cast<__nv_bfloat16*>(p.out) + (size_t)(I.r0 + c0) * p.out_ld + ncol;
+#pragma unroll
+              for (int i = 0; i < 16; ++i)
+                if (i < nv) out[(size_t)i * p.out_ld] = __float2bfloat16_rn(__uint_as_float(v[i]));
+            }
+          }
         }
       }
       tc_fence_before();
@@ -519,9 +535,9 @@ __global__ void __launch_bounds__(threads<GATED>(), 1)
     const int dw = warp - kDqWarp0;
     const int row = (dw & 3) * 32 + lane;
     const int sw = row & 7;
-    const int mat = GATED ? (dw >> 2) : 0;
-    const int half = GATED ? 0 : (dw >> 2);
-    constexpr int CHK = GATED ? 8 : 4;  // 16-byte chunks of packed words this thread takes per stage
+    const int mat = NA == 2 ? (dw >> 2) : 0;
+    const int half = NA == 2 ? 0 : (dw >> 2);
+    constexpr int CHK = NA == 2 ? 8 : 4;  // 16-byte chunks of packed words this thread takes per stage
     const uint32_t lane_base = tmem_base + ((uint32_t)((dw & 3) * 32) << 16);
     int ws = 0, ab = 0;
     uint32_t ph_w = 0, ph_a = 0;
@@ -538,7 +554,7 @@ __global__ void __launch_bounds__(threads<GATED>(), 1)
         uint4 wv[CHK];
 #pragma unroll
         for (int c = 0; c < CHK; ++c) {
-          const int lc = GATED ? c : 2 * c + half;  // logical 16-byte chunk (32 K) of the stage
+          const int lc = NA == 2 ? c : 2 * c + half;  // logical 16-byte chunk (32 K) of the stage
           wv[c] = *reinterpret_cast<const uint4*>(wrow + ((lc ^ sw) << 4));
         }
         __syncwarp();
@@ -555,7 +571,7 @@ __global__ void __launch_bounds__(threads<GATED>(), 1)
             if (!ok) break;
             tc_fence_after();  // the MMAs that last read this A slot have completed
             const uint32_t col = (uint32_t)(C::A_COL0 + (ab * NA + mat) * C::A_COLS);
-            if constexpr (GATED) {
+            if constexpr (NA == 2) {
               uint32_t r[32];
 #pragma unroll
               for (int q = 0; q < 2; ++q) {
@@ -600,9 +616,9 @@ __global__ void __launch_bounds__(threads<GATED>(), 1)
   }
 }
 
-template <bool GATED>
+template <bool GATED, int NA_>
 cudaError_t launch_t(const W4GemmProblem& pr, cudaStream_t s) {
-  using C = Cfg<GATED>;
+  using C = Cfg<GATED, NA_>;
   CUtensorMap tm_w, tm_s;
   BoxMaps tm_b;
   const uint64_t wrows = (uint64_t)pr.E * pr.rows_per_expert;
@@ -626,7 +642,8 @@ cudaError_t launch_t(const W4GemmProblem& pr, cudaStream_t s) {
   p.E = pr.E;
   p.rows_per_expert = pr.rows_per_expert;
   p.I = pr.I;
-  p.m_tiles = GATED ? pr.I / BM : pr.rows_per_expert / BM;
+  p.m_tiles = GATED ? pr.I / BM : pr.rows_per_expert / (NA_ * BM);
+  p.row_off2 = GATED ? pr.I : BM;
   p.scales_tma = scales_tma;
   p.w_s = pr.w_s;
   p.sched = pr.sched;
@@ -642,21 +659,24 @@ cudaError_t launch_t(const W4GemmProblem& pr, cudaStream_t s) {
   if (GATED && (!p.ovf_flag || !p.ovf_mask)) return cudaErrorInvalidValue;
   p.wait_limit = wait_limit_ns();
   const size_t smem = C::smem_bytes(pr.E);
-  auto kern = w4a16_gemm_kernel<GATED>;
+  auto kern = w4a16_gemm_kernel<GATED, NA_>;
   cudaError_t err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (err != cudaSuccess) return err;
   const char* name = GATED ? "w4a16_gemm_gate_up" : "w4a16_gemm_down";
   timing_before(name, s);
-  (void)launch_kernel(kern, dim3(sm_count()), dim3(threads<GATED>()), smem, s, tm_w, tm_s, tm_b, p);
+  (void)launch_kernel(kern, dim3(sm_count()), dim3(threads<NA_>()), smem, s, tm_w, tm_s, tm_b, p);
   timing_after(name, s);
   return cudaGetLastError();
 }
 
 }  // namespace w4
 
+int w4a16_tiles_per_item(int rows) { return rows % 256 == 0 ? 2 : 1; }
+
 cudaError_t launch_w4a16_gemm(const W4GemmProblem& p, cudaStream_t s) {
   if (p.nmax > w4::NMAX) return cudaErrorInvalidValue;
-  return p.gated ? w4::launch_t<true>(p, s) : w4::launch_t<false>(p, s);
+  if (p.gated) return w4::launch_t<true, 2>(p, s);
+  return w4a16_tiles_per_item(p.rows_per_expert) == 2 ? w4::launch_t<false, 2>(p, s) : w4::launch_t<false, 1>(p, s);
 }
 
 }  // namespace moe

@@ -155,6 +155,9 @@ cudaError_t launch_w4i8_gemm(const W4I8Problem& p, cudaStream_t s);
 // 128-row weight tiles per work item of the int8 GEMM: 2 (gate and up, or two adjacent output
 // tiles when the rows come in 256s), else 1
 int w4i8_tiles_per_item(bool gated, int rows_per_expert);
+// 128-row weight tiles per work item of the fp16 GEMM's plain (down) form: 2 when the output rows
+// come in 256s, else 1
+int w4a16_tiles_per_item(int rows_per_expert);
 // out[r][n] = sum over s = 0..splits-1 (in that order) of part[s][r][n] for the rows of every
 // expert e, [row_start[e], row_start[e] + row_count[e]), stored as fp32 (out_fp32) or bf16 (RNE)
 cudaError_t launch_reduce_splits(const float* part, int splits, int rows, int N, const int32_t* row_start,
