@@ -115,7 +115,7 @@ moe_status_t moe_align_noalloc(const int32_t* topk_ids, int T, int k, int E, int
  *   w2_q   int32 [E, H, I/8],  w2_s bf16 [E, H, I/32]   (down projection, same packing)
  *   out    bf16  [T, H] (RNE of the fp32 result), or fp32 [T, H] when out_fp32 != 0
  * Numerics: each expert runs on one of two GEMMs, chosen per expert from its token count (every
- * expert on the first when T <= 64; for larger T an expert with at most 16 rows on the first and
+ * expert on the first when T <= 64; for larger T an expert with at most 8 rows on the first and
  * one with more on the second):
  *   int8 GEMM: the INT4 values meet 16-bit fixed-point activations on the int8 tensor cores:
  *     per (row, 128-K block) s = max(|x|max, 1e-30) / 16383 and X = rint(x / s); each 32-K

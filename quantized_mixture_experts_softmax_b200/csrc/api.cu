@@ -148,10 +148,12 @@ bool use_i8(int max_rows_per_expert) { return max_rows_per_expert <= 64; }
 // plus a promotion step per live token), one with more on the fp16 GEMM (tiles of up to 192
 // rows, where dequantizing a weight tile once serves many tokens, but a tile of few tokens
 // costs as much dequantization as a full one).  Measured on the 384-expert model with skewed
-// routing at T = 128 ... 8192, switch points of 16, 32, 48 and 64 rows: 16 was fastest at
-// every T (T = 8192: 3% faster than 32, 6% faster than the fp16 GEMM alone).
+// routing at T = 128 ... 8192: switch points of 4, 8 and 16 rows (once both GEMMs had their
+// current form; earlier, 16 against 32, 48 and 64), 8 fastest or within 4% of the fastest at
+// every T (T = 8192: 4-6% faster than 16; T = 128 and 512: 20% faster) - one int8 tile of 8
+// rows, where an expert of 9-16 rows took two passes over its weights.
 #ifndef MOE_THIN_ROWS
-#define MOE_THIN_ROWS 16
+#define MOE_THIN_ROWS 8
 #endif
 constexpr int kThinRows = MOE_THIN_ROWS;
 
