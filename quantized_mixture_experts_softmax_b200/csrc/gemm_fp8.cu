@@ -71,6 +71,7 @@ struct Cfg {
   // that each token's 32 bytes leave in two 16-byte stores
   static constexpr int OFF_TR = OFF_CS + kNumEpi * 2 * NH * 4;
   static constexpr int OFF_PREFIX = OFF_TR + (GATED ? kNumEpi * NH * 32 : 0);
+  static_assert(OFF_TR % 16 == 0, "the transpose tiles are read as 16-byte vectors");
   static_assert(OFF_CS % 16 == 0, "float4 reads of the block scales");
   static_assert(STAGE % 1024 == 0, "swizzled tiles need 1024-byte alignment");
   static constexpr size_t smem_bytes(int E) { return (size_t)OFF_PREFIX + 4 * (size_t)(E + 1) + 1024; }

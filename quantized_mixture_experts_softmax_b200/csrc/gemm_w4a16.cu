@@ -93,7 +93,12 @@ struct Cfg {
   static constexpr int OFF_BAR = OFF_B + BST * B_ATOM;
   static constexpr int NUM_BARS = 2 * WST + 2 * BST + 2 * ABUF + 2 * ACC_BUFS + 1;
   static constexpr int OFF_MISC = OFF_BAR + NUM_BARS * 8;
-  static constexpr int OFF_PREFIX = OFF_MISC + 16;
+  // per epilogue warp a [16 tokens][32 rows] fp16 staging tile of a 16-column chunk of h, so
+  // that each token's 32 values (64 bytes) leave in 16-byte stores
+  static constexpr int STG_BYTES = 16 * 32 * 2;
+  static constexpr int OFF_STG = (OFF_MISC + 16 + 127) / 128 * 128;  // read as 16-byte vectors
+  static_assert(OFF_STG % 16 == 0 && STG_BYTES % 16 == 0, "16-byte aligned staging tiles");
+  static constexpr int OFF_PREFIX = OFF_STG + 4 * STG_BYTES;
   static_assert(W_STAGE % 1024 == 0 && W_TILE % 1024 == 0 && OFF_B % 1024 == 0 && B_ATOM % 1024 == 0,
                 "swizzled tiles need 1024-byte alignment");
   static_assert(A_COL0 + ABUF * NA * A_COLS <= 512, "TMEM has 512 columns");
@@ -433,13 +438,21 @@ __global__ void __launch_bounds__(threads<NA_>(), 1)
     const int ew = warp - kEpiWarp0;  // == warp % 4: this warp may read TMEM lanes 32*ew..32*ew+31
     const int mrow = ew * 32 + lane;
     int* rexp = sprefix + p.E + 1 + ew * NMAX;  // this warp's copy of the item's row exponents
+    uint8_t* stg = smem + C::OFF_STG + ew * C::STG_BYTES;
     int acc = 0;
     uint32_t ph = 0;
     for (int it = blockIdx.x; it < total; it += gridDim.x) {
       const Item I = decode_item(it, sprefix, p);
-      // the item's row exponents, loaded while the MMAs run
+      // the item's row exponents, loaded while the MMAs run (almost always all 0: then the
+      // accumulators need no scaling)
+      int nz = 0;
       if (p.acc_exp)
-        for (int rr = lane; rr < I.nmma; rr += 32) rexp[rr] = rr < I.nvalid ? __ldg(p.acc_exp + I.r0 + rr) : 0;
+        for (int rr = lane; rr < I.nmma; rr += 32) {
+          const int e = rr < I.nvalid ? __ldg(p.acc_exp + I.r0 + rr) : 0;
+          rexp[rr] = e;
+          nz |= e;
+        }
+      const bool scale_rows = __any_sync(0xffffffffu, nz != 0);
       __syncwarp();
       if (!__all_sync(0xffffffffu, mbar_wait(&acc_full[acc], ph, abort_flag, lim))) break;
       tc_fence_after();
@@ -451,7 +464,7 @@ __global__ void __launch_bounds__(threads<NA_>(), 1)
         if (NA == 2) tmem_ld16(tb + NMAX + c0, u);
         tmem_ld_wait();
         const int nv = min(16, I.nvalid - c0);
-        if (p.acc_exp) {  // rows whose fp16 operand was scaled by 2^-e to fit fp16: undo it
+        if (scale_rows) {  // rows whose fp16 operand was scaled by 2^-e to fit fp16: undo it
 #pragma unroll
           for (int i = 0; i < 16; ++i) {
             const float sc = exp2_int(rexp[c0 + i]);  // the same word for every lane: a broadcast
@@ -471,9 +484,20 @@ __global__ void __launch_bounds__(threads<NA_>(), 1)
             over |= i < nv && !(fabsf(hv[i]) < 65520.0f);
           }
           if (!__any_sync(0xffffffffu, over)) {
+            // the warp's 32 rows are 32 consecutive positions of h: transpose through shared
+            // memory, then each token's 64 bytes leave as four 16-byte stores
+            __half* sh = reinterpret_cast<__half*>(stg);
 #pragma unroll
-            for (int i = 0; i < 16; ++i)
-              if (i < nv) out[(size_t)i * p.out_ld] = __float2half_rn(hv[i]);
+            for (int i = 0; i < 16; ++i) sh[i * 32 + (pos & 31)] = __float2half_rn(hv[i]);
+            __syncwarp();
+#pragma unroll
+            for (int h2 = 0; h2 < 2; ++h2) {
+              const int i = (lane >> 2) + 8 * h2, q = lane & 3;
+              if (i < nv)
+                *reinterpret_cast<uint4*>(reinterpret_cast<__half*>(p.out) + (size_t)(I.r0 + c0 + i) * p.out_ld +
+                                          (pos & ~31) + q * 8) = *reinterpret_cast<const uint4*>(sh + i * 32 + q * 8);
+            }
+            __syncwarp();
           } else {
             bool huge = false;  // an h beyond even the prescaled fp16 range (2^32)
 #pragma unroll
@@ -505,6 +529,8 @@ __global__ void __launch_bounds__(threads<NA_>(), 1)
               for (int i = 0; i < 16; ++i)
                 if (i < nv) out[(size_t)i * p.out_ld] = __uint_as_float(v[i]);
             } else if (p.out_kind == OUT_F32) {
+              // a warp's store writes 32 consecutive floats (a whole 128-byte line) per token;
+              // staging these through shared memory as for h measured 10% slower
               float* out = reinterpret_cast<float*>(p.out) + (size_t)(I.r0 + c0) * p.out_ld + ncol;
 #pragma unroll
               for (int i = 0; i < 16; ++i)
