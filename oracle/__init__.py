@@ -1,4 +1,4 @@
-"""CPU oracle for the routed W4A16 / block-FP8 MoE layer (test infrastructure only).
+"""CPU oracle for the routed W4A16 / block-FP8 / W4A8 MoE layer (test infrastructure only).
 
 Only ``tests/``, ``__graft_entry__.smoke()`` and the CPU-baseline leg of ``bench.py`` may
 import this package.  The product path never does: it has no CPU fallback.  The oracle
@@ -58,6 +58,13 @@ def lib():
         L.oracle_w4a16_gemm.argtypes = [vp, i32, vp, vp, vp, i32, i32, i32, i32, vp]
         L.oracle_fp8_tokens.argtypes = [vp, vp, vp, vp, i32, i32, i32, i32, i32, vp, vp, vp, vp, vp, i32, vp, vp,
                                         i32]
+        L.oracle_e2m1.restype = ctypes.c_double
+        L.oracle_e2m1.argtypes = [ctypes.c_uint8]
+        L.oracle_e8m0.restype = ctypes.c_double
+        L.oracle_e8m0.argtypes = [ctypes.c_uint8]
+        L.oracle_mx_quant32.restype = ctypes.c_uint8
+        L.oracle_mx_quant32.argtypes = [vp, vp]
+        L.oracle_w4a8_tokens.argtypes = [vp, vp, vp, i32, i32, i32, i32, i32, vp, vp, vp, vp, vp, i32, vp, vp, i32]
         _lib = L
     return _lib
 
@@ -193,4 +200,45 @@ def fp8_tokens(x, xs, ids, w, w13, w13_s, w2, w2_s, tokens=None, want_hq=False, 
     hq = np.empty((n, k, I), np.float32) if want_hq else None
     lib().oracle_fp8_tokens(xp, xsp, idp, wp, T, H, I, E, k, a13p, b13p, a2p, b2p, tok.ctypes.data, n,
                             out.ctypes.data, hq.ctypes.data if want_hq else None, threads or nthreads())
+    return (out, hq) if want_hq else out
+
+
+def e2m1(c: int) -> float:
+    return lib().oracle_e2m1(c)
+
+
+def e8m0(c: int) -> float:
+    return lib().oracle_e8m0(c)
+
+
+def mx_quant32(v):
+    """32 fp32 values -> (e4m3 codes uint8 [32], E8M0 scale code)."""
+    v_c, vp = _c(v, np.float32)
+    assert v_c.shape == (32,)
+    q = np.empty(32, np.uint8)
+    sc = lib().oracle_mx_quant32(vp, q.ctypes.data)
+    return q, sc
+
+
+def w4a8_tokens(x, ids, w, w13, w13_sf, w2, w2_sf, tokens=None, want_hq=False, threads=None):
+    """Routed W4A8 (MXFP4 weights, MX-FP8 activations) layer output in fp64 for `tokens`."""
+    x_c, xp = _c(x, np.uint16)
+    ids_c, idp = _c(ids, np.int32)
+    w_c, wp = _c(w, np.float32)
+    a13, a13p = _c(w13, np.uint8)
+    b13, b13p = _c(w13_sf, np.uint8)
+    a2, a2p = _c(w2, np.uint8)
+    b2, b2p = _c(w2_sf, np.uint8)
+    T, H = x_c.shape
+    k = ids_c.shape[1]
+    E, twoI = a13.shape[0], a13.shape[1]
+    I = twoI // 2
+    assert a13.shape == (E, 2 * I, H // 2) and b13.shape == (E, H // 128, 2 * I, 4)
+    assert a2.shape == (E, H, I // 2) and b2.shape == (E, I // 128, H, 4)
+    tok = np.arange(T, dtype=np.int32) if tokens is None else np.ascontiguousarray(tokens, np.int32)
+    n = len(tok)
+    out = np.empty((n, H), np.float64)
+    hq = np.empty((n, k, I), np.float32) if want_hq else None
+    lib().oracle_w4a8_tokens(xp, idp, wp, T, H, I, E, k, a13p, b13p, a2p, b2p, tok.ctypes.data, n,
+                             out.ctypes.data, hq.ctypes.data if want_hq else None, threads or nthreads())
     return (out, hq) if want_hq else out

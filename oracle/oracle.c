@@ -3,13 +3,13 @@
  *
  * TEST INFRASTRUCTURE ONLY.  Nothing on the product path may link, load or call this
  * file: only the tests, the package's smoke check and the benchmark's CPU-baseline leg
- * use it.  It shares no code with the CUDA path (its own bf16/fp16/e4m3/INT4 decoders,
+ * use it.  It shares no code with the CUDA path (its own bf16/fp16/e4m3/e2m1/e8m0/INT4 decoders,
  * its own routing, sort, GEMM, activation and combine).
  *
  * What it computes is the plain definition of the layer, written out one token at a time
  * (threads only split the token list), with every dot product accumulated in fp64 in
  * ascending K order and no intermediate rounding except where the method itself rounds
- * (the block-FP8 requantization of the intermediate activation, below).
+ * (the FP8 quantization of the activations in the block-FP8 and W4A8 layers, below).
  *
  * Sources (titles of the pages the method is described on):
  *  - "Chord Rewrites the INT4 MoE Kernel for Kimi K2.x ..." (Chord article), second
@@ -18,6 +18,8 @@
  *  - "Helion Brings Autotuned GEMM Kernels to vLLM ..." (Helion article), section
  *    "Scope: Hopper and quantized formats": Block_FP8 = FP8 with 1x128 activation scaling
  *    and 128x128 weight scaling.
+ *  - "[Performance] W4A8 MoE GEMM significantly slower than W4A16 on H200" (Humming issue),
+ *    the opening report: W4A8 = MXFP4 weights with FP8 activations quantized in K groups.
  *  - "AWS Details H200 Kernel Optimizations for MoE Inference", section "Three bottlenecks
  *    require different fixes": a fused MoE operator = token routing, data movement and
  *    expert calculations.
@@ -416,5 +418,136 @@ void oracle_fp8_tokens(const uint8_t* x, const float* xs, const int32_t* ids, co
                        const int32_t* tokens, int n_tok, double* out, float* hq_out, int nthreads) {
   f8_job J = {x, xs, ids, w, T, H, I, E, k, w13, w2, w13_s, w2_s, tokens, n_tok, out, hq_out, 0, PTHREAD_MUTEX_INITIALIZER};
   run_pool(f8_worker, &J, nthreads);
+  pthread_mutex_destroy(&J.mu);
+}
+
+/* ------------------------------------------------------------------ W4A8 (MXFP4 x FP8) layer */
+
+/* The W4A8 format of the Humming issue ("[Performance] W4A8 MoE GEMM significantly slower than
+   W4A16 on H200", the opening report): weights MXFP4, activations FP8 quantized along K in
+   groups (per token, 32 or 128); this oracle takes the 32-group configuration.  MXFP4 is the
+   OCP microscaling format: FP4 E2M1 elements sharing one E8M0 power-of-two scale per block of
+   32 consecutive K elements.  The pages leave the activation scale's format open; the reading
+   taken is the microscaling one for both operands (an E8M0 power-of-two scale per 32 elements,
+   FP8 E4M3 elements), chosen as the smallest power of two that keeps the group inside E4M3's
+   finite range. */
+
+/* E2M1 code (low 4 bits) -> value: 1 sign bit, 2 exponent bits (bias 1), 1 mantissa bit;
+   exponent field 0 is subnormal (0 or 0.5).  Magnitudes 0, 0.5, 1, 1.5, 2, 3, 4, 6. */
+double oracle_e2m1(uint8_t c) {
+  int s = (c >> 3) & 1, e = (c >> 1) & 3, m = c & 1;
+  double v = e == 0 ? 0.5 * m : ldexp(1.0 + 0.5 * m, e - 1);
+  return s ? -v : v;
+}
+
+/* E8M0 scale code -> 2^(code - 127); code 255 is NaN. */
+double oracle_e8m0(uint8_t c) { return c == 255 ? NAN : ldexp(1.0, (int)c - 127); }
+
+/* One group of 32 fp32 values -> E4M3 codes q and the group's E8M0 scale code.
+   X = the smallest integer >= -127 with amax <= 448 * 2^X (at most 127); q[j] = e4m3(v[j] / 2^X),
+   nearest with ties to even (the division by a power of two is exact).  Returns X + 127. */
+uint8_t oracle_mx_quant32(const float* v, uint8_t* q) {
+  double amax = 0.0;
+  for (int j = 0; j < 32; ++j)
+    if (fabs((double)v[j]) > amax) amax = fabs((double)v[j]);
+  int X = -127;
+  while (X < 127 && amax > ldexp(448.0, X)) ++X;
+  for (int j = 0; j < 32; ++j) q[j] = oracle_e4m3_encode((float)ldexp((double)v[j], -X));
+  return (uint8_t)(X + 127);
+}
+
+/* MXFP4 weight element (n, c) of one expert's [R, K] matrix: codes packed two per byte along K
+   (even K index in the low nibble), [R, K/2]; scale codes [K/128, R, 4] (the scale of K block
+   32*(4*b + j) of row n at [b][n][j]). */
+static inline double mxw(const uint8_t* q, const uint8_t* sf, int R, int K, int n, int c) {
+  uint8_t byte = q[(size_t)n * (K / 2) + c / 2];
+  uint8_t code = (c & 1) ? (byte >> 4) : (byte & 15);
+  return oracle_e2m1(code) * oracle_e8m0(sf[((size_t)(c / 128) * R + n) * 4 + (c / 32) % 4]);
+}
+
+typedef struct {
+  const uint16_t* x;
+  const int32_t* ids;
+  const float* w;
+  int T, H, I, E, k;
+  const uint8_t *w13, *w13_sf, *w2, *w2_sf;
+  const int32_t* tokens;
+  int n_tok;
+  double* out;
+  float* hq_out; /* [n_tok, k, I] dequantized requantized h, or NULL */
+  int next;
+  pthread_mutex_t mu;
+} mx_job;
+
+static void mx_token(mx_job* J, int i) {
+  int t = J->tokens[i], H = J->H, I = J->I, k = J->k;
+  double* xr = (double*)malloc(sizeof(double) * (size_t)H);
+  double* g = (double*)malloc(sizeof(double) * 2 * (size_t)I);
+  float* hf = (float*)malloc(sizeof(float) * (size_t)I);
+  double* hd = (double*)malloc(sizeof(double) * (size_t)I);
+  double* o = J->out + (size_t)i * H;
+  float v[32];
+  uint8_t qc[32];
+  /* the bf16 input row quantized group by group (32 along K), then dequantized */
+  for (int g0 = 0; g0 < H; g0 += 32) {
+    for (int j = 0; j < 32; ++j) v[j] = (float)oracle_bf16(J->x[(size_t)t * H + g0 + j]);
+    double sc = oracle_e8m0(oracle_mx_quant32(v, qc));
+    for (int j = 0; j < 32; ++j) xr[g0 + j] = oracle_e4m3(qc[j]) * sc;
+  }
+  for (int c = 0; c < H; ++c) o[c] = 0.0;
+  for (int s = 0; s < k; ++s) {
+    int e = J->ids[(size_t)t * k + s];
+    double ws = (double)J->w[(size_t)t * k + s];
+    const uint8_t* q13 = J->w13 + (size_t)e * 2 * I * (H / 2);
+    const uint8_t* f13 = J->w13_sf + (size_t)e * (H / 128) * 2 * I * 4;
+    const uint8_t* q2 = J->w2 + (size_t)e * H * (I / 2);
+    const uint8_t* f2 = J->w2_sf + (size_t)e * (I / 128) * H * 4;
+    for (int n = 0; n < 2 * I; ++n) {
+      double acc = 0.0;
+      for (int c = 0; c < H; ++c) acc += xr[c] * mxw(q13, f13, 2 * I, H, n, c);
+      g[n] = acc;
+    }
+    /* h = SiLU(gate) * up held in fp32, requantized in groups of 32 like the input */
+    for (int j = 0; j < I; ++j) hf[j] = (float)(oracle_silu(g[j]) * g[I + j]);
+    for (int g0 = 0; g0 < I; g0 += 32) {
+      double sc = oracle_e8m0(oracle_mx_quant32(hf + g0, qc));
+      for (int j = 0; j < 32; ++j) hd[g0 + j] = oracle_e4m3(qc[j]) * sc;
+    }
+    if (J->hq_out)
+      for (int j = 0; j < I; ++j) J->hq_out[((size_t)i * k + s) * I + j] = (float)hd[j];
+    for (int c = 0; c < H; ++c) {
+      double acc = 0.0;
+      for (int j = 0; j < I; ++j) acc += hd[j] * mxw(q2, f2, H, I, c, j);
+      o[c] += ws * acc;
+    }
+  }
+  free(xr);
+  free(g);
+  free(hf);
+  free(hd);
+}
+
+static void* mx_worker(void* a) {
+  mx_job* J = (mx_job*)a;
+  for (;;) {
+    pthread_mutex_lock(&J->mu);
+    int i = J->next++;
+    pthread_mutex_unlock(&J->mu);
+    if (i >= J->n_tok) break;
+    mx_token(J, i);
+  }
+  return NULL;
+}
+
+/* Routed W4A8 MoE layer output (fp64) for the listed tokens.  x bf16 [T,H]; w13 MXFP4 codes
+   [E,2I,H/2] with scale codes [E,H/128,2I,4]; w2 codes [E,H,I/2] with scale codes
+   [E,I/128,H,4].  Input and SiLU*up activations are quantized to E4M3 with one E8M0 scale per
+   32 along K before each projection. */
+void oracle_w4a8_tokens(const uint16_t* x, const int32_t* ids, const float* w, int T, int H, int I, int E, int k,
+                        const uint8_t* w13, const uint8_t* w13_sf, const uint8_t* w2, const uint8_t* w2_sf,
+                        const int32_t* tokens, int n_tok, double* out, float* hq_out, int nthreads) {
+  mx_job J = {x, ids, w, T, H, I, E, k, w13, w13_sf, w2, w2_sf, tokens, n_tok, out, hq_out, 0,
+              PTHREAD_MUTEX_INITIALIZER};
+  run_pool(mx_worker, &J, nthreads);
   pthread_mutex_destroy(&J.mu);
 }

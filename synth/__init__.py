@@ -14,6 +14,10 @@ Distributions (the workload recipe):
     (nibble j = bits 4j..4j+3 = K index 8*word+j), w13 [E, 2I, H/8], w2 [E, H, I/8];
     bf16 scales bf16(U[0.005, 0.02]) per 32 K elements per output column,
     w13_s [E, 2I, H/32], w2_s [E, H, I/32].
+  * W4A8: MXFP4 weights, codes uniform random bytes (two uniform E2M1 codes each, even K
+    index in the low nibble), w13 [E, 2I, H/2], w2 [E, H, I/2]; E8M0 scale codes uniform in
+    {120, 121, 122} (2^-7 .. 2^-5, so that the weights' spread matches the W4A16 ones) per 32 K
+    elements, laid out [E, H/128, 2I, 4] and [E, I/128, H, 4]; activations bf16 x as above.
   * block-FP8: weights e4m3(N(0,1)) saturated at +-448, w13 [E, 2I, H], w2 [E, H, I];
     fp32 block scales U[0.001, 0.01] per 128x128 block, [E, 2I/128, H/128] and
     [E, H/128, I/128]; activations e4m3 with one fp32 scale per 1x128 group, produced from
@@ -34,7 +38,7 @@ _SRC = os.path.join(_HERE, "synth.c")
 # Tensor ids: each logical tensor draws from its own stream.
 TID = dict(x=1, logits=2, w13_q=3, w13_s=4, w2_q=5, w2_s=6, zipf_perm=7,
            x8=11, w13_8=13, w13_8s=14, w2_8=15, w2_8s=16,
-           a=21, wq=23, ws=24)
+           a=21, wq=23, ws=24, w13_mx=31, w13_mxs=32, w2_mx=33, w2_mxs=34)
 
 W4_SCALE_RANGE = (0.005, 0.02)
 FP8_SCALE_RANGE = (0.001, 0.01)
@@ -167,6 +171,32 @@ def fp8_weights(seed: int, H: int, I: int, experts) -> dict:
         fill_normal_e4m3(seed, TID["w2_8"], e * w2[0].size, w2[i])
         fill_uniform_f32(seed, TID["w2_8s"], e * w2_s[0].size, w2_s[i], lo, hi)
     return dict(w13=w13, w13_s=w13_s, w2=w2, w2_s=w2_s)
+
+
+MX_SCALE_CODES = (120, 121, 122)
+
+
+def _mx_scales(seed, tid, start, out):
+    u = np.empty(out.size, np.uint32)
+    fill_u32(seed, tid, start, u)
+    out.reshape(-1)[:] = (MX_SCALE_CODES[0] + u % len(MX_SCALE_CODES)).astype(np.uint8)
+
+
+def mxfp4_weights(seed: int, H: int, I: int, experts) -> dict:
+    """MXFP4 weights for the listed global expert ids (in that order), slices of the full
+    [E, ...] tensors like w4a16_weights."""
+    experts = list(experts)
+    n = len(experts)
+    w13 = np.empty((n, 2 * I, H // 2), np.uint8)
+    w13_sf = np.empty((n, H // 128, 2 * I, 4), np.uint8)
+    w2 = np.empty((n, H, I // 2), np.uint8)
+    w2_sf = np.empty((n, I // 128, H, 4), np.uint8)
+    for i, e in enumerate(experts):
+        fill_u32(seed, TID["w13_mx"], e * w13[0].size // 4, w13[i].view(np.uint32))
+        _mx_scales(seed, TID["w13_mxs"], e * w13_sf[0].size, w13_sf[i])
+        fill_u32(seed, TID["w2_mx"], e * w2[0].size // 4, w2[i].view(np.uint32))
+        _mx_scales(seed, TID["w2_mxs"], e * w2_sf[0].size, w2_sf[i])
+    return dict(w13=w13, w13_sf=w13_sf, w2=w2, w2_sf=w2_sf)
 
 
 def x_e4m3(seed: int, T: int, H: int, t0: int = 0):

@@ -15,6 +15,7 @@ import pytest
 import oracle
 import test_oracle_formats as F
 import test_oracle_layer as LY
+import test_oracle_mx as MX
 import test_oracle_route_align as RA
 
 SRC = os.path.join(os.path.dirname(oracle.__file__), "oracle.c")
@@ -64,6 +65,22 @@ MUTANTS = [
     ("fp8_gate_up_swapped", "hf[j] = (float)(oracle_silu(g[j]) * g[I + j]);",
      "hf[j] = (float)(oracle_silu(g[I + j]) * g[j]);", 0),
     ("fp8_combine_weight_dropped", "o[c] += ws * acc;", "o[c] += acc;", 1),
+    # W4A8 (MXFP4 x MX-FP8) layer
+    ("e2m1_bias", "ldexp(1.0 + 0.5 * m, e - 1)", "ldexp(1.0 + 0.5 * m, e - 2)", 0),
+    ("e2m1_subnormal", "e == 0 ? 0.5 * m", "e == 0 ? 1.0 * m", 0),
+    ("e8m0_bias", "ldexp(1.0, (int)c - 127)", "ldexp(1.0, (int)c - 128)", 0),
+    ("mx_range_224", "amax > ldexp(448.0, X)", "amax > ldexp(224.0, X)", 0),
+    ("mx_scale_one_too_large", "amax > ldexp(448.0, X)", "amax >= ldexp(448.0, X)", 0),
+    ("mx_zero_group_code", "int X = -127;", "int X = -126;", 0),
+    ("mx_nibble_order", "(c & 1) ? (byte >> 4) : (byte & 15)", "(c & 1) ? (byte & 15) : (byte >> 4)", 0),
+    ("mx_scale_rows_and_blocks_swapped", "sf[((size_t)(c / 128) * R + n) * 4 + (c / 32) % 4]",
+     "sf[((size_t)(n % (K / 128)) * R + (c / 128) % R) * 4 + (c / 32) % 4]", 0),
+    ("mx_scale_group_shifted", "* 4 + (c / 32) % 4]", "* 4 + (c / 32 + 1) % 4]", 0),
+    ("mx_x_not_quantized", "xr[g0 + j] = oracle_e4m3(qc[j]) * sc;", "xr[g0 + j] = v[j];", 0),
+    ("mx_h_not_requantized", "hd[g0 + j] = oracle_e4m3(qc[j]) * sc;", "hd[g0 + j] = hf[g0 + j];", 0),
+    ("mx_gate_up_swapped", "hf[j] = (float)(oracle_silu(g[j]) * g[I + j]);",
+     "hf[j] = (float)(oracle_silu(g[I + j]) * g[j]);", 1),
+    ("mx_combine_weight_dropped", "o[c] += ws * acc;", "o[c] += acc;", 2),
 ]
 
 # the pin tests, called as plain functions
@@ -78,6 +95,9 @@ PINS = [
     LY.test_gate_up_silu_down_closed_form, lambda: LY.test_dense_every_expert_then_mask_matches_routed(0),
     LY.test_e1_k1_is_a_dense_ffn, LY.test_fp8_requant_pins, LY.test_fp8_one_hot_layer,
     lambda: LY.test_fp8_dense_then_mask(0),
+    MX.test_e2m1_all_codes_hand_table, MX.test_e8m0_all_codes_vs_torch, MX.test_mx_quant_scale_pins,
+    MX.test_mx_quant_random_groups_vs_closed_form_and_torch, MX.test_mx_quant_rounding_ties_to_even,
+    MX.test_w4a8_one_hot_layer, lambda: MX.test_w4a8_dense_then_mask(0),
 ]
 
 
