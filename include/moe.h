@@ -14,6 +14,8 @@
  *  - "Helion Brings Autotuned GEMM Kernels to vLLM ...", section "Scope: Hopper and
  *    quantized formats": Block_FP8 = FP8 with 1x128 activation scaling and 128x128 weight
  *    scaling (moe_blockfp8_forward).
+ *  - "[Performance] W4A8 MoE GEMM significantly slower than W4A16 on H200" (Humming issue),
+ *    opening report: W4A8 = MXFP4 weights x FP8 activations in K groups (moe_w4a8_forward).
  *  The router (softmax, top-k, renormalised weights), SiLU*up activation and top-k-weighted
  *  combine are not written out on those pages; this library takes the textbook readings
  *  stated with each call below.
@@ -190,6 +192,51 @@ moe_status_t moe_blockfp8_forward(const moe_blockfp8_args* args, void* ws, size_
  * argument MOE_ERR_INVALID_ARG. */
 moe_status_t moe_blockfp8_intermediate(const void* ws, int T, int H, int I, int E, int k, const int32_t** inv_pos,
                                        const uint8_t** h, const float** h_scale_t);
+
+/* ------------------------------------------------------------------ W4A8 layer
+ * The W4A8 configuration of "[Performance] W4A8 MoE GEMM significantly slower than W4A16 on
+ * H200" (Humming issue, opening report): MXFP4 weights and FP8 activations quantized in groups
+ * of 32 along K.  The same routed layer as moe_w4a16_forward with
+ *   W[e][n][c] = e2m1(code) * 2^(sf - 127)
+ * where code is the 4-bit E2M1 element (sign, 2 exponent bits with bias 1, 1 mantissa bit;
+ * magnitudes 0, .5, 1, 1.5, 2, 3, 4, 6) and sf the E8M0 scale code of the 32-element K group.
+ * The activations (x, then h = SiLU(gate) * up held in fp32) are quantized per token and 32-K
+ * group to E4M3 with an E8M0 scale (the microscaling reading of the report's group-32 FP8):
+ * 2^X is the smallest power of two, X in [-127, 127], with amax <= 448 * 2^X, and the codes are
+ * e4m3_rne(v * 2^-X).  The tensor cores apply both scales per 32 K (tcgen05 block-scaled MMA)
+ * and accumulate the whole reduction in fp32.
+ *   x        bf16 [T, H]
+ *   topk_ids int32 [T, k], topk_w fp32 [T, k] (as moe_route returns them)
+ *   w13      uint8 [E, 2I, H/2]: two E2M1 codes per byte along K, even K index in the low
+ *            nibble; gate rows [0, I), up rows [I, 2I); 32-byte aligned
+ *   w13_sf   uint8 [E, H/128, 2I, 4]: w13_sf[e][b][n][j] = E8M0 code of row n's K group 4b + j
+ *   w2       uint8 [E, H, I/2], w2_sf uint8 [E, I/128, H, 4] (same packing); 32-byte aligned
+ *   out      bf16 [T, H] or fp32 when out_fp32 != 0
+ * An inf or NaN in x or h is flagged in the device status word (MOE_ERR_DEVICE_CHECK).
+ * ws: moe_w4a8_workspace_size(T, H, I, E, k) bytes. */
+typedef struct {
+  const void* x;
+  const int32_t* topk_ids;
+  const float* topk_w;
+  const uint8_t* w13;
+  const uint8_t* w13_sf;
+  const uint8_t* w2;
+  const uint8_t* w2_sf;
+  int T, H, I, E, k;
+  void* out;
+  int out_fp32;
+} moe_w4a8_args;
+
+size_t moe_w4a8_workspace_size(int T, int H, int I, int E, int k);
+moe_status_t moe_w4a8_forward(const moe_w4a8_args* args, void* ws, size_t ws_bytes, cudaStream_t stream);
+
+/* Diagnostic view of the W4A8 layer's quantized intermediate, like moe_blockfp8_intermediate:
+ *   inv_pos  int32 [T*k]               row r of pair p = t*k + s
+ *   h        e4m3  [T*k, I]            row r = the codes of the pair's quantized h
+ *   h_sf     uint8 [I/128, T*k, 4]     h_sf[b][r][j] = E8M0 code of row r's column group 4b + j
+ * so that h of pair p, column j, is e4m3(h[r][j]) * 2^(h_sf[j/128][r][(j/32)%4] - 127). */
+moe_status_t moe_w4a8_intermediate(const void* ws, int T, int H, int I, int E, int k, const int32_t** inv_pos,
+                                   const uint8_t** h, const uint8_t** h_sf);
 
 /* ------------------------------------------------------------------ grouped W4A16 GEMM
  * No activation: rows [expert_offsets[e], expert_offsets[e+1]) of a are multiplied by

@@ -14,11 +14,12 @@ import ctypes
 import torch
 
 from ._native import (MOE_ERR_CUDA, MOE_ERR_DEVICE_CHECK, MOE_ERR_INVALID_ARG, MOE_ERR_TIMEOUT,  # noqa: F401
-                      MOE_ERR_UNSUPPORTED, MOE_ERR_WORKSPACE, MOE_OK, BlockFP8Args, MoeError, W4A16Args, check,
+                      MOE_ERR_UNSUPPORTED, MOE_ERR_WORKSPACE, MOE_OK, BlockFP8Args, MoeError, W4A8Args, W4A16Args, check,
                       lib)
 
 __all__ = ["moe_route", "moe_blockfp8_intermediate", "moe_align", "moe_align_capacity", "moe_w4a16_forward", "moe_w4a16_workspace_size",
-           "moe_blockfp8_forward", "moe_blockfp8_workspace_size", "moe_w4a16_gemm", "moe_w4a16_gemm_workspace_size",
+           "moe_blockfp8_forward", "moe_blockfp8_workspace_size", "moe_w4a8_forward", "moe_w4a8_workspace_size",
+           "moe_w4a8_intermediate", "moe_w4a16_gemm", "moe_w4a16_gemm_workspace_size",
            "moe_get_device_status", "moe_debug_wait_timeout", "moe_timing_enable", "moe_timing_read", "MoeError",
            "lib"]
 
@@ -142,6 +143,47 @@ def moe_blockfp8_intermediate(workspace: torch.Tensor, T: int, H: int, I: int, E
     P = T * k
     return dict(inv_pos=view(ptrs[0], P, torch.int32), h=view(ptrs[1], P * I, torch.uint8).view(P, I),
                 h_scale_t=view(ptrs[2], (I // 128) * P, torch.float32).view(I // 128, P))
+
+
+def moe_w4a8_workspace_size(T: int, H: int, I: int, E: int, k: int) -> int:
+    return lib.moe_w4a8_workspace_size(T, H, I, E, k)
+
+
+def moe_w4a8_forward(x, topk_ids, topk_w, w13, w13_sf, w2, w2_sf, out=None, out_fp32: bool = False,
+                     workspace=None, stream=None) -> torch.Tensor:
+    """Routed W4A8 layer (MXFP4 weights, FP8 activations with E8M0 scales per 32 K).  x bf16
+    [T,H]; w13 uint8 [E,2I,H/2] (two E2M1 codes per byte) + E8M0 uint8 [E,H/128,2I,4]; w2 uint8
+    [E,H,I/2] + [E,I/128,H,4] -> out bf16/fp32 [T,H]."""
+    _cuda(x, topk_ids, topk_w, w13, w13_sf, w2, w2_sf, out)
+    T, H = x.shape
+    k = topk_ids.shape[1]
+    E, twoI = w13.shape[0], w13.shape[1]
+    I = twoI // 2
+    if out is None:
+        out = torch.empty(T, H, dtype=torch.float32 if out_fp32 else torch.bfloat16, device=x.device)
+    nbytes = lib.moe_w4a8_workspace_size(T, H, I, E, k)
+    ws = _workspace(nbytes, workspace, x.device)
+    args = W4A8Args(x.data_ptr(), topk_ids.data_ptr(), topk_w.data_ptr(), w13.data_ptr(), w13_sf.data_ptr(),
+                    w2.data_ptr(), w2_sf.data_ptr(), T, H, I, E, k, out.data_ptr(), int(out_fp32))
+    check(lib.moe_w4a8_forward(ctypes.byref(args), _p(ws), ws.numel() * ws.element_size(), _stream(stream)),
+          "moe_w4a8_forward")
+    return out
+
+
+def moe_w4a8_intermediate(workspace: torch.Tensor, T: int, H: int, I: int, E: int, k: int) -> dict:
+    """Views into the workspace of a finished moe_w4a8_forward(T, H, I, E, k) call:
+    inv_pos int32 [T*k], h e4m3 codes uint8 [T*k, I], h_sf E8M0 codes uint8 [I/128, T*k, 4]."""
+    _cuda(workspace)
+    ptrs = [ctypes.c_void_p() for _ in range(3)]
+    check(lib.moe_w4a8_intermediate(_p(workspace), T, H, I, E, k, *[ctypes.byref(q) for q in ptrs]),
+          "moe_w4a8_intermediate")
+    raw = workspace.view(torch.uint8).reshape(-1)
+    base = raw.data_ptr()
+    P = T * k
+    inv = raw[ptrs[0].value - base: ptrs[0].value - base + 4 * P].view(torch.int32)
+    h = raw[ptrs[1].value - base: ptrs[1].value - base + P * I].view(P, I)
+    h_sf = raw[ptrs[2].value - base: ptrs[2].value - base + (I // 128) * P * 4].view(I // 128, P, 4)
+    return dict(inv_pos=inv, h=h, h_sf=h_sf)
 
 
 def moe_w4a16_gemm_workspace_size(M: int, K: int, N: int, E: int) -> int:

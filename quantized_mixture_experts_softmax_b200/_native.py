@@ -22,6 +22,7 @@ EXPORTS = [
     "moe_w4a16_workspace_size", "moe_w4a16_forward", "moe_blockfp8_workspace_size", "moe_blockfp8_forward",
     "moe_w4a16_gemm_workspace_size", "moe_w4a16_gemm", "moe_get_device_status", "moe_debug_wait_timeout",
     "moe_timing_enable", "moe_timing_read", "moe_align_noalloc", "moe_blockfp8_intermediate",
+    "moe_w4a8_workspace_size", "moe_w4a8_forward", "moe_w4a8_intermediate",
 ]
 
 
@@ -44,6 +45,13 @@ class BlockFP8Args(ctypes.Structure):
                 ("w2", ctypes.c_void_p), ("w2_s", ctypes.c_void_p), ("T", ctypes.c_int), ("H", ctypes.c_int),
                 ("I", ctypes.c_int), ("E", ctypes.c_int), ("k", ctypes.c_int), ("out", ctypes.c_void_p),
                 ("out_fp32", ctypes.c_int)]
+
+
+class W4A8Args(ctypes.Structure):
+    _fields_ = [("x", ctypes.c_void_p), ("topk_ids", ctypes.c_void_p), ("topk_w", ctypes.c_void_p),
+                ("w13", ctypes.c_void_p), ("w13_sf", ctypes.c_void_p), ("w2", ctypes.c_void_p),
+                ("w2_sf", ctypes.c_void_p), ("T", ctypes.c_int), ("H", ctypes.c_int), ("I", ctypes.c_int),
+                ("E", ctypes.c_int), ("k", ctypes.c_int), ("out", ctypes.c_void_p), ("out_fp32", ctypes.c_int)]
 
 
 def _load():
@@ -72,6 +80,13 @@ def _load():
     L.moe_blockfp8_workspace_size.argtypes = [i32, i32, i32, i32, i32]
     L.moe_blockfp8_forward.restype = i32
     L.moe_blockfp8_forward.argtypes = [ctypes.POINTER(BlockFP8Args), vp, sz, vp]
+    L.moe_w4a8_workspace_size.restype = sz
+    L.moe_w4a8_workspace_size.argtypes = [i32, i32, i32, i32, i32]
+    L.moe_w4a8_forward.restype = i32
+    L.moe_w4a8_forward.argtypes = [ctypes.POINTER(W4A8Args), vp, sz, vp]
+    L.moe_w4a8_intermediate.restype = i32
+    L.moe_w4a8_intermediate.argtypes = [vp, i32, i32, i32, i32, i32, ctypes.POINTER(vp), ctypes.POINTER(vp),
+                                        ctypes.POINTER(vp)]
     L.moe_blockfp8_intermediate.restype = i32
     L.moe_blockfp8_intermediate.argtypes = [vp, i32, i32, i32, i32, i32, ctypes.POINTER(vp), ctypes.POINTER(vp),
                                             ctypes.POINTER(vp)]

@@ -275,6 +275,32 @@ F8Ws carve_fp8_forward(void* ws, int T, int H, int I, int E, int k) {
   w.bytes = c.off + 256;
   return w;
 }
+struct MxWs {
+  int32_t *counts, *offsets, *sorted, *inv, *blockcnt, *tile_prefix, *chunk;
+  uint8_t *x_perm, *h;
+  uint32_t *x_sf, *h_sf;
+  float* y;
+  size_t bytes;
+};
+MxWs carve_w4a8_forward(void* ws, int T, int H, int I, int E, int k) {
+  Carver c(ws);
+  MxWs w;
+  const size_t P = (size_t)T * k;
+  w.counts = c.take<int32_t>(E);
+  w.offsets = c.take<int32_t>(E + 1);
+  w.sorted = c.take<int32_t>(P);
+  w.inv = c.take<int32_t>(P);
+  w.blockcnt = c.take<int32_t>((size_t)align_blocks(T, k) * E);
+  w.tile_prefix = c.take<int32_t>(E + 1);
+  w.chunk = c.take<int32_t>(E);
+  w.x_perm = c.take<uint8_t>(P * H);
+  w.x_sf = c.take<uint32_t>((size_t)(H / 128) * P);
+  w.h = c.take<uint8_t>(P * I);
+  w.h_sf = c.take<uint32_t>((size_t)(I / 128) * P);
+  w.y = c.take<float>(P * H);
+  w.bytes = c.off + 256;
+  return w;
+}
 // token-tile height cap of the single grouped GEMM's kernel
 int pick_nmax(int max_rows_per_expert) { return use_i8(max_rows_per_expert) ? kI8TileRows : kWideTileRows; }
 
@@ -464,6 +490,56 @@ moe_status_t moe_blockfp8_forward(const moe_blockfp8_args* a, void* ws, size_t w
   }
   if (e == cudaSuccess) e = launch_combine(w.y, w.inv, a->topk_w, T, k, H, a->out, a->out_fp32, stream);
   return e == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
+}
+
+size_t moe_w4a8_workspace_size(int T, int H, int I, int E, int k) {
+  if (!shape_ok(T, H, I, E, k)) return 0;
+  return carve_w4a8_forward(nullptr, T, H, I, E, k).bytes;
+}
+
+moe_status_t moe_w4a8_forward(const moe_w4a8_args* a, void* ws, size_t ws_bytes, cudaStream_t stream) {
+  if (!a) return MOE_ERR_INVALID_ARG;
+  if (!shape_ok(a->T, a->H, a->I, a->E, a->k)) return MOE_ERR_UNSUPPORTED;
+  if (!aligned(a->x, 16) || !aligned(a->topk_ids, 4) || !aligned(a->topk_w, 4) || !aligned(a->w13, 32) ||
+      !aligned(a->w13_sf, 16) || !aligned(a->w2, 32) || !aligned(a->w2_sf, 16) || !aligned(a->out, 16) ||
+      !aligned(ws, 256))
+    return MOE_ERR_INVALID_ARG;
+  const int T = a->T, H = a->H, I = a->I, E = a->E, k = a->k;
+  if (ws_bytes < moe_w4a8_workspace_size(T, H, I, E, k)) return MOE_ERR_WORKSPACE;
+  if (moe_status_t st = check_device()) return st;
+  const MxWs w = carve_w4a8_forward(ws, T, H, I, E, k);
+  const int P = T * k;
+  const int nmax = T > 512 ? 64 : 32;
+  SchedOut so;
+  so.nmax = nmax;
+  so.tile_prefix = w.tile_prefix;
+  so.chunk = w.chunk;
+  cudaError_t e = launch_align(a->topk_ids, T, k, E, 1, w.counts, w.offsets, w.sorted, w.inv, w.blockcnt, &so, stream);
+  if (e == cudaSuccess)
+    e = launch_permute_mx(reinterpret_cast<const uint16_t*>(a->x), w.inv, T, k, H, w.x_perm, w.x_sf, P, stream);
+  const TileSched sched{w.offsets, w.counts, w.tile_prefix, w.chunk};
+  if (e == cudaSuccess) {
+    MxGemmProblem g{a->w13, a->w13_sf, w.x_perm, w.x_sf, P, H, E, 2 * I, true, I, sched,
+                    w.h, I, reinterpret_cast<uint8_t*>(w.h_sf), nmax};
+    e = launch_mx_gemm(g, stream);
+  }
+  if (e == cudaSuccess) {
+    MxGemmProblem g{a->w2, a->w2_sf, w.h, w.h_sf, P, I, E, H, false, 0, sched, w.y, H, nullptr, nmax};
+    e = launch_mx_gemm(g, stream);
+  }
+  if (e == cudaSuccess) e = launch_combine(w.y, w.inv, a->topk_w, T, k, H, a->out, a->out_fp32, stream);
+  return e == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
+}
+
+moe_status_t moe_w4a8_intermediate(const void* ws, int T, int H, int I, int E, int k, const int32_t** inv_pos,
+                                   const uint8_t** h, const uint8_t** h_sf) {
+  if (!shape_ok(T, H, I, E, k)) return MOE_ERR_UNSUPPORTED;
+  if (!aligned(ws, 256) || !inv_pos || !h || !h_sf) return MOE_ERR_INVALID_ARG;
+  const MxWs w = carve_w4a8_forward(const_cast<void*>(ws), T, H, I, E, k);
+  *inv_pos = w.inv;
+  *h = w.h;
+  *h_sf = reinterpret_cast<const uint8_t*>(w.h_sf);
+  return MOE_OK;
 }
 
 moe_status_t moe_blockfp8_intermediate(const void* ws, int T, int H, int I, int E, int k, const int32_t** inv_pos,

@@ -200,6 +200,26 @@ cudaError_t launch_fp8_gemm(const F8GemmProblem& p, cudaStream_t s);
 cudaError_t launch_permute_fp8(const uint8_t* x, const float* xs, const int32_t* inv_pos, int T, int k, int H,
                                uint8_t* x_perm, float* xs_t, int P, cudaStream_t s);
 
+// W4A8 grouped GEMM (gemm_mx.cu): MXFP4 weights x e4m3 activations with E8M0 scales per 32 K
+struct MxGemmProblem {
+  const uint8_t* w;        // E2M1 codes [E, rows_per_expert, K/2] (even K in the low nibble), 32-byte aligned
+  const uint8_t* w_sf;     // E8M0 [E, K/128, rows_per_expert, 4]
+  const uint8_t* act;      // e4m3 [act_rows, K]
+  const uint32_t* x_sf;    // [K/128, act_rows]: byte j = E8M0 code of the row's K group 4*blk + j
+  int act_rows;
+  int K, E, rows_per_expert;
+  bool gated;              // gate rows [0, I), up rows [I, 2I); output e4m3 h [*, I] + h_sf
+  int I;
+  TileSched sched;
+  void* out;
+  int out_ld;
+  uint8_t* h_sf;           // gated: [I/128, act_rows, 4] (the x_sf layout of the down GEMM's input)
+  int nmax;                // token rows per tile: 32 or 64 (the cap the schedule was built with)
+};
+cudaError_t launch_mx_gemm(const MxGemmProblem& p, cudaStream_t s);
+cudaError_t launch_permute_mx(const uint16_t* x, const int32_t* inv_pos, int T, int k, int H, uint8_t* x_perm,
+                              uint32_t* x_sf, int P, cudaStream_t s);
+
 // driver entry point for tensor maps (api.cu)
 // 2-D tiled tensor map over a row-major [rows, cols] tensor at `base` (zero fill out of bounds).
 CUresult encode_tmap_2d(CUtensorMap* map, const void* base, CUtensorMapDataType dt, uint64_t cols, uint64_t rows,

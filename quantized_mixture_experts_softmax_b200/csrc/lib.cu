@@ -5,5 +5,6 @@
 #include "gemm_w4a16.cu"
 #include "gemm_fp8.cu"
 #include "gemm_w4i8.cu"
+#include "gemm_mx.cu"
 #include "api.cu"
 #include "align_noalloc.cu"

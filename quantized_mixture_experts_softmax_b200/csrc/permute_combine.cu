@@ -6,6 +6,8 @@
 // That is the order in which one packed INT4 word dequantizes with two-nibbles-per-lane
 // bit tricks, so the GEMM never has to shuffle weights; applying the same permutation to
 // both operands of a dot product leaves it unchanged.
+#include <cuda_fp8.h>
+
 #include "common.cuh"
 #include "internal.h"
 
@@ -199,6 +201,55 @@ cudaError_t launch_permute_fp8(const uint8_t* x, const float* xs, const int32_t*
   (void)launch_kernel(permute_fp8_kernel, dim3(ceil_div(Pn, 8)), dim3(256), 0, s, reinterpret_cast<const uint4*>(x), xs, inv_pos, Pn, k, H,
                                                     reinterpret_cast<uint4*>(x_perm), xs_t, P);
   timing_after("permute_fp8", s);
+  return cudaGetLastError();
+}
+
+// W4A8 input rows: bf16 x -> e4m3 codes with one E8M0 scale per 32 along K (the smallest power
+// of two 2^X with amax <= 448 * 2^X; codes e4m3(x * 2^-X), nearest-even, exact scaling), written
+// to each of the token's k expert-sorted rows.  One warp per (token, 128-K block), four elements
+// per lane, a 32-group = 8 lanes; the block's four scale codes leave as one 32-bit word.
+__global__ void __launch_bounds__(256) permute_mx_kernel(const uint2* __restrict__ x,
+                                                         const int32_t* __restrict__ inv_pos, int T, int k, int H,
+                                                         uint32_t* __restrict__ x_perm, uint32_t* __restrict__ x_sf,
+                                                         int P) {
+  grid_dependency_sync();  // see common.cuh
+  const int gw = (int)((blockIdx.x * blockDim.x + threadIdx.x) >> 5);
+  const int lane = threadIdx.x & 31;
+  const int nb = H / 128;
+  if (gw >= T * nb) return;
+  const int t = gw / nb, b = gw - t * nb;
+  const uint2 v = __ldg(x + ((size_t)t * H + b * 128) / 4 + lane);
+  const float f0 = __uint_as_float(v.x << 16), f1 = __uint_as_float(v.x & 0xFFFF0000u);
+  const float f2 = __uint_as_float(v.y << 16), f3 = __uint_as_float(v.y & 0xFFFF0000u);
+  float a = fmaxf(fmaxf(fabsf(f0), fabsf(f1)), fmaxf(fabsf(f2), fabsf(f3)));
+  a = fmaxf(a, __shfl_xor_sync(0xffffffffu, a, 1));
+  a = fmaxf(a, __shfl_xor_sync(0xffffffffu, a, 2));
+  a = fmaxf(a, __shfl_xor_sync(0xffffffffu, a, 4));
+  if (!(a <= 3.402823466e38f) && (lane & 7) == 0) set_status(MOE_ERR_DEVICE_CHECK);  // an inf or NaN input
+  const int X = mx_exponent(__float_as_uint(a));
+  const float inv = exp2_neg(X);
+  const uint32_t lo = __nv_cvt_float2_to_fp8x2(make_float2(f0 * inv, f1 * inv), __NV_SATFINITE, __NV_E4M3);
+  const uint32_t hi = __nv_cvt_float2_to_fp8x2(make_float2(f2 * inv, f3 * inv), __NV_SATFINITE, __NV_E4M3);
+  const uint32_t codes = lo | (hi << 16);
+  const uint32_t sb = (uint32_t)(X + 127);
+  const uint32_t word = __shfl_sync(0xffffffffu, sb, 0) | (__shfl_sync(0xffffffffu, sb, 8) << 8) |
+                        (__shfl_sync(0xffffffffu, sb, 16) << 16) | (__shfl_sync(0xffffffffu, sb, 24) << 24);
+  for (int s = 0; s < k; ++s) {
+    const int r = __ldg(inv_pos + (size_t)t * k + s);
+    if (r < 0) continue;  // the same for the whole warp
+    x_perm[((size_t)r * H + b * 128) / 4 + lane] = codes;
+    if (lane == 0) x_sf[(size_t)b * P + r] = word;
+  }
+}
+
+cudaError_t launch_permute_mx(const uint16_t* x, const int32_t* inv_pos, int T, int k, int H, uint8_t* x_perm,
+                              uint32_t* x_sf, int P, cudaStream_t s) {
+  const int warps = T * (H / 128);
+  timing_before("permute_mx", s);
+  (void)launch_kernel(permute_mx_kernel, dim3(ceil_div(warps, 8)), dim3(256), 0, s,
+                      reinterpret_cast<const uint2*>(x), inv_pos, T, k, H, reinterpret_cast<uint32_t*>(x_perm), x_sf,
+                      P);
+  timing_after("permute_mx", s);
   return cudaGetLastError();
 }
 

@@ -85,7 +85,8 @@ def test_binding_structs_match_the_header(native, tmp_path):
     if gcc is None:
         pytest.skip("no C compiler")
     fields = {"moe_w4a16_args": [f for f, _ in native.W4A16Args._fields_],
-              "moe_blockfp8_args": [f for f, _ in native.BlockFP8Args._fields_]}
+              "moe_blockfp8_args": [f for f, _ in native.BlockFP8Args._fields_],
+              "moe_w4a8_args": [f for f, _ in native.W4A8Args._fields_]}
     lines = ["#include <stdio.h>", "#include <stddef.h>", '#include "moe.h"', "int main(void) {"]
     for st, names in fields.items():
         lines.append(f'  printf("{st} size %zu\\n", sizeof({st}));')
@@ -101,7 +102,8 @@ def test_binding_structs_match_the_header(native, tmp_path):
     for line in subprocess.check_output([str(exe)]).decode().splitlines():
         st, n, v = line.split()
         got[(st, n)] = int(v)
-    for st, cls in (("moe_w4a16_args", native.W4A16Args), ("moe_blockfp8_args", native.BlockFP8Args)):
+    for st, cls in (("moe_w4a16_args", native.W4A16Args), ("moe_blockfp8_args", native.BlockFP8Args),
+                    ("moe_w4a8_args", native.W4A8Args)):
         assert got[(st, "size")] == ctypes.sizeof(cls), st
         for n in fields[st]:
             assert got[(st, n)] == getattr(cls, n).offset, (st, n)
@@ -123,6 +125,14 @@ def _f8(native, **kw):
     return native.BlockFP8Args(*[d[f] for f, _ in native.BlockFP8Args._fields_])
 
 
+def _mx(native, **kw):
+    fake = 1 << 20
+    d = dict(x=fake, topk_ids=fake, topk_w=fake, w13=fake, w13_sf=fake, w2=fake, w2_sf=fake,
+             T=64, H=7168, I=2048, E=384, k=8, out=fake, out_fp32=0)
+    d.update(kw)
+    return native.W4A8Args(*[d[f] for f, _ in native.W4A8Args._fields_])
+
+
 # shapes outside the documented limits: T >= 1, 1 <= k <= E <= 1024, H and I multiples of 128
 BAD_SHAPES = [dict(T=0), dict(k=0), dict(E=0), dict(E=1025, k=8), dict(k=9, E=8), dict(H=7100), dict(I=2000),
               dict(H=0), dict(I=64)]
@@ -141,6 +151,9 @@ def test_forward_shape_limits(native, kw):
     f = _f8(native, **kw)
     assert L.moe_blockfp8_forward(ctypes.byref(f), fake, 1 << 40, None) == native.MOE_ERR_UNSUPPORTED
     assert L.moe_blockfp8_workspace_size(f.T, f.H, f.I, f.E, f.k) == 0
+    m = _mx(native, **kw)
+    assert L.moe_w4a8_forward(ctypes.byref(m), fake, 1 << 40, None) == native.MOE_ERR_UNSUPPORTED
+    assert L.moe_w4a8_workspace_size(m.T, m.H, m.I, m.E, m.k) == 0
 
 
 @pytest.mark.parametrize("field", BAD_PTRS_W4)
@@ -166,6 +179,23 @@ def test_blockfp8_forward_rejects_misaligned_or_null(native, field):
         assert L.moe_blockfp8_forward(ctypes.byref(f), fake, 1 << 40, None) == native.MOE_ERR_INVALID_ARG, (field, bad)
     f = _f8(native, xs=(1 << 20) + 2)
     assert L.moe_blockfp8_forward(ctypes.byref(f), fake, 1 << 40, None) == native.MOE_ERR_INVALID_ARG
+
+
+@pytest.mark.parametrize("field,bad", [("x", 8), ("w13", 16), ("w13_sf", 8), ("w2", 16), ("w2_sf", 8), ("out", 8),
+                                       ("topk_ids", 2), ("topk_w", 2), ("x", None), ("w13", None)])
+def test_w4a8_forward_rejects_misaligned_or_null(native, field, bad):
+    """The packed weights need 32-byte alignment (the TMA's 4-bit unpacking mode), the rest 16
+    (vector reads) or 4 (scalars)."""
+    L = native.lib
+    fake = ctypes.c_void_p(1 << 20)
+    m = _mx(native, **{field: 0 if bad is None else (1 << 20) + bad})
+    assert L.moe_w4a8_forward(ctypes.byref(m), fake, 1 << 40, None) == native.MOE_ERR_INVALID_ARG
+    m = _mx(native)
+    need = L.moe_w4a8_workspace_size(m.T, m.H, m.I, m.E, m.k)
+    assert need > 0
+    assert L.moe_w4a8_forward(ctypes.byref(m), fake, need - 1, None) == native.MOE_ERR_WORKSPACE
+    assert L.moe_w4a8_forward(ctypes.byref(m), ctypes.c_void_p((1 << 20) + 16), 1 << 40, None) == \
+        native.MOE_ERR_INVALID_ARG
 
 
 def test_forward_workspace_one_byte_short(native):
