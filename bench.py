@@ -7,6 +7,8 @@ One JSON line on stdout (rank 0).  Workloads (seeded synthetic inputs):
   decode            T=64 tokens, hidden 7168, intermediate 2048, 384 experts, top-8, N(0,1) logits
   prefill           T=8192 tokens, same model, logits skewed by a Zipf(1.1) per-expert bias
   fp8_t{1,16,64,512,4096}   the block-FP8 layer, 256 experts, top-8
+  w4a8_t64, w4a8_t8192      the W4A8 layer (MXFP4 weights, FP8 activations in 32-groups) on the
+                            decode / prefill shapes and routing of the W4A16 model
   gemm_m{M}_k{K}_n{N}       the single-expert grouped GEMM sweep (no activation)
 The layer models' experts (9.5 GB of INT4 weights + bf16 scales for W4A16) stay resident in HBM;
 each step streams the active experts' weights (about 7 GB for decode), far more than the
@@ -42,6 +44,9 @@ WORKLOADS = {
 for _t in (1, 16, 64, 512, 4096):  # block-FP8 layer, 256 experts
     WORKLOADS[f"fp8_t{_t}"] = dict(kind="fp8", T=_t, zipf=0.0, steps=200 if _t <= 512 else 60, warmup=10)
 FP8_MODEL = dict(H=7168, I=2048, E=256, k=8)
+# W4A8 layer: the W4A16 model's shapes and routing (384 experts, top-8), MXFP4 weights
+WORKLOADS["w4a8_t64"] = dict(kind="w4a8", T=64, zipf=0.0, steps=400, warmup=20)
+WORKLOADS["w4a8_t8192"] = dict(kind="w4a8", T=8192, zipf=1.1, steps=40, warmup=5)
 # block-FP8 benchmark model: expert e holds the generated weights of expert e mod FP8_DISTINCT (each
 # expert in its own memory); generating 11.3 GB of normal e4m3 values on the host takes minutes
 FP8_DISTINCT = 16
@@ -54,6 +59,8 @@ for (_k, _n) in ((7168, 512), (256, 7168)):
 GEMM_METRIC = "grouped W4A16 GEMM µs (one expert, no activation) and % roofline"
 W13_BYTES_PER_EXPERT = 2 * 2048 * 7168 // 2 + 2 * 2048 * (7168 // 32) * 2   # INT4 words + bf16 scales
 W2_BYTES_PER_EXPERT = 7168 * 2048 // 2 + 7168 * (2048 // 32) * 2
+W13_MX_BYTES_PER_EXPERT = 2 * 2048 * 7168 // 2 + 2 * 2048 * (7168 // 32)  # E2M1 codes + E8M0 scales
+W2_MX_BYTES_PER_EXPERT = 7168 * 2048 // 2 + 7168 * (2048 // 32)
 
 
 # Datasheet figures of a B200 (HGX): HBM3e 8 TB/s; dense tensor 2.25 PFLOP/s bf16/fp16, 4.5 fp8.
@@ -79,7 +86,7 @@ def load_peaks():
 
 
 # source file of each grouped GEMM: a measured traffic figure stands only while it is unchanged
-KERNEL_SOURCES = {"w4i8": "gemm_w4i8.cu", "w4a16": "gemm_w4a16.cu", "fp8": "gemm_fp8.cu"}
+KERNEL_SOURCES = {"w4i8": "gemm_w4i8.cu", "w4a16": "gemm_w4a16.cu", "fp8": "gemm_fp8.cu", "mx": "gemm_mx.cu"}
 
 
 def source_sha256(family: str) -> str:
@@ -250,6 +257,30 @@ def make_model_fp8(seed: int, distinct: int = 0):
     return out
 
 
+def make_model_mx(seed: int):
+    """All 384 MXFP4 experts (E2M1 codes and E8M0 scale codes), generated on the host by the
+    seeded generator and copied to HBM."""
+    import torch
+    import synth
+    H, I, E = MODEL["H"], MODEL["I"], MODEL["E"]
+    out = {}
+    chunk = 32
+    for name, shape, tid in (("w13", (E, 2 * I, H // 2), "w13_mx"), ("w13_sf", (E, H // 128, 2 * I, 4), "w13_mxs"),
+                             ("w2", (E, H, I // 2), "w2_mx"), ("w2_sf", (E, I // 128, H, 4), "w2_mxs")):
+        d = torch.empty(shape, dtype=torch.uint8, device="cuda")
+        per = int(np.prod(shape[1:]))
+        for e0 in range(0, E, chunk):
+            n = min(chunk, E - e0)
+            buf = np.empty((n, *shape[1:]), np.uint8)
+            if name.endswith("_sf"):
+                synth._mx_scales(seed, synth.TID[tid], e0 * per, buf)
+            else:
+                synth.fill_u32(seed, synth.TID[tid], e0 * per // 4, buf.view(np.uint32))
+            d[e0:e0 + n].copy_(torch.from_numpy(buf))
+        out[name] = d
+    return out
+
+
 def make_inputs(seed: int, T: int, zipf: float, kind: str = "w4a16"):
     import synth
     if kind == "fp8":
@@ -262,7 +293,8 @@ def make_inputs(seed: int, T: int, zipf: float, kind: str = "w4a16"):
 
 def layer_config(workload: str, kind: str, T: int, H: int, I: int, E: int, k: int, active: int, world: int) -> dict:
     """The `config` object of a layer workload's JSON line (the same for both arms)."""
-    return {"workload": f"{workload} {'block-FP8' if kind == 'fp8' else 'W4A16'} MoE layer T={T} H={H} I={I} E={E} "
+    label = {"fp8": "block-FP8", "w4a8": "W4A8 (MXFP4 x FP8)"}.get(kind, "W4A16")
+    return {"workload": f"{workload} {label} MoE layer T={T} H={H} I={I} E={E} "
                         f"top-{k}",
             "T": T, "H": H, "I": I, "E": E, "k": k, "active_experts": active,
             "parallelism": "replicas" if world > 1 else "single GPU",
@@ -400,6 +432,13 @@ def measure_layer(args, workload, W, world):
         def forward(xx, xxs):
             moe.moe_blockfp8_forward(xx, xxs, ids, tw, W["w13"], W["w13_s"], W["w2"], W["w2_s"], out=out,
                                      workspace=ws)
+    elif kind == "w4a8":
+        x = torch.from_numpy(x_h).cuda().view(torch.bfloat16)
+        xs = None
+        ws = torch.empty(moe.moe_w4a8_workspace_size(T, H, I, E, k), dtype=torch.uint8, device="cuda")
+
+        def forward(xx, xxs):
+            moe.moe_w4a8_forward(xx, ids, tw, W["w13"], W["w13_sf"], W["w2"], W["w2_sf"], out=out, workspace=ws)
     else:
         x = torch.from_numpy(x_h).cuda().view(torch.bfloat16)
         xs = None
@@ -527,16 +566,21 @@ def measure_layer(args, workload, W, world):
         w13_b = 2 * I * H + (2 * I // 128) * (H // 128) * 4
         w2_b = H * I + (H // 128) * (I // 128) * 4
         x_in = T * H + T * (H // 128) * 4
+    elif kind == "w4a8":
+        w13_b, w2_b = W13_MX_BYTES_PER_EXPERT, W2_MX_BYTES_PER_EXPERT
+        x_in = T * H * 2
     else:
         w13_b, w2_b = W13_BYTES_PER_EXPERT, W2_BYTES_PER_EXPERT
         x_in = T * H * 2
     out_b = T * H * 2
     layer_bytes = active * (w13_b + w2_b) + x_in + out_b + T * E * 4
     # tensor peak for the contraction's own operand type: fp16 and int8 run at the measured bf16
-    # rate, e4m3 at twice it (the nominal dense fp8 : bf16 ratio)
-    t_peak = peaks["bf16"] * (2.0 if kind == "fp8" else 1.0)
-    t_peak_src = peaks["src"] + (" bf16 GEMM x 2 (nominal fp8:bf16)" if kind == "fp8" else " bf16 GEMM, burst")
-    family = "fp8" if kind == "fp8" else ("w4i8" if T <= 64 else "w4a16")
+    # rate, e4m3 (and the e2m1 x e4m3 block-scaled kind) at twice it (the nominal dense fp8 : bf16
+    # ratio)
+    f8 = kind in ("fp8", "w4a8")
+    t_peak = peaks["bf16"] * (2.0 if f8 else 1.0)
+    t_peak_src = peaks["src"] + (" bf16 GEMM x 2 (nominal fp8:bf16)" if f8 else " bf16 GEMM, burst")
+    family = {"fp8": "fp8", "w4a8": "mx"}.get(kind, "w4i8" if T <= 64 else "w4a16")
     no_traffic = bool(args.tokens or args.experts)
     phases = {}
     for suffix, alg_b, alg_f in (("gate_up", active * w13_b + x_in, 2.0 * P * H * 2 * I),
@@ -546,7 +590,7 @@ def measure_layer(args, workload, W, world):
         if len(names) == 1 and not no_traffic:
             traffic = load_traffic(workload, names[0], family)
         phases[suffix] = _phase_roofline(kern, suffix, alg_b, alg_f, t_peak, t_peak_src, peaks, traffic,
-                                         SPEC["fp8" if kind == "fp8" else "bf16"])
+                                         SPEC["fp8" if f8 else "bf16"])
     dom = max((v for v in phases.values() if v), key=lambda r: r["launch_ms"], default=None)
     launches = sum(n for (_, n) in kern.values())
     res = {
@@ -554,6 +598,8 @@ def measure_layer(args, workload, W, world):
         "n_gpus": world, "steps": steps, "warmup": warmup, "ms_per_step": round(ms_step, 4),
         "higher_is_better": False, "scaling": "weak", "vs_baseline": None,
         "dtype": {"fp8": "e4m3 (fp32 acc)",
+                  "mx": "w4a8: MXFP4 weights x e4m3 activations, E8M0 scales per 32 K applied by the "
+                        "block-scaled MMA (fp32 acc)",
                   "w4a16": "w4a16: fp16 MMA (fp32 acc) for experts with many rows, int8 MMA on 16-bit "
                            "fixed-point activations + fp32 promotion for the rest",
                   "w4i8": "w4a16 as int8 MMA (u8 weights x 16-bit fixed-point activations, s32) + fp32 promotion"}[family],
@@ -564,7 +610,7 @@ def measure_layer(args, workload, W, world):
                   "hbm_frac": round(layer_bytes / (ms_step * 1e-3) / 1e9 / peaks["hbm"], 4),
                   "tensor_frac": round(flops / (ms_step * 1e-3) / 1e12 / t_peak, 4),
                   "hbm_frac_spec": round(layer_bytes / (ms_step * 1e-3) / 1e9 / SPEC["hbm"], 4),
-                  "tensor_frac_spec": round(flops / (ms_step * 1e-3) / 1e12 / SPEC["fp8" if kind == "fp8" else "bf16"],
+                  "tensor_frac_spec": round(flops / (ms_step * 1e-3) / 1e12 / SPEC["fp8" if f8 else "bf16"],
                                             4),
                   "algorithmic_bytes": int(layer_bytes), "flops": flops},
         "kernels_ms_per_step": {n: round(v[0] / steps, 4) for n, v in sorted(kern.items(), key=lambda kv: -kv[1][0])},
@@ -581,21 +627,22 @@ def measure_layer(args, workload, W, world):
 
 def run_ours(args, world, rank):
     wl = WORKLOADS[args.workload]
-    W = make_model_fp8(0, distinct=FP8_DISTINCT) if wl["kind"] == "fp8" else make_model(0)
+    W = {"fp8": lambda: make_model_fp8(0, distinct=FP8_DISTINCT), "w4a8": lambda: make_model_mx(0)}.get(
+        wl["kind"], lambda: make_model(0))()
     return measure_layer(args, args.workload, W, world)
 
 
 # the objects the default run adds to the decode line, measured in the same process
-DEFAULT_EXTRAS = ("prefill", "fp8_t64", "fp8_t4096")
+DEFAULT_EXTRAS = ("prefill", "fp8_t64", "fp8_t4096", "w4a8_t64", "w4a8_t8192")
 # keys of a workload's result that stay on the top-level line only
 LINE_ONLY = ("metric", "n_gpus", "higher_is_better", "scaling", "vs_baseline", "data")
 
 
 def run_default(args, world, rank):
     """The default benchmark: the decode T=64 line (its `value` is the headline), with the
-    prefill T=8192 workload on the same resident 384-expert model and the block-FP8 layer at
-    T=64 and T=4096 as nested objects, each measured like the line itself, with its own
-    CPU-oracle baseline on rank 0."""
+    prefill T=8192 workload on the same resident 384-expert model, the block-FP8 layer at T=64
+    and T=4096, and the W4A8 layer at T=64 and T=8192 as nested objects, each measured like the
+    line itself, with its own CPU-oracle baseline on rank 0."""
     import torch
     W = make_model(0)
     res, inp = measure_layer(args, "decode", W, world)
@@ -612,6 +659,14 @@ def run_default(args, world, rank):
             res[wl] = {k_: v for k_, v in sub.items() if k_ not in LINE_ONLY}
             results.append((res[wl], inp_f))
         del W8
+        torch.cuda.empty_cache()
+    if not args.no_w4a8:
+        WM = make_model_mx(0)
+        for wl in ("w4a8_t64", "w4a8_t8192"):
+            sub, inp_m = measure_layer(args, wl, WM, world)
+            res[wl] = {k_: v for k_, v in sub.items() if k_ not in LINE_ONLY}
+            results.append((res[wl], inp_m))
+        del WM
         torch.cuda.empty_cache()
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         for obj, (x_h, lg_h, T, kind) in results:
@@ -642,6 +697,10 @@ def oracle_sample_time(x_h, lg_h, T, kind="w4a16", budget_s=15.0):
             ids_l = (ids[tok] % FP8_DISTINCT).astype(np.int32)
             t0 = time.time()
             oracle.fp8_tokens(x_h[0][tok], x_h[1][tok], ids_l, w[tok], Wt["w13"], Wt["w13_s"], Wt["w2"], Wt["w2_s"])
+        elif kind == "w4a8":
+            Wt = synth.mxfp4_weights(0, M["H"], M["I"], used)
+            t0 = time.time()
+            oracle.w4a8_tokens(x_h[tok], ids_l, w[tok], Wt["w13"], Wt["w13_sf"], Wt["w2"], Wt["w2_sf"])
         else:
             Wt = synth.w4a16_weights(0, M["H"], M["I"], used)
             t0 = time.time()
@@ -731,6 +790,7 @@ def main():
     ap.add_argument("--workload", choices=sorted(WORKLOADS), default=None,
                     help="one workload's line (default: decode, with prefill and block-FP8 objects)")
     ap.add_argument("--no-fp8", action="store_true", help="default run: leave out the block-FP8 objects")
+    ap.add_argument("--no-w4a8", action="store_true", help="default run: leave out the W4A8 objects")
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--experts", type=int, default=None,

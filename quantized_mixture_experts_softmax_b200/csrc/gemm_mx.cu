@@ -26,7 +26,11 @@
 //   warp 0      TMA producer: NA weight tiles (gate and up, or two adjacent down tiles), the
 //               token tile and the weight scales, one stage per 128 K;
 //   warp 1      TMEM allocator and MMA issuer: four K = 32 block-scaled MMAs per matrix and
-//               stage into one of two accumulator tiles;
+//               stage into one of two accumulator tiles; it never waits on an mbarrier (a
+//               thread with MMAs in flight would stall there until they drain) and is released
+//               stage by stage by
+//   warp 2      the MMA scheduler, which waits for the stage's copies and scales (and, at an
+//               item's first stage, for a free accumulator tile);
 //   warps 4-7   scale warps, one per lane quarter: per stage, the weight scales from shared
 //               memory and the token scales from global memory into the stage's TMEM block;
 //   warps 8-11  epilogue, one per lane quarter, a thread per weight row: the gate/up GEMM ends
@@ -44,6 +48,8 @@ namespace mx {
 constexpr int BM = 128;  // weight rows per tile (MMA M)
 constexpr int KB = 128;  // K per stage
 constexpr int kMmaWarp = 1;
+constexpr int kSchedWarp = 2;
+constexpr int kMmaBarrier = 1;  // named barrier of the MMA and scheduler warps (0 is __syncthreads)
 constexpr int kScaleWarp0 = 4;
 constexpr int kEpiWarp0 = 8;
 constexpr int kThreads = 12 * 32;
@@ -206,17 +212,14 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   } else if (warp == kMmaWarp) {
     // ---------------------------------------------------------------- MMA issuer
+    // Released stage by stage by the scheduler warp; identical loop bounds on both sides.
     int s = 0, pb = 0;
-    uint32_t ph = 0, ph_d = 0;
     bool ok = true;
     for (int it = blockIdx.x; it < total && ok; it += gridDim.x) {
       const Item I = decode_item(it, sprefix, p);
-      if (!(ok = __all_sync(0xffffffffu, mbar_wait(&d_empty[pb], ph_d ^ 1u, abort_flag, lim)))) break;
       const uint32_t d = tmem_base + (uint32_t)(pb * C::P_COLS);
       for (int kb = 0; kb < nkb; ++kb) {
-        ok = __all_sync(0xffffffffu, mbar_wait(&full[s], ph, abort_flag, lim)) &&
-             __all_sync(0xffffffffu, mbar_wait(&sf_full[s], ph, abort_flag, lim));
-        if (!ok) break;
+        if (!(ok = bar_red_and(kMmaBarrier, 64, true))) break;
         if (lane == 0) {
           tc_fence_after();
           const uint8_t* st = smem + s * C::STAGE;
@@ -237,6 +240,25 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (kb == nkb - 1) umma_commit(&d_full[pb]);
         }
         __syncwarp();
+        if (++s == ST) s = 0;
+      }
+      if (++pb == C::NPB) pb = 0;
+    }
+    if (lane == 0) {
+      umma_commit(drain);
+      mbar_wait_plain(drain, 0, lim);
+    }
+  } else if (warp == kSchedWarp) {
+    // ---------------------------------------------------------------- MMA scheduler
+    int s = 0, pb = 0;
+    uint32_t ph = 0, ph_d = 0;
+    bool ok = true;
+    for (int it = blockIdx.x; it < total && ok; it += gridDim.x) {
+      for (int kb = 0; kb < nkb; ++kb) {
+        bool ready = kb != 0 || __all_sync(0xffffffffu, mbar_wait(&d_empty[pb], ph_d ^ 1u, abort_flag, lim));
+        ready = ready && __all_sync(0xffffffffu, mbar_wait(&full[s], ph, abort_flag, lim)) &&
+                __all_sync(0xffffffffu, mbar_wait(&sf_full[s], ph, abort_flag, lim));
+        if (!(ok = bar_red_and(kMmaBarrier, 64, ready))) break;
         if (++s == ST) {
           s = 0;
           ph ^= 1u;
@@ -246,10 +268,6 @@ __global__ void __launch_bounds__(kThreads, 1)
         pb = 0;
         ph_d ^= 1u;
       }
-    }
-    if (lane == 0) {
-      umma_commit(drain);
-      mbar_wait_plain(drain, 0, lim);
     }
   } else if (warp >= kScaleWarp0 && warp < kEpiWarp0) {
     // ---------------------------------------------------------------- scale warps
