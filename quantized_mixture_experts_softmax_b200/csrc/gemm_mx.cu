@@ -68,8 +68,10 @@ struct Cfg {
   static constexpr int ST = (232448 - 1024 - 4 * 1025 - 512) / STAGE;
   static_assert(ST >= 3, "pipeline depth");
   static constexpr int P_COLS = NA * NMAX;       // one accumulator tile: [matrix][NMAX] columns
-  static constexpr int NPB = 2;                  // accumulator tiles
   static constexpr int SF_COLS = NA * 4 + 4;     // TMEM columns of one stage's scales
+  // accumulator tiles: two (the epilogue of one item overlaps the next item's MMAs) where they
+  // fit next to the scale blocks
+  static constexpr int NPB = 2 * P_COLS + ST * SF_COLS <= 512 ? 2 : 1;
   static constexpr int SF_BASE = NPB * P_COLS;
   static constexpr int USED = SF_BASE + ST * SF_COLS;
   static constexpr int TMEM_COLS = USED <= 32 ? 32 : USED <= 64 ? 64 : USED <= 128 ? 128 : USED <= 256 ? 256 : 512;
@@ -421,11 +423,19 @@ cudaError_t launch_t(const MxGemmProblem& pr, cudaStream_t s) {
 
 }  // namespace mx
 
+template <bool GATED, int NA>
+static cudaError_t launch_nmax(const MxGemmProblem& p, cudaStream_t s) {
+  switch (p.nmax) {
+    case 32: return mx::launch_t<GATED, 32, NA>(p, s);
+    case 112: return mx::launch_t<GATED, 112, NA>(p, s);
+  }
+  return cudaErrorInvalidValue;
+}
+
 cudaError_t launch_mx_gemm(const MxGemmProblem& p, cudaStream_t s) {
-  const bool two = !p.gated && p.rows_per_expert % 256 == 0;
-  if (p.gated) return p.nmax == 64 ? mx::launch_t<true, 64, 2>(p, s) : mx::launch_t<true, 32, 2>(p, s);
-  if (two) return p.nmax == 64 ? mx::launch_t<false, 64, 2>(p, s) : mx::launch_t<false, 32, 2>(p, s);
-  return p.nmax == 64 ? mx::launch_t<false, 64, 1>(p, s) : mx::launch_t<false, 32, 1>(p, s);
+  if (p.gated) return launch_nmax<true, 2>(p, s);
+  if (p.rows_per_expert % 256 == 0) return launch_nmax<false, 2>(p, s);
+  return launch_nmax<false, 1>(p, s);
 }
 
 }  // namespace moe

@@ -214,7 +214,7 @@ struct MxGemmProblem {
   void* out;
   int out_ld;
   uint8_t* h_sf;           // gated: [I/128, act_rows, 4] (the x_sf layout of the down GEMM's input)
-  int nmax;                // token rows per tile: 32 or 64 (the cap the schedule was built with)
+  int nmax;                // token rows per tile: 32 or 112 (the cap the schedule was built with)
 };
 cudaError_t launch_mx_gemm(const MxGemmProblem& p, cudaStream_t s);
 cudaError_t launch_permute_mx(const uint16_t* x, const int32_t* inv_pos, int T, int k, int H, uint8_t* x_perm,

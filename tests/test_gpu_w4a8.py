@@ -100,17 +100,19 @@ def _onehot_logits(assign, E, seed):
     return lg
 
 
-@pytest.mark.parametrize("counts", [[15, 16, 17, 1, 31, 32, 33, 0, 64, 65], [100, 3, 0, 129]])
+@pytest.mark.parametrize("counts", [[15, 16, 17, 1, 31, 32, 33, 0, 64, 65], [100, 3, 0, 129],
+                                    [111, 112, 113, 224, 225, 1, 97, 0]])
 def test_w4a8_expert_counts_at_tile_boundaries(counts):
-    """Token tiles of at most 32 rows (T <= 512), MMAs of 16-row multiples: counts around both."""
+    """Token tiles of at most 32 rows (T <= 512) or 112 (T > 512), MMAs of 16-row multiples:
+    counts around each."""
     assign = np.repeat(np.arange(len(counts)), counts)
     E = len(counts) + 2
     run_and_check(MXLayer(6, len(assign), 256, 128, E, 1, logits=_onehot_logits(assign, E, 6)),
                   what=f"counts {counts}")
 
 
-def test_w4a8_64_row_tiles():
-    """T > 512: token tiles of up to 64 rows, experts spanning several."""
+def test_w4a8_wide_row_tiles():
+    """T > 512: token tiles of up to 112 rows, experts spanning several."""
     T, E = 600, 4
     run_and_check(MXLayer(7, T, 128, 128, E, 2), what="T=600")
 
