@@ -25,10 +25,12 @@
 // grouped GEMMs, weights in the MMA's M slot (128 rows), tokens in N.  Warp roles (384 threads):
 //   warp 0      TMA producer: NA weight tiles (gate and up, or two adjacent down tiles), the
 //               token tile and the weight scales, one stage per 128 K;
-//   warp 1      TMEM allocator and MMA issuer: four K = 32 block-scaled MMAs per matrix and
-//               stage into one of two accumulator tiles; it never waits on an mbarrier (a
-//               thread with MMAs in flight would stall there until they drain) and is released
-//               stage by stage by
+//   warps 1, 3  MMA issuers (warp 1 also allocates TMEM): four K = 32 block-scaled MMAs per
+//               matrix and stage into one of two accumulator tiles; with token tiles of up to 64
+//               rows one warp per weight matrix (the MMAs' fixed cost per instruction bounds the
+//               decode GEMMs: 6% faster than one issuer), else warp 1 alone; they never wait on
+//               an mbarrier (a thread with MMAs in flight would stall there until they drain)
+//               and are released stage by stage by
 //   warp 2      the MMA scheduler, which waits for the stage's copies and scales (and, at an
 //               item's first stage, for a free accumulator tile);
 //   warps 4-7   scale warps, one per lane quarter: per stage, the weight scales from shared
@@ -49,6 +51,7 @@ constexpr int BM = 128;  // weight rows per tile (MMA M)
 constexpr int KB = 128;  // K per stage
 constexpr int kMmaWarp = 1;
 constexpr int kSchedWarp = 2;
+constexpr int kMmaWarp2 = 3;    // the second matrix's MMA issuer (NA = 2)
 constexpr int kMmaBarrier = 1;  // named barrier of the MMA and scheduler warps (0 is __syncthreads)
 constexpr int kScaleWarp0 = 4;
 constexpr int kEpiWarp0 = 8;
@@ -60,6 +63,7 @@ struct Cfg {
   static_assert(NMAX % 16 == 0 && NMAX <= 128, "token tile");
   static_assert(!GATED || NA_ == 2, "gate and up tiles");
   static constexpr int NA = NA_;
+  static constexpr int NI = NA == 2 && NMAX <= 64 ? 2 : 1;  // MMA issuer warps
   static constexpr int W_TILE = BM * KB;   // unpacked E2M1 bytes in shared memory
   static constexpr int W_TX = BM * KB / 2;  // bytes the TMA reads (packed) and counts
   static constexpr int B_TILE = NMAX * KB;
@@ -151,14 +155,14 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (threadIdx.x == 0) {
     for (int i = 0; i < ST; ++i) {
       mbar_init(&full[i], 1);
-      mbar_init(&empty[i], 1);
+      mbar_init(&empty[i], C::NI);  // one commit per MMA issuer
       mbar_init(&sf_full[i], 4);
     }
     for (int i = 0; i < C::NPB; ++i) {
-      mbar_init(&d_full[i], 1);
+      mbar_init(&d_full[i], C::NI);
       mbar_init(&d_empty[i], 4);
     }
-    mbar_init(drain, 1);
+    mbar_init(drain, C::NI);
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -178,6 +182,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   const uint32_t tmem_base = *tmem_slot;
   const int total = p.m_tiles * sprefix[p.E];
   const int nkb = p.K / KB;
+  constexpr int kMmaThreads = 32 * (1 + C::NI);  // the scheduler and the MMA issuers
 
   if (warp == 0) {
     // ---------------------------------------------------------------- producer
@@ -212,31 +217,34 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       for (int i = max(0, issued - ST); i < issued; ++i) mbar_wait_plain(&full[i % ST], (i / ST) & 1, lim);
     }
-  } else if (warp == kMmaWarp) {
-    // ---------------------------------------------------------------- MMA issuer
-    // Released stage by stage by the scheduler warp; identical loop bounds on both sides.
+  } else if (warp == kMmaWarp || (C::NI == 2 && warp == kMmaWarp2)) {
+    // ---------------------------------------------------------------- MMA issuers
+    // Released stage by stage by the scheduler warp; identical loop bounds on all sides.  With
+    // one issuer, warp 1 issues matrix 0 and then matrix 1 per K step; with two, its own only.
+    const int mat = warp == kMmaWarp ? 0 : 1;
     int s = 0, pb = 0;
     bool ok = true;
     for (int it = blockIdx.x; it < total && ok; it += gridDim.x) {
       const Item I = decode_item(it, sprefix, p);
-      const uint32_t d = tmem_base + (uint32_t)(pb * C::P_COLS);
+      const uint32_t d = tmem_base + (uint32_t)(pb * C::P_COLS + mat * NMAX);  // this warp's first matrix
       for (int kb = 0; kb < nkb; ++kb) {
-        if (!(ok = bar_red_and(kMmaBarrier, 64, true))) break;
+        if (!(ok = bar_red_and(kMmaBarrier, kMmaThreads, true))) break;
         if (lane == 0) {
           tc_fence_after();
           const uint8_t* st = smem + s * C::STAGE;
-          const uint64_t a0 = sw128_kmajor_desc(smem_u32(st));
-          const uint64_t a1 = sw128_kmajor_desc(smem_u32(st + (NA - 1) * C::W_TILE));
+          const uint64_t a = sw128_kmajor_desc(smem_u32(st + mat * C::W_TILE));
+          const uint64_t a2 = sw128_kmajor_desc(smem_u32(st + (NA - 1) * C::W_TILE));
           const uint64_t b = sw128_kmajor_desc(smem_u32(st + NA * C::W_TILE));
           const uint32_t sfb = tmem_base + (uint32_t)(C::SF_BASE + s * C::SF_COLS + NA * 4);
-          const uint32_t sfa0 = tmem_base + (uint32_t)(C::SF_BASE + s * C::SF_COLS);
+          const uint32_t sfa = tmem_base + (uint32_t)(C::SF_BASE + s * C::SF_COLS + 4 * mat);
 #pragma unroll
           for (int kk = 0; kk < KB / 32; ++kk) {  // K = 32 codes = 32 bytes of a swizzled row per MMA
             const uint32_t idesc = make_idesc_mx(BM, I.nmma, (uint32_t)kk);
             const uint32_t id = (uint32_t)kk << 30;
             const uint32_t acc = (kb | kk) != 0;
-            umma_mx(d, a0 + 2 * kk, b + 2 * kk, idesc, acc, sfa0 | id, sfb | id);
-            if (NA == 2) umma_mx(d + NMAX, a1 + 2 * kk, b + 2 * kk, idesc, acc, (sfa0 + 4) | id, sfb | id);
+            umma_mx(d, a + 2 * kk, b + 2 * kk, idesc, acc, sfa | id, sfb | id);
+            if (C::NI == 1 && NA == 2)
+              umma_mx(d + NMAX, a2 + 2 * kk, b + 2 * kk, idesc, acc, (sfa + 4) | id, sfb | id);
           }
           umma_commit(&empty[s]);
           if (kb == nkb - 1) umma_commit(&d_full[pb]);
@@ -260,7 +268,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         bool ready = kb != 0 || __all_sync(0xffffffffu, mbar_wait(&d_empty[pb], ph_d ^ 1u, abort_flag, lim));
         ready = ready && __all_sync(0xffffffffu, mbar_wait(&full[s], ph, abort_flag, lim)) &&
                 __all_sync(0xffffffffu, mbar_wait(&sf_full[s], ph, abort_flag, lim));
-        if (!(ok = bar_red_and(kMmaBarrier, 64, ready))) break;
+        if (!(ok = bar_red_and(kMmaBarrier, kMmaThreads, ready))) break;
         if (++s == ST) {
           s = 0;
           ph ^= 1u;

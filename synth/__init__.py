@@ -150,6 +150,7 @@ def w4a16_weights(seed: int, H: int, I: int, experts) -> dict:
     w2_s = np.empty((n, H, I // 32), np.uint16)
     lo, hi = W4_SCALE_RANGE
     for i, e in enumerate(experts):
+        e = int(e)  # a numpy int32 id would overflow the flat offset
         fill_u32(seed, TID["w13_q"], e * w13_q[0].size, w13_q[i])
         fill_uniform_bf16(seed, TID["w13_s"], e * w13_s[0].size, w13_s[i], lo, hi)
         fill_u32(seed, TID["w2_q"], e * w2_q[0].size, w2_q[i])
@@ -166,6 +167,7 @@ def fp8_weights(seed: int, H: int, I: int, experts) -> dict:
     w2_s = np.empty((n, H // 128, I // 128), np.float32)
     lo, hi = FP8_SCALE_RANGE
     for i, e in enumerate(experts):
+        e = int(e)  # a numpy int32 id would overflow the flat offset
         fill_normal_e4m3(seed, TID["w13_8"], e * w13[0].size, w13[i])
         fill_uniform_f32(seed, TID["w13_8s"], e * w13_s[0].size, w13_s[i], lo, hi)
         fill_normal_e4m3(seed, TID["w2_8"], e * w2[0].size, w2[i])
@@ -192,6 +194,7 @@ def mxfp4_weights(seed: int, H: int, I: int, experts) -> dict:
     w2 = np.empty((n, H, I // 2), np.uint8)
     w2_sf = np.empty((n, I // 128, H, 4), np.uint8)
     for i, e in enumerate(experts):
+        e = int(e)  # a numpy int32 id would overflow the flat offset
         fill_u32(seed, TID["w13_mx"], e * w13[0].size // 4, w13[i].view(np.uint32))
         _mx_scales(seed, TID["w13_mxs"], e * w13_sf[0].size, w13_sf[i])
         fill_u32(seed, TID["w2_mx"], e * w2[0].size // 4, w2[i].view(np.uint32))

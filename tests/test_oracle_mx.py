@@ -181,3 +181,12 @@ def test_w4a8_weights_slice_by_expert():
     for key in full:
         assert np.array_equal(part[key][0], full[key][4]) and np.array_equal(part[key][1], full[key][1])
     assert set(np.unique(full["w13_sf"])) <= set(synth.MX_SCALE_CODES)
+
+
+def test_generator_expert_ids_as_numpy_int32():
+    """Expert ids that come from numpy (np.unique of routing ids) give the same slices as
+    Python ints, for experts whose flat offset exceeds 2^31."""
+    for gen, H, I in ((synth.mxfp4_weights, 7168, 2048), (synth.w4a16_weights, 7168, 2048)):
+        a = gen(0, H, I, np.array([383], np.int32))
+        b = gen(0, H, I, [383])
+        assert all(np.array_equal(a[k], b[k]) for k in a)
