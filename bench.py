@@ -9,6 +9,7 @@ One JSON line on stdout (rank 0).  Workloads (seeded synthetic inputs):
   fp8_t{1,16,64,512,4096}   the block-FP8 layer, 256 experts, top-8
   w4a8_t64, w4a8_t8192      the W4A8 layer (MXFP4 weights, FP8 activations in 32-groups) on the
                             decode / prefill shapes and routing of the W4A16 model
+  w4a8_t{1,16,512,4096}     the same layer at other token counts (N(0,1) routing)
   gemm_m{M}_k{K}_n{N}       the single-expert grouped GEMM sweep (no activation)
 The layer models' experts (9.5 GB of INT4 weights + bf16 scales for W4A16) stay resident in HBM;
 each step streams the active experts' weights (about 7 GB for decode), far more than the
@@ -47,6 +48,8 @@ FP8_MODEL = dict(H=7168, I=2048, E=256, k=8)
 # W4A8 layer: the W4A16 model's shapes and routing (384 experts, top-8), MXFP4 weights
 WORKLOADS["w4a8_t64"] = dict(kind="w4a8", T=64, zipf=0.0, steps=400, warmup=20)
 WORKLOADS["w4a8_t8192"] = dict(kind="w4a8", T=8192, zipf=1.1, steps=40, warmup=5)
+for _t in (1, 16, 512, 4096):  # the token-count sweep of the same layer (N(0,1) routing)
+    WORKLOADS[f"w4a8_t{_t}"] = dict(kind="w4a8", T=_t, zipf=0.0, steps=200 if _t <= 512 else 60, warmup=10)
 # block-FP8 benchmark model: expert e holds the generated weights of expert e mod FP8_DISTINCT (each
 # expert in its own memory); generating 11.3 GB of normal e4m3 values on the host takes minutes
 FP8_DISTINCT = 16
