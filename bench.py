@@ -313,8 +313,9 @@ def gemm_config(M: int, K: int, N: int) -> dict:
 def run_gemm(args, world, rank):
     """The single-expert W4A16 GEMM sweep through moe_w4a16_gemm.  Small operands fit in L2, so
     a 512 MB buffer is read between steps (a read leaves no dirty lines to write back during the
-    next step) and the step time is the sum of the library's own kernels (CUDA events around
-    each launch), the flush excluded."""
+    next step).  The step time is the call's device time: CUDA events just before and after the
+    call, the flush excluded, averaged over the steps.  A second pass with the library's per-launch
+    events (which keep consecutive kernels from overlapping) gives the per-kernel breakdown."""
     import torch
     import quantized_mixture_experts_softmax_b200 as moe
     import synth
@@ -340,19 +341,27 @@ def run_gemm(args, world, rank):
         step()
     torch.cuda.synchronize()
     assert moe.moe_get_device_status() == 0
+    stream = torch.cuda.current_stream()
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(steps)]
     with ClockSampler(torch.cuda.current_device()) as clk:
-        moe.moe_timing_enable(True)
-        moe.moe_timing_read()
         barrier(world)
-        for _ in range(steps):
+        for i in range(steps):
             flush.sum()
+            ev[i][0].record(stream)
             step()
+            ev[i][1].record(stream)
         torch.cuda.synchronize()
         barrier(world)
-        moe.moe_timing_enable(False)
+    ms_step = max_over_ranks(sum(a.elapsed_time(b) for a, b in ev) / steps, world)
+    # per-kernel breakdown (events around every launch)
+    moe.moe_timing_enable(True)
+    moe.moe_timing_read()
+    for _ in range(steps):
+        flush.sum()
+        step()
+    moe.moe_timing_enable(False)
     kern = moe.moe_timing_read()
     assert moe.moe_get_device_status() == 0
-    ms_step = max_over_ranks(sum(v[0] for v in kern.values()) / steps, world)
     launches = sum(n for (_, n) in kern.values())
     peaks = load_peaks()
     bytes_ = K * N // 2 + (K // 32) * N * 2 + M * K * 2 + M * N * 2

@@ -574,11 +574,10 @@ moe_status_t moe_w4a16_gemm(const void* a, int a_is_bf16, const int32_t* w_q, co
   if (moe_status_t st = check_device()) return st;
   const GemmWs w = carve_gemm(ws, M, K, N, E);
   const int nmax = pick_nmax(M);
-  cudaError_t e = launch_sched_from_offsets(expert_offsets, E, M, nmax, w.row_count, w.tile_prefix, w.chunk, stream);
   const TileSched sched{expert_offsets, w.row_count, w.tile_prefix, w.chunk};
   if (use_i8(M)) {
-    if (e == cudaSuccess)
-      e = launch_planes(static_cast<const uint16_t*>(a), a_is_bf16, nullptr, M, 1, K, w.aq.x, w.aq.meta, stream);
+    cudaError_t e = launch_sched_planes(expert_offsets, E, nmax, w.row_count, w.tile_prefix, w.chunk,
+                                        static_cast<const uint16_t*>(a), a_is_bf16, M, K, w.aq.x, w.aq.meta, stream);
     const int sp = gemm_splits(M, K, N);
     if (e == cudaSuccess) {
       W4I8Problem g{w_q, static_cast<const uint16_t*>(w_s), w.aq.x, w.aq.meta, M, K, E, N, false, 0, sched,
@@ -588,6 +587,7 @@ moe_status_t moe_w4a16_gemm(const void* a, int a_is_bf16, const int32_t* w_q, co
     if (e == cudaSuccess && sp > 1) e = launch_reduce_splits(w.part, sp, M, N, expert_offsets, w.row_count, E, out, out_fp32, stream);
     return e == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
   }
+  cudaError_t e = launch_sched_from_offsets(expert_offsets, E, M, nmax, w.row_count, w.tile_prefix, w.chunk, stream);
   if (e == cudaSuccess)
     e = launch_convert_rows(static_cast<const uint16_t*>(a), a_is_bf16, M, K, w.a, w.a_exp, stream);
   const int sp = gemm_splits(M, K, N);

@@ -217,6 +217,10 @@ struct MxGemmProblem {
   int nmax;                // token rows per tile: 32 or 112 (the cap the schedule was built with)
 };
 cudaError_t launch_mx_gemm(const MxGemmProblem& p, cudaStream_t s);
+// the single grouped GEMM's schedule from caller offsets and its rows' activation planes, one launch
+cudaError_t launch_sched_planes(const int32_t* offsets, int E, int nmax, int32_t* row_count, int32_t* tile_prefix,
+                                int32_t* chunk, const uint16_t* a, int a_is_bf16, int M, int K, int8_t* planes,
+                                int32_t* meta, cudaStream_t s);
 cudaError_t launch_permute_mx(const uint16_t* x, const int32_t* inv_pos, int T, int k, int H, uint8_t* x_perm,
                               uint32_t* x_sf, int P, cudaStream_t s);
 

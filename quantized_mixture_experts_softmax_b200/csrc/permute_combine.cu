@@ -497,6 +497,41 @@ cudaError_t launch_planes(const uint16_t* a, int a_is_bf16, const int32_t* inv_p
   return cudaGetLastError();
 }
 
+// The single grouped GEMM's int8 path: its tile schedule (block 0, a thread per expert) and the
+// activation planes of its M rows (the other blocks, 16 threads per (row, 128-K block)) in one
+// launch - the two are independent, and a launch saved is most of a small GEMM's time.
+__global__ void __launch_bounds__(1024) sched_planes_kernel(const int32_t* __restrict__ offsets, int E, int nmax,
+                                                            int32_t* __restrict__ row_count,
+                                                            int32_t* __restrict__ tile_prefix,
+                                                            int32_t* __restrict__ chunk, const uint4* __restrict__ a,
+                                                            int a_is_bf16, int M, int K, uint2* __restrict__ planes,
+                                                            int32_t* __restrict__ meta) {
+  grid_dependency_sync();  // see common.cuh
+  if (blockIdx.x == 0) {
+    sched_from_offsets_block(offsets, E, M, nmax, row_count, tile_prefix, chunk);
+    return;
+  }
+  const int nblk = K / 128;
+  const size_t unit = ((blockIdx.x - 1) * (size_t)blockDim.x + threadIdx.x) >> 4;  // (row, block)
+  const int i = threadIdx.x & 15;
+  const bool live = unit < (size_t)M * nblk;
+  const int p = live ? (int)(unit / nblk) : 0;
+  const int blk = live ? (int)(unit % nblk) : 0;
+  planes_unit(a, a_is_bf16, live ? p : -1, p, blk, i, K, planes, meta);
+}
+
+cudaError_t launch_sched_planes(const int32_t* offsets, int E, int nmax, int32_t* row_count, int32_t* tile_prefix,
+                                int32_t* chunk, const uint16_t* a, int a_is_bf16, int M, int K, int8_t* planes,
+                                int32_t* meta, cudaStream_t s) {
+  const size_t threads = (size_t)M * (K / 128) * 16;
+  timing_before("sched_planes", s);
+  (void)launch_kernel(sched_planes_kernel, dim3(1 + (unsigned)((threads + 1023) / 1024)), dim3(1024), 0, s, offsets,
+                      E, nmax, row_count, tile_prefix, chunk, reinterpret_cast<const uint4*>(a), a_is_bf16, M, K,
+                      reinterpret_cast<uint2*>(planes), meta);
+  timing_after("sched_planes", s);
+  return cudaGetLastError();
+}
+
 // the rows of a list of expert runs: list row j < row_prefix[E] is row j - row_prefix[e] of
 // expert e (row_prefix[e] <= j < row_prefix[e+1]), i.e. sorted row offsets[e] + j - row_prefix[e],
 // whose pair is sorted_ids of that row; the grid covers an upper bound of the list length

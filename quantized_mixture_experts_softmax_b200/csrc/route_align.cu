@@ -278,11 +278,11 @@ cudaError_t launch_align(const int32_t* ids, int T, int k, int E, int align, int
 }
 
 // ------------------------------------------------------------------ scheduler from caller offsets
-__global__ void __launch_bounds__(1024) sched_from_offsets_kernel(const int32_t* __restrict__ offsets, int E, int M,
-                                                                  int nmax, int32_t* __restrict__ row_count,
-                                                                  int32_t* __restrict__ tile_prefix,
-                                                                  int32_t* __restrict__ chunk) {
-  grid_dependency_sync();  // see common.cuh
+// One block of 1024 threads (one per expert, E <= 1024).
+__device__ __forceinline__ void sched_from_offsets_block(const int32_t* __restrict__ offsets, int E, int M, int nmax,
+                                                         int32_t* __restrict__ row_count,
+                                                         int32_t* __restrict__ tile_prefix,
+                                                         int32_t* __restrict__ chunk) {
   __shared__ int warp_tot[32];
   __shared__ int total;
   const int e = threadIdx.x;
@@ -304,6 +304,14 @@ __global__ void __launch_bounds__(1024) sched_from_offsets_kernel(const int32_t*
     chunk[e] = ch;
   }
   if (e == 0) tile_prefix[E] = total;
+}
+
+__global__ void __launch_bounds__(1024) sched_from_offsets_kernel(const int32_t* __restrict__ offsets, int E, int M,
+                                                                  int nmax, int32_t* __restrict__ row_count,
+                                                                  int32_t* __restrict__ tile_prefix,
+                                                                  int32_t* __restrict__ chunk) {
+  grid_dependency_sync();  // see common.cuh
+  sched_from_offsets_block(offsets, E, M, nmax, row_count, tile_prefix, chunk);
 }
 
 cudaError_t launch_sched_from_offsets(const int32_t* offsets, int E, int M, int nmax, int32_t* row_count,
