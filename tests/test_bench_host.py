@@ -70,12 +70,25 @@ def test_weight_bytes_per_expert_match_the_stored_layout():
     assert W["w13_q"].dtype == np.int32 and W["w13_q"].shape == (1, 2 * I, H // 8)
 
 
+def test_w4a8_weight_bytes_per_expert_match_the_stored_layout():
+    H, I = bench.MODEL["H"], bench.MODEL["I"]
+    W = synth.mxfp4_weights(0, H, I, [0])
+    assert W["w13"].nbytes + W["w13_sf"].nbytes == bench.W13_MX_BYTES_PER_EXPERT
+    assert W["w2"].nbytes + W["w2_sf"].nbytes == bench.W2_MX_BYTES_PER_EXPERT
+    # MXFP4: two E2M1 codes per byte, one 1-byte E8M0 scale per 32 weights
+    assert bench.W13_MX_BYTES_PER_EXPERT == 2 * I * H // 2 + 2 * I * H // 32
+    assert W["w13"].shape == (1, 2 * I, H // 2) and W["w13_sf"].shape == (1, H // 128, 2 * I, 4)
+
+
 def test_workloads_cover_the_layer_configurations():
     w = bench.WORKLOADS
     assert w["decode"]["T"] == 64 and w["prefill"]["T"] == 8192
     assert bench.MODEL == dict(H=7168, I=2048, E=384, k=8)
     assert bench.FP8_MODEL == dict(H=7168, I=2048, E=256, k=8)
     assert sorted(v["T"] for n, v in w.items() if n.startswith("fp8_")) == [1, 16, 64, 512, 4096]
+    # W4A8 on the decode and prefill configurations (same model and routing) plus the T sweep
+    assert w["w4a8_t64"] == dict(w["decode"], kind="w4a8") and w["w4a8_t8192"] == dict(w["prefill"], kind="w4a8")
+    assert {"w4a8_t64", "w4a8_t8192"} <= set(bench.DEFAULT_EXTRAS)
     for v in w.values():
         assert v["warmup"] >= 3  # the timing rule's minimum
 
