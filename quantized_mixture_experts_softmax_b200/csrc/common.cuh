@@ -317,12 +317,13 @@ __device__ __forceinline__ void bulk_load(void* dst, const void* src, uint32_t b
 // Microscaling exponent of an FP8 E4M3 group: the smallest X in [-127, 127] with
 // amax <= 448 * 2^X, from the bits of amax (>= 0).  448 = 1.75 * 2^8, so with amax = 1.f * 2^e
 // X = e - 8 when the fraction f is at most 0.75 (bits 0x600000) and e - 7 above; zero and
-// subnormal amax (< 2^-126 <= 448 * 2^-127) take -127.
-__device__ __forceinline__ int mx_exponent(uint32_t amax_bits) {
+// subnormal amax (< 2^-126 <= 448 * 2^-127) take -127.  (Host-callable for its CPU test; an inf
+// or NaN amax gives 120 or 121, and the callers flag such a group.)
+__host__ __device__ __forceinline__ int mx_exponent(uint32_t amax_bits) {
   const int eb = (int)(amax_bits >> 23);
   if (eb == 0) return -127;
   const int X = eb - 127 - 8 + ((amax_bits & 0x7FFFFFu) > 0x600000u ? 1 : 0);
-  return max(-127, min(127, X));
+  return X < -127 ? -127 : (X > 127 ? 127 : X);
 }
 // 2^-X as a float for X in [-127, 126] (exact)
 __device__ __forceinline__ float exp2_neg(int X) { return __int_as_float((127 - X) << 23); }
