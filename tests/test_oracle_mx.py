@@ -190,3 +190,17 @@ def test_generator_expert_ids_as_numpy_int32():
         a = gen(0, H, I, np.array([383], np.int32))
         b = gen(0, H, I, [383])
         assert all(np.array_equal(a[k], b[k]) for k in a)
+
+
+def test_w4a8_token_permutation_and_subsets():
+    """Each token is computed on its own: permuting the tokens (rows of x, ids and weights)
+    permutes the output rows bit for bit, and a token subset reproduces those rows exactly."""
+    T, H, I, E, k = 7, 256, 128, 5, 2
+    x, ids, w, W = _layer_inputs(4, T, H, I, E, k)
+    full = oracle.w4a8_tokens(x, ids, w, W["w13"], W["w13_sf"], W["w2"], W["w2_sf"])
+    perm = np.random.default_rng(1).permutation(T)
+    permuted = oracle.w4a8_tokens(x[perm], ids[perm], w[perm], W["w13"], W["w13_sf"], W["w2"], W["w2_sf"])
+    assert np.array_equal(permuted, full[perm])
+    sub = np.array([5, 0, 3], np.int32)
+    part = oracle.w4a8_tokens(x, ids, w, W["w13"], W["w13_sf"], W["w2"], W["w2_sf"], tokens=sub)
+    assert np.array_equal(part, full[sub])
